@@ -1,0 +1,335 @@
+// Sparse scaled-dot-product attention over the selected keys, one index set per token shared by
+// every GQA KV group:
+//   out[t,h,:] = sum_{s in S_t} softmax_s(scale * q[t,h,:] . k[s,g,:]) v[s,g,:],  g = h / (Hq/Hkv)
+// (page "从“看”到“想”多模态大模型推理能力的瓶颈与突破", wmrh.cn, section 2, step 3: standard
+// scaled dot-product attention on the small selected candidate set; page "快手开源大模型
+// Keye-VL-2.0：一个能“看懂“两小时视频AI", gsyq.cn, section 一: GQA adaptation of DSA).
+//
+// The work is a gather: per token, 2048 keys x Hkv x 128 x (K and V) x 2 bytes = 4 MiB at the
+// 32/4/128 shape against 32 x 128 x 2048 x 4 flop, i.e. 8 flop per byte, far below the ridge
+// of the tensor cores.  The kernel therefore spends its effort on the memory side:
+//   - one CTA per (token, key split); each selected key's K and V rows for all KV heads are
+//     one contiguous Hkv*256-byte span, gathered with coalesced 16-byte cp.async copies into a
+//     3-stage shared-memory ring (rows padded by 16 bytes: conflict-free ldmatrix);
+//   - 2 warps per KV group; a warp owns its group's G query heads (GQA head packing: the
+//     K/V tile it reads from shared memory serves all G heads at once);
+//   - S^T[keys x heads] = K . Q^T and O^T += V^T . P^T on warp-level bf16 MMAs
+//     (m16n8k16, keys or head-dimension rows as M, 8 heads as N), so no MMA lane is wasted on
+//     the small head count; P^T goes from the accumulator layout to the operand layout with
+//     movmatrix; online softmax in fp32 (exp2 domain);
+//   - masked and padding slots (index -1) are zero-filled copies with logit -inf.
+// With nsplit > 1 every CTA writes unnormalised partial results (O, running max, running sum)
+// for its slice of the index list; attn_combine_kernel merges them.
+#pragma once
+
+#include "ptx.cuh"
+
+namespace dsa {
+
+constexpr int kAttnD = 128;
+constexpr int kAttnStages = 3;
+constexpr int kAttnWPG = 2;  // warps per KV group
+
+struct AttnParams {
+    const __nv_bfloat16* q;   // [T, Hq, D]
+    const __nv_bfloat16* k;   // [*, Hkv, D] per batch entry
+    const __nv_bfloat16* v;
+    long long kv_bstride;     // elements between batch entries of k/v (decode); 0 for prefill
+    const int* idx;           // [T, topk]
+    int topk;
+    int T;                    // tokens in this launch
+    long long q_pos0;         // prefill: token t sees min(topk, q_pos0 + t + 1) keys
+    const int* ctx_len;       // decode: token t sees min(topk, ctx_len[t] + 1) keys, batch entry t
+    long long n_keys;         // valid key rows per batch entry (bounds check on indices)
+    int Hq, Hkv;
+    float scale_log2;         // scale * log2(e)
+    __nv_bfloat16* out;       // [T, Hq, D]
+    float* lse;               // [T, Hq] natural-log LSE, may be null
+    int nsplit;               // key splits per token
+    float* part;              // nsplit > 1: [T, nsplit, Hq, D + 2]
+};
+
+__host__ __device__ constexpr int attn_keys_per_stage(int hkv) { return 128 / hkv; }
+__host__ __device__ constexpr int attn_row_bytes(int hkv) { return hkv * kAttnD * 2 + 16; }
+__host__ __device__ constexpr int attn_smem_bytes(int hkv) {
+    return kAttnStages * attn_keys_per_stage(hkv) * attn_row_bytes(hkv) * 2;
+}
+
+// NT: n-tiles of 8 query heads per KV group (G <= 8 * NT).
+template <int NT>
+__global__ void __launch_bounds__(256) sparse_attn_kernel(const AttnParams P) {
+    extern __shared__ __align__(1024) uint8_t smem[];
+    const int Hkv = P.Hkv, G = P.Hq / P.Hkv;
+    const int KS = attn_keys_per_stage(Hkv);        // keys per stage (all groups)
+    const int RB = attn_row_bytes(Hkv);             // padded row bytes (K or V of one key)
+    const int STAGE = KS * RB * 2;                  // K rows then V rows
+    const int nthreads = blockDim.x;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int grp = warp / kAttnWPG, wsub = warp % kAttnWPG;
+
+    const int t = blockIdx.x / P.nsplit;
+    const int split = blockIdx.x % P.nsplit;
+    long long n_ll;
+    const __nv_bfloat16 *kb = P.k, *vb = P.v;
+    if (P.ctx_len) {
+        n_ll = (long long)P.ctx_len[t] + 1;
+        n_ll = n_ll < 1 ? 1 : (n_ll > P.n_keys ? P.n_keys : n_ll);
+        kb += (long long)t * P.kv_bstride;
+        vb += (long long)t * P.kv_bstride;
+    } else {
+        n_ll = P.q_pos0 + t + 1;
+    }
+    const int n_sel = (int)min((long long)P.topk, n_ll);
+    const int per_split = (n_sel + P.nsplit - 1) / P.nsplit;
+    const int p_begin = split * per_split;
+    const int p_end = min(n_sel, p_begin + per_split);
+    const int* idx_row = P.idx + (long long)t * P.topk;
+    const int nsteps = p_end > p_begin ? (p_end - p_begin + KS - 1) / KS : 0;
+
+    // ---- Q^T fragments (B operand, K = head dim, N = 8 heads): head lane/4, dims 2*(lane%4)+{0,1}(+8)
+    uint32_t qf[NT][8][2];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+        const int hl = nt * 8 + (lane >> 2);
+        const bool hv = hl < G;
+        const __nv_bfloat16* qrow = P.q + ((long long)t * P.Hq + grp * G + (hv ? hl : 0)) * kAttnD;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+            const int d = kk * 16 + 2 * (lane & 3);
+            qf[nt][kk][0] = hv ? *reinterpret_cast<const uint32_t*>(qrow + d) : 0u;
+            qf[nt][kk][1] = hv ? *reinterpret_cast<const uint32_t*>(qrow + d + 8) : 0u;
+        }
+    }
+
+    // ---- async gather of one stage: KS keys x (all KV heads) of K and V
+    const int chunks_per_row = Hkv * kAttnD * 2 / 16;
+    auto load_stage = [&](int step, int buf) {
+        uint8_t* sk = smem + buf * STAGE;
+        uint8_t* sv = sk + KS * RB;
+        const int p0 = p_begin + step * KS;
+        for (int c = threadIdx.x; c < KS * chunks_per_row; c += nthreads) {
+            const int key = c / chunks_per_row, ch = c % chunks_per_row;
+            const int p = p0 + key;
+            int s = (p < p_end) ? idx_row[p] : -1;
+            bool ok = s >= 0 && s < P.n_keys;
+            const long long off = (ok ? (long long)s : 0) * (Hkv * kAttnD) + ch * 8;
+            cp_async_16(sk + key * RB + ch * 16, kb + off, ok);
+            cp_async_16(sv + key * RB + ch * 16, vb + off, ok);
+        }
+    };
+
+    float o[NT][8][4];  // O^T: [d-tile][4] per n-tile; rows = head dims, cols = heads
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int dt = 0; dt < 8; ++dt)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) o[nt][dt][i] = 0.f;
+    float m_run[NT][2], l_run[NT][2];  // per owned head (cols 2*(lane%4)+{0,1})
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) m_run[nt][0] = m_run[nt][1] = -INFINITY, l_run[nt][0] = l_run[nt][1] = 0.f;
+
+#pragma unroll
+    for (int s = 0; s < kAttnStages - 1; ++s) {
+        if (s < nsteps) load_stage(s, s);
+        cp_async_commit();
+    }
+
+    const int tiles_per_warp = KS / 16 / kAttnWPG;  // 16-key tiles this warp takes per stage
+    for (int step = 0; step < nsteps; ++step) {
+        cp_async_wait<kAttnStages - 2>();
+        __syncthreads();
+        if (step + kAttnStages - 1 < nsteps) load_stage(step + kAttnStages - 1, (step + kAttnStages - 1) % kAttnStages);
+        cp_async_commit();
+
+        const uint8_t* sk = smem + (step % kAttnStages) * STAGE;
+        const uint8_t* sv = sk + KS * RB;
+        for (int tt = 0; tt < tiles_per_warp; ++tt) {
+            const int kt = wsub * tiles_per_warp + tt;       // 16-key tile inside the stage
+            const int pbase = p_begin + step * KS + kt * 16;  // index-list slot of its first key
+            // S^T = K Q^T : 16 keys x 8 heads per n-tile
+            float sacc[NT][4];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) sacc[nt][0] = sacc[nt][1] = sacc[nt][2] = sacc[nt][3] = 0.f;
+            {
+                const int mi = lane >> 3, ri = lane & 7;
+                const uint8_t* arow = sk + (kt * 16 + (mi & 1) * 8 + ri) * RB + (grp * kAttnD + (mi >> 1) * 8) * 2;
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    uint32_t a[4];
+                    ldmatrix_x4(a, arow + kk * 32);
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) mma_16816(sacc[nt], a, qf[nt][kk][0], qf[nt][kk][1]);
+                }
+            }
+            // mask slots beyond this CTA's range; rows: key lane/4 (c0,c1) and lane/4+8 (c2,c3)
+            const bool v0 = pbase + (lane >> 2) < p_end, v1 = pbase + (lane >> 2) + 8 < p_end;
+            uint32_t pb[NT][2];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                float z[4];
+                z[0] = v0 ? sacc[nt][0] * P.scale_log2 : -INFINITY;
+                z[1] = v0 ? sacc[nt][1] * P.scale_log2 : -INFINITY;
+                z[2] = v1 ? sacc[nt][2] * P.scale_log2 : -INFINITY;
+                z[3] = v1 ? sacc[nt][3] * P.scale_log2 : -INFINITY;
+                float mx[2] = {fmaxf(z[0], z[2]), fmaxf(z[1], z[3])};
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    mx[j] = fmaxf(mx[j], __shfl_xor_sync(0xffffffffu, mx[j], 4));
+                    mx[j] = fmaxf(mx[j], __shfl_xor_sync(0xffffffffu, mx[j], 8));
+                    mx[j] = fmaxf(mx[j], __shfl_xor_sync(0xffffffffu, mx[j], 16));
+                }
+                float alpha[2], base[2];
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    const float m_new = fmaxf(m_run[nt][j], mx[j]);
+                    base[j] = m_new == -INFINITY ? 0.f : m_new;
+                    alpha[j] = exp2f(m_run[nt][j] - base[j]);
+                    m_run[nt][j] = m_new;
+                }
+                const float p0 = exp2f(z[0] - base[0]), p1 = exp2f(z[1] - base[1]);
+                const float p2 = exp2f(z[2] - base[0]), p3 = exp2f(z[3] - base[1]);
+                l_run[nt][0] = l_run[nt][0] * alpha[0] + p0 + p2;
+                l_run[nt][1] = l_run[nt][1] * alpha[1] + p1 + p3;
+#pragma unroll
+                for (int dt = 0; dt < 8; ++dt) {
+                    o[nt][dt][0] *= alpha[0];
+                    o[nt][dt][1] *= alpha[1];
+                    o[nt][dt][2] *= alpha[0];
+                    o[nt][dt][3] *= alpha[1];
+                }
+                // P^T (keys x heads) -> B operand layout (keys as K, heads as N)
+                pb[nt][0] = movmatrix_trans(pack_bf16x2(p0, p1));
+                pb[nt][1] = movmatrix_trans(pack_bf16x2(p2, p3));
+            }
+            // O^T += V^T P^T : A = V^T (16 dims x 16 keys) via transposing ldmatrix
+            {
+                const int mi = lane >> 3, ri = lane & 7;
+                const uint8_t* vrow = sv + (kt * 16 + (mi >> 1) * 8 + ri) * RB + (grp * kAttnD + (mi & 1) * 8) * 2;
+#pragma unroll
+                for (int dt = 0; dt < 8; ++dt) {
+                    uint32_t a[4];
+                    ldmatrix_x4_trans(a, vrow + dt * 32);
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) mma_16816(o[nt][dt], a, pb[nt][0], pb[nt][1]);
+                }
+            }
+        }
+    }
+    cp_async_wait<0>();
+
+    // ---- finish: full row sums, merge the kAttnWPG warps of a group through shared memory
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            float l = l_run[nt][j];
+            l += __shfl_xor_sync(0xffffffffu, l, 4);
+            l += __shfl_xor_sync(0xffffffffu, l, 8);
+            l += __shfl_xor_sync(0xffffffffu, l, 16);
+            l_run[nt][j] = l;
+        }
+    __syncthreads();  // stage buffers are free now
+    // per warp: [NT][8][4] O values per lane + m, l per owned head
+    float* xch = reinterpret_cast<float*>(smem) + (size_t)warp * (NT * 36 * 32);
+    if (wsub != 0) {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+            for (int dt = 0; dt < 8; ++dt)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) xch[((nt * 36) + dt * 4 + i) * 32 + lane] = o[nt][dt][i];
+            xch[(nt * 36 + 32) * 32 + lane] = m_run[nt][0];
+            xch[(nt * 36 + 33) * 32 + lane] = m_run[nt][1];
+            xch[(nt * 36 + 34) * 32 + lane] = l_run[nt][0];
+            xch[(nt * 36 + 35) * 32 + lane] = l_run[nt][1];
+        }
+    }
+    __syncthreads();
+    if (wsub == 0) {
+#pragma unroll
+        for (int w2 = 1; w2 < kAttnWPG; ++w2) {
+            const float* x2 = reinterpret_cast<const float*>(smem) + (size_t)(warp + w2) * (NT * 36 * 32);
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                float a1[2], a2[2];
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    const float m2 = x2[(nt * 36 + 32 + j) * 32 + lane];
+                    const float l2 = x2[(nt * 36 + 34 + j) * 32 + lane];
+                    const float mn = fmaxf(m_run[nt][j], m2);
+                    const float bs = mn == -INFINITY ? 0.f : mn;
+                    a1[j] = exp2f(m_run[nt][j] - bs);
+                    a2[j] = exp2f(m2 - bs);
+                    l_run[nt][j] = l_run[nt][j] * a1[j] + l2 * a2[j];
+                    m_run[nt][j] = mn;
+                }
+#pragma unroll
+                for (int dt = 0; dt < 8; ++dt)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        o[nt][dt][i] = o[nt][dt][i] * a1[i & 1] + x2[((nt * 36) + dt * 4 + i) * 32 + lane] * a2[i & 1];
+            }
+        }
+        // write: fragment (dims dt*16 + lane/4 (+8), heads nt*8 + 2*(lane%4) + {0,1})
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const int hl = nt * 8 + 2 * (lane & 3) + j;
+                if (hl >= G) continue;
+                const int h = grp * G + hl;
+                if (P.nsplit == 1) {
+                    const float inv = l_run[nt][j] > 0.f ? 1.f / l_run[nt][j] : 0.f;
+                    __nv_bfloat16* orow = P.out + ((long long)t * P.Hq + h) * kAttnD;
+#pragma unroll
+                    for (int dt = 0; dt < 8; ++dt) {
+                        orow[dt * 16 + (lane >> 2)] = __float2bfloat16_rn(o[nt][dt][j] * inv);
+                        orow[dt * 16 + (lane >> 2) + 8] = __float2bfloat16_rn(o[nt][dt][2 + j] * inv);
+                    }
+                    if (P.lse && (lane >> 2) == 0)
+                        P.lse[(long long)t * P.Hq + h] =
+                            l_run[nt][j] > 0.f ? (m_run[nt][j] + log2f(l_run[nt][j])) * 0.69314718055994531f : -INFINITY;
+                } else {
+                    float* prow = P.part + (((long long)t * P.nsplit + split) * P.Hq + h) * (kAttnD + 2);
+#pragma unroll
+                    for (int dt = 0; dt < 8; ++dt) {
+                        prow[dt * 16 + (lane >> 2)] = o[nt][dt][j];
+                        prow[dt * 16 + (lane >> 2) + 8] = o[nt][dt][2 + j];
+                    }
+                    if ((lane >> 2) == 0) {
+                        prow[kAttnD] = m_run[nt][j];
+                        prow[kAttnD + 1] = l_run[nt][j];
+                    }
+                }
+            }
+        }
+    }
+}
+
+// Merge split partials: one warp per (token, head).
+__global__ void __launch_bounds__(128) attn_combine_kernel(const float* part, int T, int nsplit, int Hq,
+                                                           __nv_bfloat16* out, float* lse) {
+    const int wid = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (wid >= T * Hq) return;
+    const int t = wid / Hq, h = wid % Hq;
+    float mx = -INFINITY;
+    for (int s = 0; s < nsplit; ++s) mx = fmaxf(mx, part[(((long long)t * nsplit + s) * Hq + h) * (kAttnD + 2) + kAttnD]);
+    const float bs = mx == -INFINITY ? 0.f : mx;
+    float acc[4] = {0.f, 0.f, 0.f, 0.f}, l = 0.f;
+    for (int s = 0; s < nsplit; ++s) {
+        const float* pr = part + (((long long)t * nsplit + s) * Hq + h) * (kAttnD + 2);
+        const float a = exp2f(pr[kAttnD] - bs);
+        l += pr[kAttnD + 1] * a;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[i] += pr[lane * 4 + i] * a;
+    }
+    const float inv = l > 0.f ? 1.f / l : 0.f;
+    __nv_bfloat16* orow = out + ((long long)t * Hq + h) * kAttnD;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) orow[lane * 4 + i] = __float2bfloat16_rn(acc[i] * inv);
+    if (lse && lane == 0) lse[(long long)t * Hq + h] = l > 0.f ? (mx + log2f(l)) * 0.69314718055994531f : -INFINITY;
+}
+
+}  // namespace dsa

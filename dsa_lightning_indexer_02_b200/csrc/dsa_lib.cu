@@ -1,0 +1,608 @@
+// libdsa.so: the C ABI declared in include/dsa.h.  Host side: argument validation, workspace
+// carving, TMA descriptor encoding, launch configuration and the fused prefill/decode drivers.
+// Every computation of the path runs in the kernels of indexer.cuh, topk.cuh and attn.cuh.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "attn.cuh"
+#include "dsa.h"
+#include "indexer.cuh"
+#include "ptx.cuh"
+#include "topk.cuh"
+
+using namespace dsa;
+
+namespace {
+
+constexpr int kVersion = 10000;
+constexpr int kMaxTopk = 65536;
+constexpr int kMaxDecodeSplits = 16;
+constexpr int kDecodeIdxStages = 8;
+constexpr int kPrefillIdxStages = 4;
+
+// ------------------------------------------------------------------ launch accounting / profiling
+std::atomic<long long> g_launches{0};
+std::mutex g_prof_mu;
+bool g_prof_on = false;
+struct ProfRec {
+    int kind;
+    cudaEvent_t a, b;
+};
+std::vector<ProfRec> g_prof_recs;
+std::vector<cudaEvent_t> g_event_pool;
+
+cudaEvent_t pooled_event() {
+    if (!g_event_pool.empty()) {
+        cudaEvent_t e = g_event_pool.back();
+        g_event_pool.pop_back();
+        return e;
+    }
+    cudaEvent_t e = nullptr;
+    cudaEventCreate(&e);
+    return e;
+}
+
+struct LaunchScope {
+    int kind;
+    cudaStream_t s;
+    cudaEvent_t a = nullptr, b = nullptr;
+    LaunchScope(int kind_, cudaStream_t s_) : kind(kind_), s(s_) {
+        g_launches.fetch_add(1);
+        std::lock_guard<std::mutex> lk(g_prof_mu);
+        if (g_prof_on) {
+            a = pooled_event();
+            b = pooled_event();
+            cudaEventRecord(a, s);
+        }
+    }
+    ~LaunchScope() {
+        if (a) {
+            cudaEventRecord(b, s);
+            std::lock_guard<std::mutex> lk(g_prof_mu);
+            g_prof_recs.push_back({kind, a, b});
+        }
+    }
+};
+
+enum { K_INDEX = 0, K_TOPK = 1, K_ATTN = 2, K_COMBINE = 3, K_APPEND = 4, K_ADVANCE = 5, K_SELFTEST = 6 };
+
+dsa_status launch_status() {
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------ device properties
+int num_sms() {
+    static int n = 0;
+    if (n == 0) {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    }
+    return n;
+}
+
+// ------------------------------------------------------------------ TMA descriptors
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+// bf16 tensor [d2][d1][64] (rows of 128 bytes), box {64, box_rows, 1}, 128-byte swizzle.
+bool make_rows_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t batch, uint64_t batch_stride_bytes,
+                   uint32_t box_rows) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {64, rows, batch};
+    cuuint64_t strides[2] = {128, batch_stride_bytes};
+    cuuint32_t box[3] = {64, box_rows, 1};
+    cuuint32_t es[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+bool hi_supported_prefill(int HI) {
+    return HI == 1 || HI == 2 || HI == 4 || HI == 8 || HI == 16 || HI == 32 || HI == 64;
+}
+bool hi_supported_decode(int HI) { return HI == 16 || HI == 32 || HI == 64; }
+
+dsa_status check_attn_shape(int Hq, int Hkv, int D) {
+    if (Hq <= 0 || Hkv <= 0 || D <= 0) return DSA_ERR_INVALID_ARG;
+    if (D != kAttnD) return DSA_ERR_UNSUPPORTED;
+    if (!(Hkv == 1 || Hkv == 2 || Hkv == 4)) return DSA_ERR_UNSUPPORTED;
+    if (Hq % Hkv != 0 || Hq / Hkv > 16) return DSA_ERR_UNSUPPORTED;
+    return DSA_OK;
+}
+
+// ------------------------------------------------------------------ indexer launch
+template <int HI, int BN, int STAGES>
+dsa_status launch_indexer_t(const CUtensorMap& mq, const CUtensorMap& mk, const IndexerParams& P, int grid,
+                            cudaStream_t s) {
+    using C = IndexerCfg<HI, BN, STAGES>;
+    auto kern = indexer_kernel<HI, BN, STAGES>;
+    static bool attr_set = false;
+    if (!attr_set) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
+            return DSA_ERR_CUDA;
+        attr_set = true;
+    }
+    LaunchScope ls(K_INDEX, s);
+    kern<<<grid, C::THREADS, C::SMEM, s>>>(mq, mk, P);
+    return launch_status();
+}
+
+// Shared by dsa_index (P = 1) and the decode step (P = B, one query each).
+dsa_status run_indexer(const void* qI, const void* kI, const __nv_bfloat16* w, int P_, int Lq, int64_t q_pos0,
+                       const int* ctx_len, int64_t Lk, int HI, float* scores, int64_t ld, cudaStream_t s) {
+    const bool decode = ctx_len != nullptr;
+    const int BN = decode ? HI : 256;
+    const int TB = BN / HI;
+    IndexerParams P{};
+    P.P = P_;
+    P.Lq = Lq;
+    P.q_pos0 = q_pos0;
+    P.ctx_len = ctx_len;
+    P.Lk = Lk;
+    P.w = w;
+    P.scores = scores;
+    P.ld = ld;
+    P.num_qb = (Lq + TB - 1) / TB;
+    const int sms = num_sms();
+    if (sms <= 0) return DSA_ERR_CUDA;
+    const int64_t ktiles = (Lk + kIdxBM - 1) / kIdxBM;
+    if (decode) {
+        int ns = std::max(1, (2 * sms + P_ - 1) / P_);
+        ns = (int)std::min<int64_t>(ns, ktiles);
+        P.kt_per_split = (int)((ktiles + ns - 1) / ns);
+        P.nsplit = (int)((ktiles + P.kt_per_split - 1) / P.kt_per_split);
+    } else {
+        P.nsplit = 1;
+        P.kt_per_split = (int)ktiles;
+    }
+    P.num_units = P_ * P.num_qb * P.nsplit;
+    const uint64_t qrows = (uint64_t)Lq * HI;
+    const uint32_t qbox = (uint32_t)std::min<uint64_t>(BN, qrows);
+    const uint32_t kbox = (uint32_t)std::min<int64_t>(kIdxBM, Lk);
+    P.q_box_bytes = qbox * 128u;
+    P.k_box_bytes = kbox * 128u;
+    CUtensorMap mq, mk;
+    if (!make_rows_map(&mq, qI, qrows, (uint64_t)P_, qrows * 128ull, qbox)) return DSA_ERR_CUDA;
+    if (!make_rows_map(&mk, kI, (uint64_t)Lk, (uint64_t)P_, (uint64_t)Lk * 128ull, kbox)) return DSA_ERR_CUDA;
+    const int grid = std::min(P.num_units, sms);
+    if (grid <= 0) return DSA_OK;
+    if (!decode) {
+        switch (HI) {
+        case 1: return launch_indexer_t<1, 256, kPrefillIdxStages>(mq, mk, P, grid, s);
+        case 2: return launch_indexer_t<2, 256, kPrefillIdxStages>(mq, mk, P, grid, s);
+        case 4: return launch_indexer_t<4, 256, kPrefillIdxStages>(mq, mk, P, grid, s);
+        case 8: return launch_indexer_t<8, 256, kPrefillIdxStages>(mq, mk, P, grid, s);
+        case 16: return launch_indexer_t<16, 256, kPrefillIdxStages>(mq, mk, P, grid, s);
+        case 32: return launch_indexer_t<32, 256, kPrefillIdxStages>(mq, mk, P, grid, s);
+        case 64: return launch_indexer_t<64, 256, kPrefillIdxStages>(mq, mk, P, grid, s);
+        }
+    } else {
+        switch (HI) {
+        case 16: return launch_indexer_t<16, 16, kDecodeIdxStages>(mq, mk, P, grid, s);
+        case 32: return launch_indexer_t<32, 32, kDecodeIdxStages>(mq, mk, P, grid, s);
+        case 64: return launch_indexer_t<64, 64, kDecodeIdxStages>(mq, mk, P, grid, s);
+        }
+    }
+    return DSA_ERR_UNSUPPORTED;
+}
+
+// ------------------------------------------------------------------ top-k launch
+dsa_status run_topk(const float* scores, int64_t ld, int rows, int64_t q_pos0, const int* ctx_len, int64_t n_max,
+                    int k, int* idx, cudaStream_t s) {
+    static bool attr_set = false;
+    if (!attr_set) {
+        if (cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(TopkShared)) !=
+            cudaSuccess)
+            return DSA_ERR_CUDA;
+        attr_set = true;
+    }
+    TopkParams P{scores, ld, rows, q_pos0, ctx_len, n_max, k, idx};
+    LaunchScope ls(K_TOPK, s);
+    topk_kernel<<<rows, kTopkThreads, sizeof(TopkShared), s>>>(P);
+    return launch_status();
+}
+
+// ------------------------------------------------------------------ attention launch
+template <int NT>
+dsa_status launch_attn_t(const AttnParams& P, cudaStream_t s) {
+    const int smem = attn_smem_bytes(P.Hkv);
+    auto kern = sparse_attn_kernel<NT>;
+    static int attr_bytes = 0;
+    if (attr_bytes < smem) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, attn_smem_bytes(1)) !=
+            cudaSuccess)
+            return DSA_ERR_CUDA;
+        attr_bytes = attn_smem_bytes(1);
+    }
+    LaunchScope ls(K_ATTN, s);
+    kern<<<P.T * P.nsplit, P.Hkv * kAttnWPG * 32, smem, s>>>(P);
+    return launch_status();
+}
+
+dsa_status run_attn(const AttnParams& P, cudaStream_t s) {
+    const int G = P.Hq / P.Hkv;
+    if (G <= 8) return launch_attn_t<1>(P, s);
+    return launch_attn_t<2>(P, s);
+}
+
+// ------------------------------------------------------------------ decode helpers
+__global__ void decode_append_kernel(const __nv_bfloat16* k_new, const __nv_bfloat16* v_new,
+                                     const __nv_bfloat16* kI_new, __nv_bfloat16* k_cache, __nv_bfloat16* v_cache,
+                                     __nv_bfloat16* kI_cache, const int* ctx_len, long long Lmax, int kv_elems,
+                                     int dI) {
+    const int b = blockIdx.x;
+    const long long pos = ctx_len[b];
+    if (pos < 0 || pos >= Lmax) {
+        if (threadIdx.x == 0) record_error(DSA_DEV_ERR_BOUNDS, 0x501);
+        return;
+    }
+    const int kv16 = kv_elems / 8, kI16 = dI / 8;  // 16-byte vectors
+    const uint4* ks = reinterpret_cast<const uint4*>(k_new + (long long)b * kv_elems);
+    const uint4* vs = reinterpret_cast<const uint4*>(v_new + (long long)b * kv_elems);
+    uint4* kd = reinterpret_cast<uint4*>(k_cache + ((long long)b * Lmax + pos) * kv_elems);
+    uint4* vd = reinterpret_cast<uint4*>(v_cache + ((long long)b * Lmax + pos) * kv_elems);
+    for (int i = threadIdx.x; i < kv16; i += blockDim.x) {
+        kd[i] = ks[i];
+        vd[i] = vs[i];
+    }
+    const uint4* is = reinterpret_cast<const uint4*>(kI_new + (long long)b * dI);
+    uint4* id = reinterpret_cast<uint4*>(kI_cache + ((long long)b * Lmax + pos) * dI);
+    for (int i = threadIdx.x; i < kI16; i += blockDim.x) id[i] = is[i];
+}
+
+__global__ void decode_advance_kernel(int* ctx_len, int B, long long Lmax) {
+    const int b = blockIdx.x * blockDim.x + threadIdx.x;
+    if (b < B && ctx_len[b] >= 0 && ctx_len[b] < Lmax) ctx_len[b] += 1;
+}
+
+// Sequences whose ctx_len is out of range must not be read past the caches by the other kernels;
+// the indexer, top-k and attention kernels clamp their key counts to the cache capacity, and the
+// append kernel reports the bad input.
+
+__global__ void selftest_timeout_kernel(unsigned long long limit_ns) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        // nothing ever arrives on `bar`: the wait must end by its time limit
+        const unsigned long long t0 = globaltimer_ns();
+        while (!mbar_try_wait(&bar, 0)) {
+            if (globaltimer_ns() - t0 > limit_ns) {
+                record_error(DSA_DEV_ERR_TIMEOUT, 0x901);
+                break;
+            }
+        }
+    }
+}
+
+int decode_attn_splits(int B) {
+    const int sms = std::max(1, num_sms());
+    return std::max(1, std::min(kMaxDecodeSplits, sms / std::max(1, B)));
+}
+
+struct DecodeWs {
+    size_t scores, idx, part, total;
+};
+DecodeWs decode_ws_layout(int64_t Lmax, int B, int Hq, int topk, bool need_idx) {
+    DecodeWs w{};
+    const int64_t ld = (int64_t)align_up((size_t)Lmax, 4);
+    w.scores = 0;
+    size_t off = align_up((size_t)B * ld * 4, 256);
+    w.idx = off;
+    if (need_idx) off = align_up(off + (size_t)B * topk * 4, 256);
+    w.part = off;
+    off = align_up(off + (size_t)B * kMaxDecodeSplits * Hq * (kAttnD + 2) * 4, 256);
+    w.total = off;
+    return w;
+}
+
+int64_t prefill_ld(int64_t L) { return (int64_t)align_up((size_t)L, 4); }
+
+}  // namespace
+
+// ====================================================================== C ABI
+extern "C" {
+
+const char* dsa_status_string(int status) {
+    switch (status) {
+    case DSA_OK: return "DSA_OK";
+    case DSA_ERR_INVALID_ARG: return "DSA_ERR_INVALID_ARG: invalid argument (null/misaligned pointer or bad size)";
+    case DSA_ERR_UNSUPPORTED: return "DSA_ERR_UNSUPPORTED: shape outside the supported set";
+    case DSA_ERR_WORKSPACE: return "DSA_ERR_WORKSPACE: workspace missing or too small";
+    case DSA_ERR_CUDA: return "DSA_ERR_CUDA: a CUDA call or kernel launch failed";
+    case DSA_ERR_TIMEOUT: return "DSA_ERR_TIMEOUT: a kernel's bounded wait expired";
+    case DSA_ERR_DEVICE_INPUT: return "DSA_ERR_DEVICE_INPUT: a device-side input check failed";
+    default: return "DSA_ERR_UNKNOWN";
+    }
+}
+
+int dsa_version(void) { return kVersion; }
+
+dsa_status dsa_index(const void* qI, const void* kI, const void* w, int Lq, int64_t Lk, int HI, int dI,
+                     int64_t q_pos0, float* scores, int64_t ld_scores, dsa_stream_t stream) {
+    if (!qI || !kI || !w || !scores) return DSA_ERR_INVALID_ARG;
+    if (!aligned16(qI) || !aligned16(kI) || !aligned16(scores)) return DSA_ERR_INVALID_ARG;
+    if (Lq <= 0 || Lk <= 0 || HI <= 0 || dI <= 0 || q_pos0 < 0) return DSA_ERR_INVALID_ARG;
+    if (q_pos0 + Lq > Lk || ld_scores < q_pos0 + Lq || ld_scores % 4 != 0) return DSA_ERR_INVALID_ARG;
+    if (dI != kIdxBK || !hi_supported_prefill(HI)) return DSA_ERR_UNSUPPORTED;
+    if ((int64_t)Lq * HI > (int64_t)INT32_MAX || Lk > (int64_t)INT32_MAX) return DSA_ERR_UNSUPPORTED;
+    return run_indexer(qI, kI, static_cast<const __nv_bfloat16*>(w), 1, Lq, q_pos0, nullptr, Lk, HI, scores,
+                       ld_scores, reinterpret_cast<cudaStream_t>(stream));
+}
+
+dsa_status dsa_topk(const float* scores, int64_t ld_scores, int Lq, int64_t q_pos0, int k, int32_t* idx, void* ws,
+                    size_t ws_bytes, dsa_stream_t stream) {
+    (void)ws;
+    (void)ws_bytes;
+    if (!scores || !idx) return DSA_ERR_INVALID_ARG;
+    if (!aligned16(scores) || !aligned16(idx)) return DSA_ERR_INVALID_ARG;
+    if (Lq <= 0 || q_pos0 < 0 || ld_scores % 4 != 0 || ld_scores < q_pos0 + Lq) return DSA_ERR_INVALID_ARG;
+    if (k <= 0) return DSA_ERR_INVALID_ARG;
+    if (k > kMaxTopk || q_pos0 + Lq > (int64_t)INT32_MAX) return DSA_ERR_UNSUPPORTED;
+    return run_topk(scores, ld_scores, Lq, q_pos0, nullptr, q_pos0 + Lq, k, idx,
+                    reinterpret_cast<cudaStream_t>(stream));
+}
+
+dsa_status dsa_sparse_attn(const void* q, const void* k, const void* v, const int32_t* idx, int Lq, int64_t Lk,
+                           int64_t q_pos0, int Hq, int Hkv, int D, int topk, float scale, void* out, float* lse,
+                           dsa_stream_t stream) {
+    if (!q || !k || !v || !idx || !out) return DSA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(idx) || !aligned16(out))
+        return DSA_ERR_INVALID_ARG;
+    if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return DSA_ERR_INVALID_ARG;
+    if (Lq <= 0 || Lk <= 0 || q_pos0 < 0 || topk <= 0 || !(scale == scale)) return DSA_ERR_INVALID_ARG;
+    dsa_status st = check_attn_shape(Hq, Hkv, D);
+    if (st != DSA_OK) return st;
+    if (topk > kMaxTopk || Lk > (int64_t)INT32_MAX) return DSA_ERR_UNSUPPORTED;
+    AttnParams P{};
+    P.q = static_cast<const __nv_bfloat16*>(q);
+    P.k = static_cast<const __nv_bfloat16*>(k);
+    P.v = static_cast<const __nv_bfloat16*>(v);
+    P.kv_bstride = 0;
+    P.idx = idx;
+    P.topk = topk;
+    P.T = Lq;
+    P.q_pos0 = q_pos0;
+    P.ctx_len = nullptr;
+    P.n_keys = Lk;
+    P.Hq = Hq;
+    P.Hkv = Hkv;
+    P.scale_log2 = scale * 1.4426950408889634f;
+    P.out = static_cast<__nv_bfloat16*>(out);
+    P.lse = lse;
+    P.nsplit = 1;
+    P.part = nullptr;
+    return run_attn(P, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t dsa_workspace_size(int op, int64_t L, int B, int Hq, int HI, int topk) {
+    if (L <= 0 || topk <= 0 || HI <= 0) return 0;
+    switch (op) {
+    case DSA_OP_INDEX:
+    case DSA_OP_TOPK:
+    case DSA_OP_SPARSE_ATTN: return 0;
+    case DSA_OP_PREFILL: {
+        const int64_t ld = prefill_ld(L);
+        int64_t rows = (int64_t(4) << 30) / (ld * 4);
+        rows = std::max<int64_t>(256, rows / 256 * 256);
+        rows = std::min<int64_t>(rows, L);
+        return align_up((size_t)rows * ld * 4, 256) + align_up((size_t)rows * topk * 4, 256);
+    }
+    case DSA_OP_DECODE:
+        if (B <= 0 || Hq <= 0) return 0;
+        return decode_ws_layout(L, B, Hq, topk, true).total;
+    default: return 0;
+    }
+}
+
+dsa_status dsa_prefill(const void* q, const void* k, const void* v, const void* qI, const void* kI, const void* w,
+                       int64_t L, int Hq, int Hkv, int D, int HI, int dI, int topk, float scale, void* out,
+                       int32_t* idx_out, void* ws, size_t ws_bytes, dsa_stream_t stream) {
+    if (!q || !k || !v || !qI || !kI || !w || !out) return DSA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(qI) || !aligned16(kI) || !aligned16(w) ||
+        !aligned16(out) || (idx_out && !aligned16(idx_out)))
+        return DSA_ERR_INVALID_ARG;
+    if (L <= 0 || topk <= 0 || HI <= 0 || dI <= 0 || !(scale == scale)) return DSA_ERR_INVALID_ARG;
+    dsa_status st = check_attn_shape(Hq, Hkv, D);
+    if (st != DSA_OK) return st;
+    if (dI != kIdxBK || !hi_supported_prefill(HI) || topk > kMaxTopk || L * HI > (int64_t)INT32_MAX)
+        return DSA_ERR_UNSUPPORTED;
+    if (!ws || !aligned16(ws)) return DSA_ERR_WORKSPACE;
+    const int64_t ld = prefill_ld(L);
+    const int TB = 256 / HI;
+    const size_t per_row = (size_t)ld * 4 + (idx_out ? 0 : (size_t)topk * 4);
+    int64_t C = (int64_t)((ws_bytes > 512 ? ws_bytes - 512 : 0) / per_row);  // 512: alignment slack
+    C = std::min<int64_t>(C, L);
+    if (C >= TB) C = C / TB * TB;
+    if (C < std::min<int64_t>(L, TB)) return DSA_ERR_WORKSPACE;
+    float* scores = static_cast<float*>(ws);
+    int32_t* idx_ws = idx_out ? nullptr
+                              : reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) +
+                                                           align_up((size_t)C * ld * 4, 256));
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const auto* qb = static_cast<const __nv_bfloat16*>(q);
+    const auto* qIb = static_cast<const __nv_bfloat16*>(qI);
+    const auto* wb = static_cast<const __nv_bfloat16*>(w);
+    auto* ob = static_cast<__nv_bfloat16*>(out);
+    for (int64_t c0 = 0; c0 < L; c0 += C) {
+        const int rows = (int)std::min<int64_t>(C, L - c0);
+        int32_t* idx_c = idx_out ? idx_out + c0 * topk : idx_ws;
+        st = run_indexer(qIb + c0 * HI * dI, kI, wb + c0 * HI, 1, rows, c0, nullptr, c0 + rows, HI, scores, ld, s);
+        if (st != DSA_OK) return st;
+        st = run_topk(scores, ld, rows, c0, nullptr, c0 + rows, topk, idx_c, s);
+        if (st != DSA_OK) return st;
+        AttnParams P{};
+        P.q = qb + c0 * Hq * D;
+        P.k = static_cast<const __nv_bfloat16*>(k);
+        P.v = static_cast<const __nv_bfloat16*>(v);
+        P.idx = idx_c;
+        P.topk = topk;
+        P.T = rows;
+        P.q_pos0 = c0;
+        P.n_keys = L;
+        P.Hq = Hq;
+        P.Hkv = Hkv;
+        P.scale_log2 = scale * 1.4426950408889634f;
+        P.out = ob + c0 * Hq * D;
+        P.nsplit = 1;
+        st = run_attn(P, s);
+        if (st != DSA_OK) return st;
+    }
+    return DSA_OK;
+}
+
+dsa_status dsa_decode(const void* q, const void* qI, const void* w, const void* k_new, const void* v_new,
+                      const void* kI_new, void* k_cache, void* v_cache, void* kI_cache, int32_t* ctx_len, int B,
+                      int64_t Lmax, int Hq, int Hkv, int D, int HI, int dI, int topk, float scale, int update_ctx,
+                      void* out, int32_t* idx_out, void* ws, size_t ws_bytes, dsa_stream_t stream) {
+    const void* ptrs[] = {q, qI, w, k_new, v_new, kI_new, k_cache, v_cache, kI_cache, ctx_len, out};
+    for (const void* p : ptrs)
+        if (!p || !aligned16(p)) return DSA_ERR_INVALID_ARG;
+    if (idx_out && !aligned16(idx_out)) return DSA_ERR_INVALID_ARG;
+    if (B <= 0 || Lmax <= 0 || topk <= 0 || HI <= 0 || dI <= 0 || !(scale == scale)) return DSA_ERR_INVALID_ARG;
+    dsa_status st = check_attn_shape(Hq, Hkv, D);
+    if (st != DSA_OK) return st;
+    if (dI != kIdxBK || !hi_supported_decode(HI) || topk > kMaxTopk || Lmax > (int64_t)INT32_MAX)
+        return DSA_ERR_UNSUPPORTED;
+    const DecodeWs L = decode_ws_layout(Lmax, B, Hq, topk, idx_out == nullptr);
+    if (!ws || !aligned16(ws)) return DSA_ERR_WORKSPACE;
+    if (ws_bytes < L.total) return DSA_ERR_WORKSPACE;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t* wsb = static_cast<uint8_t*>(ws);
+    float* scores = reinterpret_cast<float*>(wsb + L.scores);
+    int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(wsb + L.idx);
+    float* part = reinterpret_cast<float*>(wsb + L.part);
+    const int64_t ld = (int64_t)align_up((size_t)Lmax, 4);
+    {
+        LaunchScope ls(K_APPEND, s);
+        decode_append_kernel<<<B, 128, 0, s>>>(
+            static_cast<const __nv_bfloat16*>(k_new), static_cast<const __nv_bfloat16*>(v_new),
+            static_cast<const __nv_bfloat16*>(kI_new), static_cast<__nv_bfloat16*>(k_cache),
+            static_cast<__nv_bfloat16*>(v_cache), static_cast<__nv_bfloat16*>(kI_cache), ctx_len, Lmax, Hkv * D, dI);
+        if ((st = launch_status()) != DSA_OK) return st;
+    }
+    st = run_indexer(qI, kI_cache, static_cast<const __nv_bfloat16*>(w), B, 1, 0, ctx_len, Lmax, HI, scores, ld, s);
+    if (st != DSA_OK) return st;
+    st = run_topk(scores, ld, B, 0, ctx_len, Lmax, topk, idx, s);
+    if (st != DSA_OK) return st;
+    AttnParams P{};
+    P.q = static_cast<const __nv_bfloat16*>(q);
+    P.k = static_cast<const __nv_bfloat16*>(k_cache);
+    P.v = static_cast<const __nv_bfloat16*>(v_cache);
+    P.kv_bstride = Lmax * Hkv * D;
+    P.idx = idx;
+    P.topk = topk;
+    P.T = B;
+    P.ctx_len = ctx_len;
+    P.n_keys = Lmax;
+    P.Hq = Hq;
+    P.Hkv = Hkv;
+    P.scale_log2 = scale * 1.4426950408889634f;
+    P.out = static_cast<__nv_bfloat16*>(out);
+    P.nsplit = decode_attn_splits(B);
+    P.part = part;
+    st = run_attn(P, s);
+    if (st != DSA_OK) return st;
+    if (P.nsplit > 1) {
+        LaunchScope ls(K_COMBINE, s);
+        const int warps = B * Hq;
+        attn_combine_kernel<<<(warps + 3) / 4, 128, 0, s>>>(part, B, P.nsplit, Hq, P.out, nullptr);
+        if ((st = launch_status()) != DSA_OK) return st;
+    }
+    if (update_ctx) {
+        LaunchScope ls(K_ADVANCE, s);
+        decode_advance_kernel<<<(B + 127) / 128, 128, 0, s>>>(ctx_len, B, Lmax);
+        if ((st = launch_status()) != DSA_OK) return st;
+    }
+    return DSA_OK;
+}
+
+dsa_status dsa_sync_status(dsa_stream_t stream) {
+    if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return DSA_ERR_CUDA;
+    if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
+    unsigned int err = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&err, g_dev_error, sizeof(err)) != cudaSuccess) return DSA_ERR_CUDA;
+    if (err) {
+        if (cudaMemcpyToSymbol(g_dev_error, &zero, sizeof(zero)) != cudaSuccess) return DSA_ERR_CUDA;
+    }
+    if (err & DSA_DEV_ERR_TIMEOUT) return DSA_ERR_TIMEOUT;
+    if (err & DSA_DEV_ERR_BOUNDS) return DSA_ERR_DEVICE_INPUT;
+    return DSA_OK;
+}
+
+void dsa_profile_begin(void) {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    for (auto& r : g_prof_recs) {
+        g_event_pool.push_back(r.a);
+        g_event_pool.push_back(r.b);
+    }
+    g_prof_recs.clear();
+    g_prof_on = true;
+}
+
+dsa_status dsa_profile_end(int64_t* launches, double* total_ms) {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    g_prof_on = false;
+    dsa_status st = DSA_OK;
+    for (int i = 0; i < DSA_PROFILE_KINDS; ++i) {
+        if (launches) launches[i] = 0;
+        if (total_ms) total_ms[i] = 0.0;
+    }
+    for (auto& r : g_prof_recs) {
+        float ms = 0.f;
+        if (cudaEventSynchronize(r.b) != cudaSuccess || cudaEventElapsedTime(&ms, r.a, r.b) != cudaSuccess) {
+            st = DSA_ERR_CUDA;
+            continue;
+        }
+        if (launches) launches[r.kind] += 1;
+        if (total_ms) total_ms[r.kind] += ms;
+    }
+    for (auto& r : g_prof_recs) {
+        g_event_pool.push_back(r.a);
+        g_event_pool.push_back(r.b);
+    }
+    g_prof_recs.clear();
+    return st;
+}
+
+int64_t dsa_launch_count(void) { return g_launches.load(); }
+
+dsa_status dsa_selftest_timeout(int64_t wait_ns, dsa_stream_t stream) {
+    if (wait_ns <= 0 || wait_ns > 2000000000ll) return DSA_ERR_INVALID_ARG;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    LaunchScope ls(K_SELFTEST, s);
+    selftest_timeout_kernel<<<1, 32, 0, s>>>((unsigned long long)wait_ns);
+    return launch_status();
+}
+
+}  // extern "C"

@@ -1,0 +1,315 @@
+// Lightning-indexer scores on the 5th-generation tensor cores.
+//
+//   score(t, s) = sum_h w[t,h] * max(0, qI[t,h,:] . kI[s,:])      for keys s <= t
+//
+// The pages describe a light "scout" with one MQA-shared key per position that scores every
+// position for the current token (page "快手开源大模型Keye-VL-2.0：一个能“看懂“两小时视频AI",
+// gsyq.cn, section 一); the formula above is the one this library adopts (the pages give none).
+//
+// Tiling.  One MMA tile is D[128 keys, BN columns] = kI_tile[128 x 64] . Qtile[BN x 64]^T where
+// the BN columns are (token, head) pairs of TB = BN/HI consecutive query tokens.  The key tile
+// is the M operand, so every TMEM lane holds one key and the head sum for a token is a plain
+// in-thread reduction over that token's HI columns; the weights are a broadcast from shared
+// memory and consecutive lanes write consecutive keys (coalesced 128-byte score stores).
+//
+// Roles (one CTA per SM, persistent):
+//   warp 0        TMA producer: the unit's Q tile (once per unit) and a ring of kI tiles
+//   warp 1        TMEM allocator + single-thread tcgen05.mma issuer
+//   warps 2..     epilogue: tcgen05.ld, ReLU, weight FMA, head sum, score store;
+//                 NWG warpgroups split the BN columns between them
+// Two TMEM accumulators (2 x BN fp32 columns) let the MMA of tile j+1 overlap the epilogue of
+// tile j.  Work units are (problem p, query block qb, key-tile range); prefill uses one problem
+// and whole causal key ranges, decode uses one problem per sequence and splits its keys.
+#pragma once
+
+#include "ptx.cuh"
+
+namespace dsa {
+
+constexpr int kIdxBM = 128;  // keys per tile
+constexpr int kIdxBK = 64;   // = d_I, one 128-byte swizzled row per key / per (token, head)
+
+struct IndexerParams {
+    int P;                      // problems: 1 (prefill) or B sequences (decode)
+    int Lq;                     // query rows per problem
+    long long q_pos0;           // prefill: absolute position of query row 0
+    const int* ctx_len;         // decode: query position of problem p is ctx_len[p]; else null
+    long long Lk;               // keys addressable per problem (TMA extent)
+    const __nv_bfloat16* w;     // [P, Lq, HI]
+    float* scores;              // row (p*Lq + i) at scores + row*ld
+    long long ld;
+    int num_qb;                 // query blocks per problem
+    int nsplit;                 // key-range splits per (p, qb)
+    int kt_per_split;           // key tiles per split (nsplit > 1)
+    int num_units;              // P * num_qb * nsplit
+    uint32_t q_box_bytes;       // bytes one Q TMA box brings
+    uint32_t k_box_bytes;       // bytes one kI TMA box brings
+};
+
+struct IndexerUnit {
+    int p, qb, kt0, kt1;        // key tiles [kt0, kt1)
+    long long tq0;              // absolute position of the block's first query row
+    int rows;                   // valid query rows in the block
+};
+
+template <int TB>
+__device__ __forceinline__ IndexerUnit indexer_unit(const IndexerParams& P, int u) {
+    IndexerUnit r;
+    const int per_p = P.num_qb * P.nsplit;
+    r.p = u / per_p;
+    const int rem = u - r.p * per_p;
+    // prefill: the last query blocks carry the most keys, start with them
+    r.qb = P.num_qb - 1 - rem / P.nsplit;
+    const int split = rem % P.nsplit;
+    long long base = P.q_pos0;
+    if (P.ctx_len) {  // decode: clamp a bad context length to the cache (the append kernel reports it)
+        base = P.ctx_len[r.p];
+        base = base < 0 ? 0 : (base >= P.Lk ? P.Lk - 1 : base);
+    }
+    r.tq0 = base + (long long)r.qb * TB;
+    const int first = r.qb * TB;
+    r.rows = min(TB, P.Lq - first);
+    const long long t_last = r.tq0 + r.rows - 1;
+    const int nkt = (int)(t_last / kIdxBM) + 1;
+    if (P.nsplit == 1) {
+        r.kt0 = 0;
+        r.kt1 = nkt;
+    } else {
+        r.kt0 = split * P.kt_per_split;
+        r.kt1 = min(nkt, r.kt0 + P.kt_per_split);
+    }
+    return r;
+}
+
+// Snake order over CTAs so that long and short units mix evenly.
+__device__ __forceinline__ int indexer_unit_of(int round, int cta, int grid) {
+    return round * grid + ((round & 1) ? (grid - 1 - cta) : cta);
+}
+
+template <int HI, int BN, int STAGES>
+struct IndexerCfg {
+    static constexpr int TB = BN / HI;
+    static constexpr int NWG = (BN >= 128 && BN / 2 >= HI) ? 2 : 1;
+    static constexpr int COLS_WG = BN / NWG;
+    static constexpr int CHUNK = COLS_WG >= 32 ? 32 : 16;
+    static constexpr int NCHUNK = COLS_WG / CHUNK;
+    static constexpr int THREADS = 64 + NWG * 128;
+    static constexpr int A_BYTES = kIdxBM * kIdxBK * 2;  // 16 KB
+    static constexpr int B_BYTES = BN * kIdxBK * 2;
+    static constexpr int TMEM_COLS = (2 * BN <= 32) ? 32 : (2 * BN <= 64) ? 64 : (2 * BN <= 128) ? 128 : (2 * BN <= 256) ? 256 : 512;
+    // shared memory layout (offsets from a 1024-aligned base)
+    static constexpr int OFF_A = 0;
+    static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
+    static constexpr int OFF_W = OFF_B + 2 * B_BYTES;       // per epilogue warp: 2 x COLS_WG weights
+    static constexpr int OFF_BAR = OFF_W + NWG * 4 * 2 * COLS_WG * 4;
+    static constexpr int NBAR = 2 * STAGES + 8;
+    static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+    static constexpr int SMEM = OFF_MISC + 16 + 1024;  // + alignment slack
+    static_assert(BN % HI == 0 && BN >= 16 && BN <= 256 && BN % 16 == 0, "bad BN");
+    static_assert(HI <= COLS_WG, "a token's heads must stay inside one warpgroup");
+    static_assert(HI <= CHUNK || HI % CHUNK == 0, "bad HI");
+};
+
+template <int HI, int BN, int STAGES>
+__global__ void __launch_bounds__(IndexerCfg<HI, BN, STAGES>::THREADS, 1)
+    indexer_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
+                   const IndexerParams P) {
+    using C = IndexerCfg<HI, BN, STAGES>;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sA = smem + C::OFF_A;
+    uint8_t* sB = smem + C::OFF_B;
+    float* sW = reinterpret_cast<float*>(smem + C::OFF_W);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+    uint64_t* a_full = bars;
+    uint64_t* a_empty = bars + STAGES;
+    uint64_t* q_full = bars + 2 * STAGES;
+    uint64_t* q_empty = q_full + 2;
+    uint64_t* acc_full = q_full + 4;
+    uint64_t* acc_empty = q_full + 6;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < STAGES; ++i) {
+            mbar_init(&a_full[i], 1);
+            mbar_init(&a_empty[i], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&q_full[i], 1);
+            mbar_init(&q_empty[i], 1);
+            mbar_init(&acc_full[i], 1);
+            mbar_init(&acc_empty[i], C::NWG * 128);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+        prefetch_tensormap(&map_q);
+        prefetch_tensormap(&map_k);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    const int grid = gridDim.x, cta = blockIdx.x;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            int st = 0;
+            uint32_t a_ph = 0, q_ph = 0;
+            int qbuf = 0;
+            bool ok = true;
+            for (int rd = 0; ok; ++rd) {
+                const int u = indexer_unit_of(rd, cta, grid);
+                if (u >= P.num_units) break;
+                const IndexerUnit U = indexer_unit<C::TB>(P, u);
+                if (U.kt0 >= U.kt1) continue;
+                ok = wait_parity(&q_empty[qbuf], q_ph ^ 1, 0x101, abort_flag);
+                if (!ok) break;
+                mbar_arrive_expect_tx(&q_full[qbuf], P.q_box_bytes);
+                tma_load_3d(sB + qbuf * C::B_BYTES, &map_q, &q_full[qbuf], 0, U.qb * C::TB * HI, U.p);
+                if (++qbuf == 2) { qbuf = 0; q_ph ^= 1; }
+                for (int kt = U.kt0; kt < U.kt1; ++kt) {
+                    ok = wait_parity(&a_empty[st], a_ph ^ 1, 0x102, abort_flag);
+                    if (!ok) break;
+                    mbar_arrive_expect_tx(&a_full[st], P.k_box_bytes);
+                    tma_load_3d(sA + st * C::A_BYTES, &map_k, &a_full[st], 0, kt * kIdxBM, U.p);
+                    if (++st == STAGES) { st = 0; a_ph ^= 1; }
+                }
+            }
+            if (!ok) {
+                // Let the copies already issued land before the CTA leaves (bounded waits).  The
+                // last copy into stage i used phase a_ph if i < st, else a_ph ^ 1; waiting on a
+                // phase that already completed returns at once.
+                for (int i = 0; i < STAGES; ++i) wait_parity(&a_full[i], i < st ? a_ph : a_ph ^ 1, 0x103, nullptr);
+                for (int i = 0; i < 2; ++i) wait_parity(&q_full[i], i < qbuf ? q_ph : q_ph ^ 1, 0x104, nullptr);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_bf16_f32<kIdxBM, BN>();
+            int st = 0, ab = 0, qbuf = 0;
+            uint32_t a_ph = 0, acc_ph = 0, q_ph = 0;
+            bool ok = true;
+            for (int rd = 0; ok; ++rd) {
+                const int u = indexer_unit_of(rd, cta, grid);
+                if (u >= P.num_units) break;
+                const IndexerUnit U = indexer_unit<C::TB>(P, u);
+                if (U.kt0 >= U.kt1) continue;
+                ok = wait_parity(&q_full[qbuf], q_ph, 0x201, abort_flag);
+                if (!ok) break;
+                const uint64_t bdesc = smem_desc_k128_sw128(sB + qbuf * C::B_BYTES);
+                for (int kt = U.kt0; kt < U.kt1; ++kt) {
+                    ok = wait_parity(&a_full[st], a_ph, 0x202, abort_flag) &&
+                         wait_parity(&acc_empty[ab], acc_ph ^ 1, 0x203, abort_flag);
+                    if (!ok) break;
+                    tc_fence_after();
+                    const uint64_t adesc = smem_desc_k128_sw128(sA + st * C::A_BYTES);
+                    const uint32_t d_tmem = tmem_base + ab * BN;
+#pragma unroll
+                    for (int kk = 0; kk < kIdxBK / 16; ++kk)  // K = 16 per MMA, 32 bytes along the row
+                        umma_bf16(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, idesc, kk > 0 ? 1u : 0u);
+                    umma_commit(&a_empty[st]);
+                    umma_commit(&acc_full[ab]);
+                    if (++st == STAGES) { st = 0; a_ph ^= 1; }
+                    if (++ab == 2) { ab = 0; acc_ph ^= 1; }
+                }
+                if (!ok) break;
+                umma_commit(&q_empty[qbuf]);
+                if (++qbuf == 2) { qbuf = 0; q_ph ^= 1; }
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue warpgroups
+        const int et = threadIdx.x - 64;            // 0 .. NWG*128-1
+        const int wg = et >> 7;                     // column half
+        const int quarter = warp & 3;               // TMEM lanes this warp may access
+        const int key_in_tile = quarter * 32 + lane;
+        int ab = 0, ubuf = 0;
+        uint32_t acc_ph = 0;
+        for (int rd = 0;; ++rd) {
+            const int u = indexer_unit_of(rd, cta, grid);
+            if (u >= P.num_units) break;
+            const IndexerUnit U = indexer_unit<C::TB>(P, u);
+            if (U.kt0 >= U.kt1) continue;
+            // Weights of this unit's tokens for this warpgroup's columns (column c = token*HI + head),
+            // one private copy per warp so that only __syncwarp is needed.
+            float* w_s = sW + ((warp - 2) * 2 + ubuf) * C::COLS_WG;
+            for (int cc = lane; cc < C::COLS_WG; cc += 32) {
+                const int c = wg * C::COLS_WG + cc;
+                const int tok = c / HI;
+                float wv = 0.f;
+                if (tok < U.rows)
+                    wv = __bfloat162float(P.w[((long long)U.p * P.Lq + (long long)U.qb * C::TB + tok) * HI + (c % HI)]);
+                w_s[cc] = wv;
+            }
+            __syncwarp();
+            bool ok = true;
+            for (int kt = U.kt0; kt < U.kt1; ++kt) {
+                ok = wait_parity(&acc_full[ab], acc_ph, 0x301, abort_flag);
+                __syncwarp();  // reconverge before the warp-collective tcgen05.ld
+                ok = __all_sync(0xffffffffu, ok);
+                if (!ok) break;
+                tc_fence_after();
+                const long long s = (long long)kt * kIdxBM + key_in_tile;
+                const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + ab * BN;
+                float carry = 0.f;
+#pragma unroll
+                for (int ch = 0; ch < C::NCHUNK; ++ch) {
+                    const int col0 = wg * C::COLS_WG + ch * C::CHUNK;
+                    float v[C::CHUNK];
+                    if constexpr (C::CHUNK == 32) tmem_ld_32x32b_x32(taddr + col0, v);
+                    else tmem_ld_32x32b_x16(taddr + col0, v);
+                    tmem_ld_wait();
+                    if (ch == C::NCHUNK - 1) {
+                        // every TMEM read of this accumulator is done: hand it back to the MMA
+                        tc_fence_before();
+                        mbar_arrive(&acc_empty[ab]);
+                    }
+                    if constexpr (HI <= C::CHUNK) {
+#pragma unroll
+                        for (int j = 0; j < C::CHUNK / HI; ++j) {
+                            float a = 0.f;
+#pragma unroll
+                            for (int h = 0; h < HI; ++h)
+                                a = fmaf(w_s[ch * C::CHUNK + j * HI + h], fmaxf(v[j * HI + h], 0.f), a);
+                            const int tok = (col0 + j * HI) / HI;
+                            const long long tq = U.tq0 + tok;
+                            if (tok < U.rows && s <= tq && s < P.Lk)
+                                P.scores[((long long)U.p * P.Lq + (long long)U.qb * C::TB + tok) * P.ld + s] = a;
+                        }
+                    } else {
+#pragma unroll
+                        for (int h = 0; h < C::CHUNK; ++h) carry = fmaf(w_s[ch * C::CHUNK + h], fmaxf(v[h], 0.f), carry);
+                        if ((col0 + C::CHUNK) % HI == 0) {
+                            const int tok = col0 / HI;
+                            const long long tq = U.tq0 + tok;
+                            if (tok < U.rows && s <= tq && s < P.Lk)
+                                P.scores[((long long)U.p * P.Lq + (long long)U.qb * C::TB + tok) * P.ld + s] = carry;
+                            carry = 0.f;
+                        }
+                    }
+                }
+                if (++ab == 2) { ab = 0; acc_ph ^= 1; }
+            }
+            if (!ok) break;
+            ubuf ^= 1;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, C::TMEM_COLS);
+    }
+}
+
+}  // namespace dsa

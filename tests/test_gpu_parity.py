@@ -1,0 +1,322 @@
+"""GPU parity of the CUDA path (through the C ABI) against the fp64 oracle, step by step and fused.
+
+Sizes: the whole 'tiny' workload (L=1024, k=256, 8/2/128, HI=4) and slices / the whole of the
+'32k' workload (L=32768, k=2048, 32/4/128, HI=32), so that the kernels run over many tiles plus
+ragged tails.  Tolerances: see tests/parity.py.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from parity import assert_output_ok, bf16_tensor_to_f64, index_set_mismatch
+
+pytestmark = pytest.mark.gpu
+
+dsa = pytest.importorskip("dsa_lightning_indexer_02_b200")
+
+
+def dev(a: np.ndarray) -> torch.Tensor:
+    return synth.to_torch(a).cuda()
+
+
+def score_bound(qI, w, kI, t_rows):
+    """|fp32 score - exact score| bound: 64 u * sum_h |w_h| sum_d |q_hd k_d| (fp32 MMA sum of 64
+    exact products) + 32 u * sum_h |w_h| relu_h (fp32 head sum), u = 2^-24; taken as 1e-5 * B."""
+    qa = np.abs(synth.bf16_to_f64(qI))          # [r, HI, dI]
+    wa = np.abs(synth.bf16_to_f64(w))           # [r, HI]
+    ka = np.abs(synth.bf16_to_f64(kI))          # [Lk, dI]
+    return np.einsum("rh,rhd,sd->rs", wa, qa, ka[: int(np.max(t_rows)) + 1])
+
+
+@pytest.fixture(scope="module")
+def tiny():
+    cfg = synth.CONFIGS["tiny"]
+    x = synth.inputs(cfg, 0, cfg.L)
+    rows = np.arange(cfg.L)
+    ref = oracle.dsa_rows(x["q"], x["qI"], x["w"], x["k"], x["v"], x["kI"], rows, cfg.k, cfg.scale,
+                          keep_scores=True)
+    return cfg, x, ref
+
+
+def test_index_tiny_full(cuda_ok, tiny):
+    cfg, x, ref = tiny
+    L = cfg.L
+    scores = torch.full((L, L), float("nan"), device="cuda")
+    dsa.dsa_index(dev(x["qI"]), dev(x["kI"]), dev(x["w"]), 0, scores)
+    assert dsa.sync_status() == dsa.DSA_OK
+    got = scores.cpu().double().numpy()
+    mask = np.tril(np.ones((L, L), dtype=bool))
+    bound = 1e-5 * score_bound(x["qI"], x["w"], x["kI"], np.arange(L)) + 1e-30
+    err = np.abs(got - ref["scores"])
+    assert np.all(err[mask] <= bound[mask]), float(np.max(err[mask] / bound[mask]))
+    assert np.all(np.isnan(got[~mask]))  # nothing written above the diagonal
+
+
+@pytest.mark.parametrize("q_pos0,Lq", [(32768 - 96, 96), (1000, 37), (0, 5)])
+def test_index_32k_slices(cuda_ok, q_pos0, Lq):
+    cfg = synth.CONFIGS["32k"]
+    Lk = q_pos0 + Lq
+    qI, w = synth.tensor(cfg, "qI", q_pos0, Lq), synth.tensor(cfg, "w", q_pos0, Lq)
+    kI = synth.tensor(cfg, "kI", 0, Lk)
+    ld = (Lk + 3) // 4 * 4
+    scores = torch.full((Lq, ld), float("nan"), device="cuda")
+    dsa.dsa_index(dev(qI), dev(kI), dev(w), q_pos0, scores)
+    assert dsa.sync_status() == dsa.DSA_OK
+    rows = np.arange(q_pos0, q_pos0 + Lq)
+    ref = oracle.index_rows(qI, w, kI, rows)
+    got = scores.cpu().double().numpy()[:, :Lk]
+    bound = 1e-5 * score_bound(qI, w, kI, rows)
+    for r in range(Lq):
+        n = rows[r] + 1
+        assert np.all(np.abs(got[r, :n] - ref[r, :n]) <= bound[r, :n]), r
+        assert np.all(np.isnan(got[r, n:]))
+
+
+def test_topk_exact_on_oracle_scores(cuda_ok, tiny):
+    """Fed the oracle's scores rounded to fp32, the GPU top-k must equal the oracle's top-k of the
+    same fp32 values exactly (ties by lower index)."""
+    cfg, x, ref = tiny
+    L = cfg.L
+    s32 = np.nan_to_num(ref["scores"], nan=0.0).astype(np.float32)
+    idx = torch.empty((L, cfg.k), dtype=torch.int32, device="cuda")
+    dsa.dsa_topk(torch.from_numpy(s32).cuda(), 0, cfg.k, idx)
+    assert dsa.sync_status() == dsa.DSA_OK
+    want, _ = oracle.topk_rows(s32.astype(np.float64), np.arange(L) + 1, cfg.k)
+    got = idx.cpu().numpy()
+    for r in range(L):
+        assert sorted(got[r][got[r] >= 0].tolist()) == sorted(want[r][want[r] >= 0].tolist()), r
+        assert np.all(got[r][min(cfg.k, r + 1):] == -1)
+
+
+@pytest.mark.parametrize("kind", ["ties", "zeros", "wide"])
+def test_topk_long_rows_and_heavy_ties(cuda_ok, kind):
+    """Long rows (beyond the candidate buffer), massive exact ties, -0/+0, the global-memory path."""
+    rng = np.random.default_rng(11)
+    rows, n, k = 6, 40000, 2048
+    ld = n
+    if kind == "ties":
+        s = rng.integers(-3, 4, size=(rows, ld)).astype(np.float32)       # 7 distinct values
+    elif kind == "zeros":
+        s = np.zeros((rows, ld), dtype=np.float32)
+        s[:, ::7] = -0.0
+        s[:, 5::11] = 1.0
+    else:
+        s = (rng.standard_normal((rows, ld)) * 30).astype(np.float32)
+    q_pos0 = n - rows
+    idx = torch.empty((rows, k), dtype=torch.int32, device="cuda")
+    dsa.dsa_topk(torch.from_numpy(s).cuda(), q_pos0, k, idx)
+    assert dsa.sync_status() == dsa.DSA_OK
+    want, _ = oracle.topk_rows(s.astype(np.float64), q_pos0 + np.arange(rows) + 1, k)
+    got = idx.cpu().numpy()
+    for r in range(rows):
+        assert sorted(got[r].tolist()) == sorted(want[r].tolist()), r
+
+
+def test_sparse_attn_on_oracle_indices(cuda_ok, tiny):
+    cfg, x, ref = tiny
+    L = cfg.L
+    out = torch.empty((L, cfg.Hq, cfg.D), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((L, cfg.Hq), dtype=torch.float32, device="cuda")
+    dsa.dsa_sparse_attn(dev(x["q"]), dev(x["k"]), dev(x["v"]), torch.from_numpy(ref["idx"]).cuda(), 0, cfg.scale,
+                        out, lse)
+    assert dsa.sync_status() == dsa.DSA_OK
+    assert_output_ok(bf16_tensor_to_f64(out), ref["out"], "attn")
+    np.testing.assert_allclose(lse.cpu().numpy(), ref["lse"], rtol=0, atol=2e-3)
+
+
+def test_sparse_attn_gqa_shapes(cuda_ok):
+    """G = 16 (two 8-head tiles), Hkv = 1 and 2, topk not a multiple of the stage size."""
+    rng = np.random.default_rng(12)
+    for Hq, Hkv, topk in ((32, 2, 300), (16, 1, 77), (8, 4, 129)):
+        L = 700
+        q = rng.standard_normal((L, Hq, 128)).astype(np.float32)
+        k = rng.standard_normal((L, Hkv, 128)).astype(np.float32)
+        v = rng.standard_normal((L, Hkv, 128)).astype(np.float32)
+        tq, tk, tv = (torch.from_numpy(a).to(torch.bfloat16) for a in (q, k, v))
+        bits = [t.view(torch.int16).numpy().view(np.uint16) for t in (tq, tk, tv)]
+        idx = np.full((L, topk), -1, dtype=np.int32)
+        for t in range(L):
+            m = min(topk, t + 1)
+            idx[t, :m] = rng.choice(t + 1, size=m, replace=False)
+        out = torch.empty((L, Hq, 128), dtype=torch.bfloat16, device="cuda")
+        dsa.dsa_sparse_attn(tq.cuda(), tk.cuda(), tv.cuda(), torch.from_numpy(idx).cuda(), 0, 0.0883883, out)
+        assert dsa.sync_status() == dsa.DSA_OK
+        want, _ = oracle.sparse_attn_rows(bits[0], bits[1], bits[2], idx, 0.0883883)
+        assert_output_ok(bf16_tensor_to_f64(out), want, f"Hq={Hq} Hkv={Hkv}")
+
+
+def check_prefill(cfg, x, idx_gpu, out_gpu, rows):
+    """Index sets within the near-tie band and outputs within tolerance on sampled rows."""
+    ref = oracle.dsa_rows(x["q"][rows], x["qI"][rows], x["w"][rows], x["k"], x["v"], x["kI"], rows, cfg.k,
+                          cfg.scale, keep_scores=True)
+    mm = index_set_mismatch(idx_gpu, ref["idx"], ref["scores"], ref["tau"], ref["absmax"], rows + 1)
+    assert mm["structural"] == 0 and mm["out_of_band"] == 0, mm
+    own, _ = oracle.sparse_attn_rows(x["q"][rows], x["k"], x["v"], idx_gpu, cfg.scale)
+    assert_output_ok(out_gpu, own, "vs oracle on GPU indices")
+    if mm["rows_diff"] == 0:
+        assert_output_ok(out_gpu, ref["out"], "vs oracle end to end")
+    return mm
+
+
+def run_prefill(cfg, x, ws_bytes=None):
+    L = cfg.L
+    out = torch.empty((L, cfg.Hq, cfg.D), dtype=torch.bfloat16, device="cuda")
+    idx = torch.empty((L, cfg.k), dtype=torch.int32, device="cuda")
+    ws = None
+    if ws_bytes is not None:
+        ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
+    dsa.dsa_prefill(dev(x["q"]), dev(x["k"]), dev(x["v"]), dev(x["qI"]), dev(x["kI"]), dev(x["w"]), cfg.k,
+                    cfg.scale, out, idx, ws)
+    assert dsa.sync_status() == dsa.DSA_OK
+    return out, idx
+
+
+def test_prefill_tiny_full(cuda_ok, tiny):
+    cfg, x, ref = tiny
+    out, idx = run_prefill(cfg, x)
+    rows = np.arange(cfg.L)
+    check_prefill(cfg, x, idx.cpu().numpy(), bf16_tensor_to_f64(out), rows)
+
+
+def test_prefill_tiny_chunked_is_identical_and_deterministic(cuda_ok, tiny):
+    cfg, x, _ = tiny
+    out1, idx1 = run_prefill(cfg, x)
+    per_row = cfg.L * 4
+    out2, idx2 = run_prefill(cfg, x, ws_bytes=200 * per_row + 4096)   # chunks of 192 rows
+    out3, idx3 = run_prefill(cfg, x)
+    for a, b in ((out1, out2), (out1, out3)):
+        assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+    assert torch.equal(idx1, idx2) and torch.equal(idx1, idx3)
+
+
+@pytest.fixture(scope="module")
+def c32k():
+    cfg = synth.CONFIGS["32k"]
+    return cfg, synth.inputs(cfg, 0, cfg.L)
+
+
+def test_prefill_32k_sampled_rows(cuda_ok, c32k):
+    cfg, x = c32k
+    out, idx = run_prefill(cfg, x)
+    L = cfg.L
+    rows = np.unique(np.concatenate([[0, 1, cfg.k - 2, cfg.k - 1, cfg.k, 255, 256, 4095, 4096, L - 257, L - 1],
+                                     synth.sample_rows(21, L, seed=1)]))
+    mm = check_prefill(cfg, x, idx.cpu().numpy()[rows], bf16_tensor_to_f64(out[torch.from_numpy(rows).cuda()]),
+                       rows)
+    # idx rows of short prefixes hold every causal key
+    got = idx[:cfg.k].cpu().numpy()
+    for t in (0, 7, cfg.k - 1):
+        assert sorted(got[t][got[t] >= 0].tolist()) == list(range(t + 1))
+    print("32k index mismatch stats", mm)
+
+
+def test_prefill_32k_deterministic(cuda_ok, c32k):
+    cfg, x = c32k
+    out1, idx1 = run_prefill(cfg, x)
+    out2, idx2 = run_prefill(cfg, x, ws_bytes=3000 * cfg.L * 4)       # several chunks
+    assert torch.equal(idx1, idx2)
+    assert torch.equal(out1.view(torch.int16), out2.view(torch.int16))
+
+
+def make_decode_case(B, Lmax, ctx, steps, seed_cfg="32k"):
+    """Sequences of the 32k workload's layout; ctx[b] tokens cached, `steps` new tokens each."""
+    cfg = synth.CONFIGS[seed_cfg]
+    data = [synth.inputs(cfg, 0, int(ctx[b]) + steps, seq=b) for b in range(B)]
+    kc = np.zeros((B, Lmax, cfg.Hkv, cfg.D), dtype=np.uint16)
+    vc = np.zeros_like(kc)
+    kIc = np.zeros((B, Lmax, cfg.dI), dtype=np.uint16)
+    for b in range(B):
+        c = int(ctx[b])
+        kc[b, :c], vc[b, :c], kIc[b, :c] = data[b]["k"][:c], data[b]["v"][:c], data[b]["kI"][:c]
+    return cfg, data, kc, vc, kIc
+
+
+def test_decode_steps_against_oracle(cuda_ok):
+    B, Lmax, steps = 4, 6144, 3
+    ctx = np.array([5, 1500, 2047, 6000])
+    cfg, data, kc, vc, kIc = make_decode_case(B, Lmax, ctx, steps)
+    kc_t, vc_t, kIc_t = dev(kc), dev(vc), dev(kIc)
+    ctx_t = torch.from_numpy(ctx.astype(np.int32)).cuda()
+    out = torch.empty((B, cfg.Hq, cfg.D), dtype=torch.bfloat16, device="cuda")
+    idx = torch.empty((B, cfg.k), dtype=torch.int32, device="cuda")
+    for j in range(steps):
+        pos = ctx + j
+        sel = lambda name: np.stack([data[b][name][pos[b]] for b in range(B)])  # noqa: E731
+        dsa.dsa_decode(dev(sel("q")), dev(sel("qI")), dev(sel("w")), dev(sel("k")), dev(sel("v")), dev(sel("kI")),
+                       kc_t, vc_t, kIc_t, ctx_t, cfg.k, cfg.scale, out, idx, update_ctx=True)
+        assert dsa.sync_status() == dsa.DSA_OK
+        assert np.array_equal(ctx_t.cpu().numpy(), pos + 1)
+        got_idx, got_out = idx.cpu().numpy(), bf16_tensor_to_f64(out)
+        for b in range(B):
+            t = int(pos[b])
+            d = data[b]
+            r = np.array([t])
+            ref = oracle.dsa_rows(d["q"][r], d["qI"][r], d["w"][r], d["k"], d["v"], d["kI"], r, cfg.k, cfg.scale,
+                                  keep_scores=True)
+            mm = index_set_mismatch(got_idx[b:b + 1], ref["idx"], ref["scores"], ref["tau"], ref["absmax"], r + 1)
+            assert mm["structural"] == 0 and mm["out_of_band"] == 0, (b, j, mm)
+            own, _ = oracle.sparse_attn_rows(d["q"][r], d["k"], d["v"], got_idx[b:b + 1], cfg.scale)
+            assert_output_ok(got_out[b:b + 1], own, f"decode b={b} step={j}")
+
+
+def test_decode_matches_prefill_row(cuda_ok):
+    """A decode step at position t gives the prefill result of row t (same indices, close output)."""
+    cfg = synth.CONFIGS["32k"]
+    L = 3000
+    x = synth.inputs(cfg, 0, L)
+    sub = synth.Config("sub", cfg.cid, L, cfg.k, layout=cfg.layout, p0=cfg.p0)
+    out_p, idx_p = run_prefill(sub, x)
+    Lmax, t = 3072, L - 1
+    kc = np.zeros((1, Lmax, cfg.Hkv, cfg.D), dtype=np.uint16)
+    vc, kIc = np.zeros_like(kc), np.zeros((1, Lmax, cfg.dI), dtype=np.uint16)
+    kc[0, :t], vc[0, :t], kIc[0, :t] = x["k"][:t], x["v"][:t], x["kI"][:t]
+    ctx = torch.tensor([t], dtype=torch.int32, device="cuda")
+    out = torch.empty((1, cfg.Hq, cfg.D), dtype=torch.bfloat16, device="cuda")
+    idx = torch.empty((1, cfg.k), dtype=torch.int32, device="cuda")
+    dsa.dsa_decode(dev(x["q"][t:t + 1]), dev(x["qI"][t:t + 1]), dev(x["w"][t:t + 1]), dev(x["k"][t:t + 1]),
+                   dev(x["v"][t:t + 1]), dev(x["kI"][t:t + 1]), dev(kc), dev(vc), dev(kIc), ctx, cfg.k, cfg.scale,
+                   out, idx)
+    assert dsa.sync_status() == dsa.DSA_OK
+    assert sorted(idx[0].tolist()) == sorted(idx_p[t].tolist())
+    d = (out[0].double() - out_p[t].double()).abs().max().item()
+    assert d <= 1e-2
+
+
+def test_decode_bad_context_length_reports_error(cuda_ok):
+    B, Lmax = 2, 1024
+    cfg = synth.CONFIGS["32k"]
+    kc = torch.zeros((B, Lmax, cfg.Hkv, cfg.D), dtype=torch.bfloat16, device="cuda")
+    vc = torch.zeros_like(kc)
+    kIc = torch.zeros((B, Lmax, cfg.dI), dtype=torch.bfloat16, device="cuda")
+    q = torch.zeros((B, cfg.Hq, cfg.D), dtype=torch.bfloat16, device="cuda")
+    qI = torch.zeros((B, cfg.HI, cfg.dI), dtype=torch.bfloat16, device="cuda")
+    w = torch.zeros((B, cfg.HI), dtype=torch.bfloat16, device="cuda")
+    kn = torch.zeros((B, cfg.Hkv, cfg.D), dtype=torch.bfloat16, device="cuda")
+    kIn = torch.zeros((B, cfg.dI), dtype=torch.bfloat16, device="cuda")
+    ctx = torch.tensor([10, Lmax + 5], dtype=torch.int32, device="cuda")
+    out = torch.empty_like(q)
+    dsa.dsa_decode(q, qI, w, kn, kn, kIn, kc, vc, kIc, ctx, 256, 0.1, out)
+    assert dsa.sync_status() == dsa.DSA_ERR_DEVICE_INPUT
+    assert dsa.sync_status() == dsa.DSA_OK          # the error word was cleared
+    torch.cuda.synchronize()
+
+
+def test_bounded_wait_timeout_reports_and_context_survives(cuda_ok):
+    dsa.selftest_timeout(50_000_000)                # 50 ms wait on a barrier nobody completes
+    assert dsa.sync_status() == dsa.DSA_ERR_TIMEOUT
+    assert dsa.sync_status() == dsa.DSA_OK
+    x = torch.ones(1000, device="cuda")             # the context is still usable
+    assert float(x.sum()) == 1000.0
+
+
+def test_profile_and_launch_counter(cuda_ok, tiny):
+    cfg, x, _ = tiny
+    n0 = dsa.launch_count()
+    dsa.profile_begin()
+    run_prefill(cfg, x)
+    prof = dsa.profile_end()
+    assert dsa.launch_count() - n0 == 3
+    assert prof["indexer"]["launches"] == 1 and prof["topk"]["launches"] == 1 and prof["sparse_attn"]["launches"] == 1
+    assert all(v["ms"] > 0 for k, v in prof.items() if v["launches"])

@@ -177,6 +177,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--chunk-rows", type=int, default=0,
+                    help="limit the prefill workspace to this many score rows (small profiling cases)")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
@@ -215,8 +217,10 @@ def main():
     d = {n: host[n].cuda() for n in names}
     out = torch.empty((cfg.L, cfg.Hq, cfg.D), dtype=torch.bfloat16, device="cuda")
     idx = torch.empty((cfg.L, cfg.k), dtype=torch.int32, device="cuda")
-    ws = torch.empty(dsa.workspace_size(dsa.DSA_OP_PREFILL, cfg.L, 1, cfg.Hq, cfg.HI, cfg.k), dtype=torch.uint8,
-                     device="cuda")
+    ws_bytes = dsa.workspace_size(dsa.DSA_OP_PREFILL, cfg.L, 1, cfg.Hq, cfg.HI, cfg.k)
+    if args.chunk_rows:
+        ws_bytes = args.chunk_rows * ((cfg.L + 3) // 4 * 4) * 4 + 4096
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
     stream = torch.cuda.current_stream()
 
     def step():

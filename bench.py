@@ -173,6 +173,7 @@ def main():
     ap.add_argument("--impl", default="dsa", choices=["dsa", "reference"])
     ap.add_argument("--workload", default="128k", choices=["32k", "128k", "256k"])
     ap.add_argument("--decode-steps", type=int, default=256)
+    ap.add_argument("--decode-ctx", type=int, default=0, help="override the cached context (small profiling cases)")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
@@ -187,6 +188,7 @@ def main():
     import torch.distributed as dist
 
     import dsa_lightning_indexer_02_b200 as dsa
+    from dsa_lightning_indexer_02_b200.sharding import reduce_max, weak_scaling_value
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -203,11 +205,7 @@ def main():
             dist.barrier()
 
     def max_over_ranks(v: float) -> float:
-        if world == 1:
-            return v
-        t = torch.tensor([v], device="cuda", dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return reduce_max(v, dist if world > 1 else None, device="cuda")
 
     peaks, peak_src = load_peaks()
     cfg = synth.CONFIGS[args.workload]
@@ -250,7 +248,8 @@ def main():
     if dsa.sync_status() != dsa.DSA_OK:
         raise SystemExit("device error during the timed region")
     ms_step = max_over_ranks(ev0.elapsed_time(ev1) / args.steps)
-    value = world * cfg.L / (ms_step / 1000.0)
+    value = weak_scaling_value(cfg.L, world, ms_step / 1000.0)
+    union16 = adjacent_union_stat(idx, cfg, torch)
     clk = clocks.summary()
 
     # ---- per-kernel roofline (event-timed launches inside the timed region)
@@ -327,8 +326,11 @@ def main():
     # ---- decode: 16 sequences x 131072 cached tokens, 256 steps
     decode = None
     if not args.no_decode:
-        decode = run_decode(torch, dsa, synth.CONFIGS["decode"], args.decode_steps, rank, world, barrier,
-                            max_over_ranks, peaks)
+        dcfg = synth.CONFIGS["decode"]
+        if args.decode_ctx:
+            import dataclasses
+            dcfg = dataclasses.replace(dcfg, L=args.decode_ctx, iid_from=args.decode_ctx)
+        decode = run_decode(torch, dsa, dcfg, args.decode_steps, rank, world, barrier, max_over_ranks, peaks)
 
     cpu = None
     if rank == 0 and not args.no_cpu and world == 1:
@@ -343,12 +345,24 @@ def main():
                        "parallelism": f"dp{world} (independent sequences)",
                        "l2": "inputs (1.8 GB) larger than L2; no flush"},
             "roofline": roofline, "kernels": kern, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
-            "clocks": clk, "decode": decode}
+            "clocks": clk, "decode": decode, "adjacent_union_16": union16}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
     return 0
+
+
+def adjacent_union_stat(idx, cfg, torch, windows: int = 32) -> dict:
+    """Mean size of the union of 16 adjacent index sets (rows t..t+15, t >= k) on evenly spaced
+    windows: the statistic the pages quote for their adjacent-query dedup (about 8000 of 32768
+    at 128K, k = 2048)."""
+    starts = np.linspace(cfg.k, cfg.L - 16, windows).astype(np.int64)
+    sizes = []
+    for t0 in starts:
+        rows = idx[int(t0):int(t0) + 16].cpu().numpy()
+        sizes.append(len(np.unique(rows[rows >= 0])))
+    return {"mean_unique": float(np.mean(sizes)), "naive": 16 * cfg.k, "windows": windows}
 
 
 def lib_hash() -> str:

@@ -29,6 +29,7 @@ namespace dsa {
 constexpr int kAttnD = 128;
 constexpr int kAttnStages = 3;
 constexpr int kAttnWPG = 2;  // warps per KV group
+constexpr int kAttnIdxWin = 2048;  // index-list window kept in shared memory
 
 struct AttnParams {
     const __nv_bfloat16* q;   // [T, Hq, D]
@@ -52,7 +53,7 @@ struct AttnParams {
 __host__ __device__ constexpr int attn_keys_per_stage(int hkv) { return 128 / hkv; }
 __host__ __device__ constexpr int attn_row_bytes(int hkv) { return hkv * kAttnD * 2 + 16; }
 __host__ __device__ constexpr int attn_smem_bytes(int hkv) {
-    return kAttnStages * attn_keys_per_stage(hkv) * attn_row_bytes(hkv) * 2;
+    return kAttnStages * attn_keys_per_stage(hkv) * attn_row_bytes(hkv) * 2 + kAttnIdxWin * 4;
 }
 
 // NT: n-tiles of 8 query heads per KV group (G <= 8 * NT).
@@ -101,6 +102,19 @@ __global__ void __launch_bounds__(256) sparse_attn_kernel(const AttnParams P) {
         }
     }
 
+    // ---- the index list, kAttnIdxWin entries at a time, in shared memory: the gathers of a stage
+    // are issued without waiting on a global load of their indices
+    int* sidx = reinterpret_cast<int*>(smem + kAttnStages * STAGE);
+    int win_off = 0;  // window covers slots [p_begin + win_off, p_begin + win_off + kAttnIdxWin)
+    auto fill_window = [&]() {
+        for (int i = threadIdx.x; i < kAttnIdxWin; i += nthreads) {
+            const int p = p_begin + win_off + i;
+            sidx[i] = p < p_end ? __ldg(idx_row + p) : -1;
+        }
+    };
+    fill_window();
+    __syncthreads();
+
     // ---- async gather of one stage: KS keys x (all KV heads) of K and V
     const int chunks_per_row = Hkv * kAttnD * 2 / 16;
     auto load_stage = [&](int step, int buf) {
@@ -110,7 +124,7 @@ __global__ void __launch_bounds__(256) sparse_attn_kernel(const AttnParams P) {
         for (int c = threadIdx.x; c < KS * chunks_per_row; c += nthreads) {
             const int key = c / chunks_per_row, ch = c % chunks_per_row;
             const int p = p0 + key;
-            int s = (p < p_end) ? idx_row[p] : -1;
+            int s = (p < p_end) ? sidx[p - p_begin - win_off] : -1;
             bool ok = s >= 0 && s < P.n_keys;
             const long long off = (ok ? (long long)s : 0) * (Hkv * kAttnD) + ch * 8;
             cp_async_16(sk + key * RB + ch * 16, kb + off, ok);
@@ -139,7 +153,15 @@ __global__ void __launch_bounds__(256) sparse_attn_kernel(const AttnParams P) {
     for (int step = 0; step < nsteps; ++step) {
         cp_async_wait<kAttnStages - 2>();
         __syncthreads();
-        if (step + kAttnStages - 1 < nsteps) load_stage(step + kAttnStages - 1, (step + kAttnStages - 1) % kAttnStages);
+        const int ls = step + kAttnStages - 1;
+        if (ls < nsteps) {
+            if (ls * KS >= win_off + kAttnIdxWin) {  // uniform: next window of the index list
+                win_off += kAttnIdxWin;
+                fill_window();
+                __syncthreads();
+            }
+            load_stage(ls, ls % kAttnStages);
+        }
         cp_async_commit();
 
         const uint8_t* sk = smem + (step % kAttnStages) * STAGE;

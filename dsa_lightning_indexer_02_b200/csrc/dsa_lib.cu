@@ -224,6 +224,32 @@ dsa_status run_topk(const float* scores, int64_t ld, int rows, int64_t q_pos0, c
         attr_set = true;
     }
     TopkParams P{scores, ld, rows, q_pos0, ctx_len, n_max, k, idx};
+    const int sms = num_sms();
+    // Few long rows: a cluster of CTAs per row; otherwise one CTA per row.
+    if ((long long)rows * kTopkCluster <= 2LL * sms && n_max > 4LL * kTopkCap) {
+        static bool cattr = false;
+        if (!cattr) {
+            if (cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)sizeof(TopkShared)) != cudaSuccess)
+                return DSA_ERR_CUDA;
+            cattr = true;
+        }
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(rows * kTopkCluster);
+        cfg.blockDim = dim3(kTopkThreads);
+        cfg.dynamicSmemBytes = sizeof(TopkShared);
+        cfg.stream = s;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = kTopkCluster;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        LaunchScope ls(K_TOPK, s);
+        if (cudaLaunchKernelEx(&cfg, topk_cluster_kernel, P) != cudaSuccess) return DSA_ERR_CUDA;
+        return launch_status();
+    }
     LaunchScope ls(K_TOPK, s);
     topk_kernel<<<rows, kTopkThreads, sizeof(TopkShared), s>>>(P);
     return launch_status();

@@ -86,6 +86,60 @@ __device__ __forceinline__ int indexer_unit_of(int round, int cta, int grid) {
     return round * grid + ((round & 1) ? (grid - 1 - cta) : cta);
 }
 
+template <int CHUNK>
+__device__ __forceinline__ void tmem_ld_chunk(uint32_t taddr, float (&v)[CHUNK]) {
+    if constexpr (CHUNK == 32) tmem_ld_32x32b_x32(taddr, v);
+    else tmem_ld_32x32b_x16(taddr, v);
+}
+
+// c + a * b on packed fp32 pairs (one fma.rn.f32x2).
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+    uint64_t pa, pb, pc, pd;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(pa) : "f"(a.x), "f"(a.y));
+    asm("mov.b64 %0, {%1, %2};" : "=l"(pb) : "f"(b.x), "f"(b.y));
+    asm("mov.b64 %0, {%1, %2};" : "=l"(pc) : "f"(c.x), "f"(c.y));
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(pd) : "l"(pa), "l"(pb), "l"(pc));
+    float2 d;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(d.x), "=f"(d.y) : "l"(pd));
+    return d;
+}
+
+// sum_h w[h] * max(v[h], 0) over N >= 1 heads, with independent partial sums (no long
+// dependent FMA chain) on packed fp32 pairs.
+template <int N>
+__device__ __forceinline__ float head_sum(const float* v, const float* w) {
+    if constexpr (N == 1) {
+        return w[0] * fmaxf(v[0], 0.f);
+    } else {
+        constexpr int NP = N / 2;                 // pairs
+        constexpr int NA = NP < 4 ? NP : 4;       // independent accumulators
+        float2 acc[NA];
+#pragma unroll
+        for (int i = 0; i < NA; ++i) acc[i] = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int p = 0; p < NP; ++p) {
+            const float2 x = make_float2(fmaxf(v[2 * p], 0.f), fmaxf(v[2 * p + 1], 0.f));
+            const float2 ww = *reinterpret_cast<const float2*>(w + 2 * p);
+            acc[p % NA] = ffma2(x, ww, acc[p % NA]);
+        }
+        float r = 0.f;
+#pragma unroll
+        for (int i = 0; i < NA; ++i) r += acc[i].x + acc[i].y;
+        return r;
+    }
+}
+
+// carry[0..3] += packed partial sums of w[h] * max(v[h], 0) over one chunk of N heads.
+template <int N>
+__device__ __forceinline__ void head_sum_acc(const float* v, const float* w, float2 (&carry)[4]) {
+#pragma unroll
+    for (int p = 0; p < N / 2; ++p) {
+        const float2 x = make_float2(fmaxf(v[2 * p], 0.f), fmaxf(v[2 * p + 1], 0.f));
+        const float2 ww = *reinterpret_cast<const float2*>(w + 2 * p);
+        carry[p % 4] = ffma2(x, ww, carry[p % 4]);
+    }
+}
+
 template <int HI, int BN, int STAGES>
 struct IndexerCfg {
     static constexpr int TB = BN / HI;
@@ -259,43 +313,46 @@ __global__ void __launch_bounds__(IndexerCfg<HI, BN, STAGES>::THREADS, 1)
                 if (!ok) break;
                 tc_fence_after();
                 const long long s = (long long)kt * kIdxBM + key_in_tile;
-                const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + ab * BN;
-                float carry = 0.f;
+                const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + ab * BN + wg * C::COLS_WG;
+                const long long row0 = (long long)U.p * P.Lq + (long long)U.qb * C::TB;
+                // TMEM loads run one chunk ahead of the math: ld(c+1) is in flight while chunk c is
+                // reduced; the accumulator is released right after the last load completes.
+                float va[C::CHUNK], vb[C::CHUNK];
+                float2 carry[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) carry[i] = make_float2(0.f, 0.f);
+                tmem_ld_chunk<C::CHUNK>(taddr, va);
+                tmem_ld_wait();
 #pragma unroll
                 for (int ch = 0; ch < C::NCHUNK; ++ch) {
-                    const int col0 = wg * C::COLS_WG + ch * C::CHUNK;
-                    float v[C::CHUNK];
-                    if constexpr (C::CHUNK == 32) tmem_ld_32x32b_x32(taddr + col0, v);
-                    else tmem_ld_32x32b_x16(taddr + col0, v);
-                    tmem_ld_wait();
-                    if (ch == C::NCHUNK - 1) {
-                        // every TMEM read of this accumulator is done: hand it back to the MMA
+                    float(&cur)[C::CHUNK] = (ch & 1) ? vb : va;
+                    float(&nxt)[C::CHUNK] = (ch & 1) ? va : vb;
+                    if (ch + 1 < C::NCHUNK) {
+                        tmem_ld_chunk<C::CHUNK>(taddr + (ch + 1) * C::CHUNK, nxt);
+                    } else {
                         tc_fence_before();
                         mbar_arrive(&acc_empty[ab]);
                     }
+                    const int cw = ch * C::CHUNK;  // column offset inside this warpgroup
                     if constexpr (HI <= C::CHUNK) {
 #pragma unroll
                         for (int j = 0; j < C::CHUNK / HI; ++j) {
-                            float a = 0.f;
-#pragma unroll
-                            for (int h = 0; h < HI; ++h)
-                                a = fmaf(w_s[ch * C::CHUNK + j * HI + h], fmaxf(v[j * HI + h], 0.f), a);
-                            const int tok = (col0 + j * HI) / HI;
-                            const long long tq = U.tq0 + tok;
-                            if (tok < U.rows && s <= tq && s < P.Lk)
-                                P.scores[((long long)U.p * P.Lq + (long long)U.qb * C::TB + tok) * P.ld + s] = a;
+                            const float a = head_sum<HI>(cur + j * HI, w_s + cw + j * HI);
+                            const int tok = (wg * C::COLS_WG + cw) / HI + j;
+                            if (tok < U.rows && s <= U.tq0 + tok && s < P.Lk) P.scores[(row0 + tok) * P.ld + s] = a;
                         }
                     } else {
+                        head_sum_acc<C::CHUNK>(cur, w_s + cw, carry);
+                        if ((wg * C::COLS_WG + cw + C::CHUNK) % HI == 0) {
+                            const float a = (carry[0].x + carry[0].y) + (carry[1].x + carry[1].y) +
+                                            (carry[2].x + carry[2].y) + (carry[3].x + carry[3].y);
+                            const int tok = (wg * C::COLS_WG + cw) / HI;
+                            if (tok < U.rows && s <= U.tq0 + tok && s < P.Lk) P.scores[(row0 + tok) * P.ld + s] = a;
 #pragma unroll
-                        for (int h = 0; h < C::CHUNK; ++h) carry = fmaf(w_s[ch * C::CHUNK + h], fmaxf(v[h], 0.f), carry);
-                        if ((col0 + C::CHUNK) % HI == 0) {
-                            const int tok = col0 / HI;
-                            const long long tq = U.tq0 + tok;
-                            if (tok < U.rows && s <= tq && s < P.Lk)
-                                P.scores[((long long)U.p * P.Lq + (long long)U.qb * C::TB + tok) * P.ld + s] = carry;
-                            carry = 0.f;
+                            for (int i = 0; i < 4; ++i) carry[i] = make_float2(0.f, 0.f);
                         }
                     }
+                    if (ch + 1 < C::NCHUNK) tmem_ld_wait();
                 }
                 if (++ab == 2) { ab = 0; acc_ph ^= 1; }
             }

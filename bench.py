@@ -245,6 +245,7 @@ def main():
         barrier()
     prof = dsa.profile_end()
     launches = dsa.launch_count() - n_launch0
+    counters = dsa.read_counters(reset=True)
     if dsa.sync_status() != dsa.DSA_OK:
         raise SystemExit("device error during the timed region")
     ms_step = max_over_ranks(ev0.elapsed_time(ev1) / args.steps)
@@ -345,7 +346,7 @@ def main():
                        "parallelism": f"dp{world} (independent sequences)",
                        "l2": "inputs (1.8 GB) larger than L2; no flush"},
             "roofline": roofline, "kernels": kern, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
-            "clocks": clk, "decode": decode, "adjacent_union_16": union16}
+            "clocks": clk, "decode": decode, "adjacent_union_16": union16, "path_counters": counters}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -416,6 +417,7 @@ def run_decode(torch, dsa, cfg, steps, rank, world, barrier, max_over_ranks, pea
     ev1.record(stream)
     torch.cuda.synchronize()
     prof = dsa.profile_end()
+    dcount = dsa.read_counters(reset=True)
     barrier()
     ms = max_over_ranks(ev0.elapsed_time(ev1))
     kmeans = {k: v["ms"] / steps for k, v in prof.items() if v["launches"]}
@@ -425,7 +427,7 @@ def run_decode(torch, dsa, cfg, steps, rank, world, barrier, max_over_ranks, pea
     return {"value": world * B * steps / (ms / 1e3), "unit": UNIT, "steps": steps, "batch": B, "ctx": ctx0,
             "ms_per_decode_step": ms / steps, "kernel_ms_per_step": kmeans,
             "hbm_frac": bytes_step / (ms / steps / 1e3) / 1e9 / peaks["hbm_gbs"],
-            "algorithmic_bytes_per_step": bytes_step}
+            "algorithmic_bytes_per_step": bytes_step, "path_counters": dcount}
 
 
 if __name__ == "__main__":

@@ -49,6 +49,7 @@ _SIGS = {
     "dsa_profile_begin": (None, []),
     "dsa_profile_end": (_i, [_p, _p]),
     "dsa_launch_count": (_i64, []),
+    "dsa_read_counters": (_i, [_p, _i, _i]),
     "dsa_selftest_timeout": (_i, [_i64, _p]),
 }
 for _name, (_res, _args) in _SIGS.items():
@@ -199,6 +200,14 @@ def profile_end() -> dict:
     ms = (ctypes.c_double * len(PROFILE_KINDS))()
     _check(_lib.dsa_profile_end(launches, ms), "dsa_profile_end")
     return {k: {"launches": int(launches[i]), "ms": float(ms[i])} for i, k in enumerate(PROFILE_KINDS)}
+
+
+def read_counters(reset: bool = False) -> dict:
+    """Device path counters: top-k rows and sampled-threshold fallbacks (see dsa.h)."""
+    buf = (ctypes.c_int64 * 8)()
+    _check(_lib.dsa_read_counters(buf, 8, int(bool(reset))), "dsa_read_counters")
+    return {"topk_rows": buf[0], "topk_retry": buf[1], "topk_global": buf[4], "topk_cluster_rows": buf[2],
+            "topk_cluster_retry": buf[3], "topk_cluster_global": buf[5]}
 
 
 def launch_count() -> int:

@@ -216,32 +216,26 @@ dsa_status run_indexer(const void* qI, const void* kI, const __nv_bfloat16* w, i
 // ------------------------------------------------------------------ top-k launch
 dsa_status run_topk(const float* scores, int64_t ld, int rows, int64_t q_pos0, const int* ctx_len, int64_t n_max,
                     int k, int* idx, cudaStream_t s) {
-    static bool attr_set = false;
-    if (!attr_set) {
-        if (cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(TopkShared)) !=
-            cudaSuccess)
-            return DSA_ERR_CUDA;
-        attr_set = true;
-    }
     TopkParams P{scores, ld, rows, q_pos0, ctx_len, n_max, k, idx};
     const int sms = num_sms();
+    const int smem = (int)sizeof(TopkSmem);
     // Few long rows: a cluster of CTAs per row; otherwise one CTA per row.
-    if ((long long)rows * kTopkCluster <= 2LL * sms && n_max > 4LL * kTopkCap) {
+    if ((long long)rows * kTkCluster <= 2LL * sms && n_max > 4LL * kTkCap) {
         static bool cattr = false;
         if (!cattr) {
-            if (cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     (int)sizeof(TopkShared)) != cudaSuccess)
+            if (cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+                cudaSuccess)
                 return DSA_ERR_CUDA;
             cattr = true;
         }
         cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3(rows * kTopkCluster);
-        cfg.blockDim = dim3(kTopkThreads);
-        cfg.dynamicSmemBytes = sizeof(TopkShared);
+        cfg.gridDim = dim3(rows * kTkCluster);
+        cfg.blockDim = dim3(kTkThreads);
+        cfg.dynamicSmemBytes = smem;
         cfg.stream = s;
         cudaLaunchAttribute attr[1];
         attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = kTopkCluster;
+        attr[0].val.clusterDim.x = kTkCluster;
         attr[0].val.clusterDim.y = 1;
         attr[0].val.clusterDim.z = 1;
         cfg.attrs = attr;
@@ -250,8 +244,14 @@ dsa_status run_topk(const float* scores, int64_t ld, int rows, int64_t q_pos0, c
         if (cudaLaunchKernelEx(&cfg, topk_cluster_kernel, P) != cudaSuccess) return DSA_ERR_CUDA;
         return launch_status();
     }
+    static bool attr_set = false;
+    if (!attr_set) {
+        if (cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+            return DSA_ERR_CUDA;
+        attr_set = true;
+    }
     LaunchScope ls(K_TOPK, s);
-    topk_kernel<<<rows, kTopkThreads, sizeof(TopkShared), s>>>(P);
+    topk_kernel<<<rows, kTkThreads, smem, s>>>(P);
     return launch_status();
 }
 
@@ -622,6 +622,19 @@ dsa_status dsa_profile_end(int64_t* launches, double* total_ms) {
 }
 
 int64_t dsa_launch_count(void) { return g_launches.load(); }
+
+dsa_status dsa_read_counters(int64_t* out, int n, int reset) {
+    if (!out || n < 0 || n > DSA_NUM_COUNTERS) return DSA_ERR_INVALID_ARG;
+    unsigned long long c[DSA_NUM_COUNTERS] = {};
+    if (cudaDeviceSynchronize() != cudaSuccess) return DSA_ERR_CUDA;
+    if (cudaMemcpyFromSymbol(c, g_counters, sizeof(c)) != cudaSuccess) return DSA_ERR_CUDA;
+    for (int i = 0; i < n; ++i) out[i] = (int64_t)c[i];
+    if (reset) {
+        unsigned long long z[DSA_NUM_COUNTERS] = {};
+        if (cudaMemcpyToSymbol(g_counters, z, sizeof(z)) != cudaSuccess) return DSA_ERR_CUDA;
+    }
+    return DSA_OK;
+}
 
 dsa_status dsa_selftest_timeout(int64_t wait_ns, dsa_stream_t stream) {
     if (wait_ns <= 0 || wait_ns > 2000000000ll) return DSA_ERR_INVALID_ARG;

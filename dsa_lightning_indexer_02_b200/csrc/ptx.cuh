@@ -17,6 +17,8 @@ namespace dsa {
 #define DSA_DEV_ERR_BOUNDS 2u
 __device__ unsigned int g_dev_error;
 __device__ unsigned int g_dev_error_where;
+// Path counters for diagnostics, read with dsa_read_counters() (meaning of each slot in dsa.h).
+__device__ unsigned long long g_counters[8];
 
 constexpr unsigned long long kWaitLimitNs = 4000000000ull;  // 4 s per wait
 

@@ -6,20 +6,25 @@
 // training and inference select the same keys (same page, section 八).  This kernel is exact
 // and deterministic: the output of a row depends only on the row's scores.
 //
-// One CTA per row, order-preserving 32-bit keys (larger score -> larger key).
-// Fast path (one HBM read of the row):
-//   sample   256 evenly spaced float4 of the row give an estimate T0 of the key at rank ~2k
-//            (rows with n <= 8192 skip this: T0 = 0 keeps every key);
-//   collect  stream the row once; keys >= T0 are compacted, in index order, into a shared
-//            candidate list through block scans;
-//   refine   if the list holds at least k and at most 8192 keys it contains the exact top-k:
-//            radix rounds over the candidates' offsets from T0 (first round scaled to the key
-//            range, so the bins spread evenly) find the exact k-th key tau and the number of
-//            keys equal to tau to take; an ordered scan emits keys > tau and the first keys
-//            == tau.  Output order: ascending key index.
-// Fallback (the estimate missed): a two-pass radix select over the row -- histogram of the top
-// 12 bits, then keys above the threshold bin are written in index order and the bin's keys are
-// collected (or, past the buffer, re-read from memory) and refined the same way.
+// Scores are compared through an order-preserving map float -> uint32 ("key"; -0 folded onto
+// +0).  One CTA of 4 warps per row (a cluster of CTAs per row when rows are few and long):
+//   sample   ~n/32 scores at evenly spaced float4s give T0, an estimate of the key at rank
+//            1.5k (two 10-bit histogram rounds over the sample keys);
+//   stream   the row is read once; each warp takes every 4th 128-byte piece (so frames of
+//            correlated scores spread evenly over the warps) and compacts the scores >= T0 into
+//            its own shared-memory region with warp-level scans -- no block barrier per load;
+//   refine   if every region fits and the total is >= k, the candidates contain the exact
+//            top-k: radix rounds over the key offsets from T0 (first round scaled to the
+//            candidates' key range) give the exact k-th key tau and the number r of keys equal
+//            to tau to keep;
+//   emit     keys > tau are written region by region; the keys == tau are ranked by index and
+//            the r lowest kept.
+// If the candidates miss the window [k, capacity], the estimate is redone once, aimed using the
+// observed count, and the row streamed again.  Rows that still miss (or where more than 1024
+// keys tie at tau) take an exact radix select over the row itself (10-bit rounds, then one
+// ordered pass): slower, and rare.
+// Output order: keys > tau region by region (each region ascending), then the kept ties
+// ascending.
 #pragma once
 
 #include <cooperative_groups.h>
@@ -28,88 +33,115 @@
 
 namespace dsa {
 
-constexpr int kTopkThreads = 512;
-constexpr int kTopkCap = 8192;   // candidate list capacity (shared memory)
-constexpr int kTopkSampleVec = 256;  // float4 samples per row for the threshold estimate
-constexpr int kTopkUnroll = 4;       // float4 loads in flight per thread
-constexpr int kTopkBins = 4096;
+namespace cg = cooperative_groups;
+
+constexpr int kTkThreads = 128;               // 4 warps per row (per cluster CTA)
+constexpr int kTkWarps = kTkThreads / 32;
+constexpr int kTkBins = 1024;                 // 10-bit radix digits
+constexpr int kTkRegion = 1024;               // candidates per warp region
+constexpr int kTkCap = kTkWarps * kTkRegion;  // 4096 candidates per CTA
+constexpr int kTkMaxSample4 = kTkCap / 4;     // at most 1024 sampled float4 (4096 keys)
+constexpr int kTkUnroll = 8;                  // float4 loads in flight per lane
+constexpr int kTkCluster = 8;                 // CTAs per row in the cluster kernel
+constexpr int kTkMaxRegions = kTkCluster * kTkWarps;
 
 struct TopkParams {
-    const float* scores;     // row r at scores + r*ld (16-byte aligned rows)
+    const float* scores;  // row r at scores + r*ld (16-byte aligned rows)
     long long ld;
     int rows;
-    long long q_pos0;        // prefill: row r has n = q_pos0 + r + 1 keys
-    const int* ctx_len;      // decode: row r has n = ctx_len[r] + 1 keys (null for prefill)
-    long long n_max;         // upper bound on n (keys addressable in a row)
+    long long q_pos0;     // prefill: row r has n = q_pos0 + r + 1 keys
+    const int* ctx_len;   // decode: row r has n = ctx_len[r] + 1 keys (null for prefill)
+    long long n_max;      // upper bound on n (keys addressable in a row)
     int k;
-    int* idx;                // [rows, k]
+    int* idx;             // [rows, k]
 };
 
-// Order-preserving map float -> uint32 (larger float -> larger key); -0 is folded onto +0 so
-// that the two zeros tie exactly as they do in real arithmetic.
+struct TopkSmem {
+    uint32_t hist[kTkBins];
+    uint32_t cand_key[kTkCap];  // also holds the sample keys before streaming
+    int cand_idx[kTkCap];
+    int reg_off[kTkMaxRegions], reg_cnt[kTkMaxRegions], reg_gt[kTkMaxRegions], reg_eq[kTkMaxRegions];
+    int nreg;
+    uint32_t red[kTkWarps];
+    uint32_t sel_bin, sel_gt;
+    uint32_t T0;
+};
+
 __device__ __forceinline__ uint32_t score_key(float f) {
     uint32_t u = __float_as_uint(f);
     if (u == 0x80000000u) u = 0u;
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
+// Smallest float whose key is >= T, so that (f >= key_floor_float(T)) == (score_key(f) >= T).
+__device__ __forceinline__ float key_floor_float(uint32_t T) {
+    if (T == 0u) return -INFINITY;
+    return (T & 0x80000000u) ? __uint_as_float(T & 0x7FFFFFFFu) : __uint_as_float(~T);
+}
 
-struct TopkShared {
-    uint32_t hist[kTopkBins];
-    uint32_t cand_key[kTopkCap];
-    int cand_idx[kTopkCap];
-    uint32_t warp_sum[2][kTopkThreads / 32];
-    uint32_t sel_bin, sel_gt;  // result of a threshold search
-    uint32_t red[kTopkThreads / 32];
-};
+__device__ __forceinline__ long long row_length(const TopkParams& P, int r, bool report) {
+    long long n = P.ctx_len ? (long long)P.ctx_len[r] + 1 : P.q_pos0 + r + 1;
+    if (n > P.n_max || n < 1) {
+        if (report) record_error(DSA_DEV_ERR_BOUNDS, 0x401);
+        n = n < 1 ? 1 : P.n_max;
+    }
+    return n;
+}
 
-// Exclusive prefix sum over the block of a packed counter; returns the block total.  `buf`
-// alternates between calls so that one __syncthreads per scan suffices.
-__device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t& total, uint32_t* warp_sum) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    uint32_t x = v;
+// Inclusive warp prefix sum.
+__device__ __forceinline__ uint32_t warp_incl_scan(uint32_t x) {
+    const int lane = threadIdx.x & 31;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-        uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+        const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
         if (lane >= o) x += y;
     }
-    if (lane == 31) warp_sum[warp] = x;
+    return x;
+}
+
+// Exclusive block prefix sum (4 warps); returns the block total.
+__device__ __forceinline__ uint32_t block_excl_scan(TopkSmem& S, uint32_t v, uint32_t& total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const uint32_t x = warp_incl_scan(v);
+    __syncthreads();
+    if (lane == 31) S.red[warp] = x;
     __syncthreads();
     uint32_t before = 0, tot = 0;
 #pragma unroll
-    for (int w = 0; w < kTopkThreads / 32; ++w) {
-        const uint32_t s = warp_sum[w];
-        before += (w < warp) ? s : 0u;
-        tot += s;
+    for (int w = 0; w < kTkWarps; ++w) {
+        before += (w < warp) ? S.red[w] : 0u;
+        tot += S.red[w];
     }
     total = tot;
     return before + x - v;
 }
 
-// Find bin b with (count of bins above b) < need <= (count above b) + hist[b].  Bins [0, nbins).
-__device__ __forceinline__ void find_threshold_bin(TopkShared& S, int nbins, uint32_t need, int& scan_buf) {
-    const int per = nbins >= kTopkThreads ? nbins / kTopkThreads : 1;
+// Bin b of S.hist[0, nbins) with (count above b) < need <= (count above b) + hist[b]; result in
+// S.sel_bin / S.sel_gt.  nbins <= kTkBins; needs the histogram total >= need.
+__device__ __forceinline__ void find_threshold_bin(TopkSmem& S, int nbins, uint32_t need) {
+    constexpr int kMaxPer = kTkBins / kTkThreads;
+    const int per = (nbins + kTkThreads - 1) / kTkThreads;
     const int lo = threadIdx.x * per;
     uint32_t mine = 0;
-    if (lo < nbins)
-        for (int b = 0; b < per; ++b) mine += S.hist[lo + b];
-    // suffix sums: scan on reversed thread order
+#pragma unroll
+    for (int b = 0; b < kMaxPer; ++b)
+        if (b < per && lo + b < nbins) mine += S.hist[lo + b];
+    // suffix sums over threads (a higher thread owns higher bins)
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     uint32_t x = mine;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-        uint32_t y = __shfl_down_sync(0xffffffffu, x, o);
+        const uint32_t y = __shfl_down_sync(0xffffffffu, x, o);
         if (lane + o < 32) x += y;
     }
-    uint32_t* ws = S.warp_sum[scan_buf];
-    scan_buf ^= 1;
-    if (lane == 0) ws[warp] = x;
     __syncthreads();
-    uint32_t above = x - mine;  // bins of later lanes in this warp
+    if (lane == 0) S.red[warp] = x;
+    __syncthreads();
+    uint32_t above = x - mine;
 #pragma unroll
-    for (int w = 0; w < kTopkThreads / 32; ++w) above += (w > warp) ? ws[w] : 0u;
+    for (int w = 0; w < kTkWarps; ++w) above += (w > warp) ? S.red[w] : 0u;
     if (lo < nbins && above < need && need <= above + mine) {
         uint32_t cum = above;
-        for (int b = lo + per - 1; b >= lo; --b) {
+        for (int b = min(lo + per, nbins) - 1; b >= lo; --b) {
             const uint32_t h = S.hist[b];
             if (cum + h >= need) {
                 S.sel_bin = (uint32_t)b;
@@ -122,454 +154,397 @@ __device__ __forceinline__ void find_threshold_bin(TopkShared& S, int nbins, uin
     __syncthreads();
 }
 
-__device__ __forceinline__ void clear_hist(TopkShared& S, int nbins) {
-    for (int b = threadIdx.x; b < nbins; b += kTopkThreads) S.hist[b] = 0;
+__device__ __forceinline__ void clear_hist(TopkSmem& S, int nbins) {
+    for (int b = threadIdx.x; b < nbins; b += kTkThreads) S.hist[b] = 0;
 }
 
-// Items of a refinement round: either the shared-memory candidate list or the global row
-// filtered to the threshold bin of pass 1.
-struct CandSource {
-    const TopkShared* S;
-    int m;
-    __device__ __forceinline__ int count() const { return m; }
-    __device__ __forceinline__ bool get(int e, uint32_t& key, int& idx) const {
-        if (e >= m) return false;
-        key = S->cand_key[e];
-        idx = S->cand_idx[e];
-        return true;
-    }
-};
-struct RowSource {
-    const float* row;
-    int n;
-    uint32_t b0;
-    __device__ __forceinline__ int count() const { return n; }
-    __device__ __forceinline__ bool get(int e, uint32_t& key, int& idx) const {
-        if (e >= n) return false;
-        key = score_key(row[e]);
-        idx = e;
-        return (key >> 20) == b0;
-    }
-};
-
-template <class Src>
-__device__ __forceinline__ void refine_round(TopkShared& S, const Src& src, int shift, int width, uint32_t pmask,
-                                             uint32_t pval, uint32_t& need, uint32_t& out_bin, int& scan_buf) {
-    const int nbins = 1 << width;
-    clear_hist(S, nbins);
+// T0 from m sample keys in S.cand_key[0, m): the key at rank rs, truncated to its top 20 bits
+// (two 10-bit rounds).  Every sample key >= T0 is counted, so at least rs samples are >= T0.
+__device__ __forceinline__ uint32_t sample_threshold(TopkSmem& S, int m, uint32_t rs) {
+    clear_hist(S, kTkBins);
     __syncthreads();
-    for (int e = threadIdx.x; e < src.count(); e += kTopkThreads) {
-        uint32_t key;
-        int idx;
-        if (src.get(e, key, idx) && (key & pmask) == pval) atomicAdd(&S.hist[(key >> shift) & (nbins - 1)], 1u);
+    for (int e = threadIdx.x; e < m; e += kTkThreads) atomicAdd(&S.hist[S.cand_key[e] >> 22], 1u);
+    __syncthreads();
+    find_threshold_bin(S, kTkBins, rs);
+    const uint32_t b1 = S.sel_bin, need = rs - S.sel_gt;
+    clear_hist(S, kTkBins);
+    __syncthreads();
+    for (int e = threadIdx.x; e < m; e += kTkThreads) {
+        const uint32_t key = S.cand_key[e];
+        if ((key >> 22) == b1) atomicAdd(&S.hist[(key >> 12) & 0x3FF], 1u);
     }
     __syncthreads();
-    find_threshold_bin(S, nbins, need, scan_buf);
-    out_bin = S.sel_bin;
-    need -= S.sel_gt;
+    find_threshold_bin(S, kTkBins, need);
+    return (b1 << 22) | (S.sel_bin << 12);
 }
 
-// Emit, in source order, items with key > tau and the first `ties` items with key == tau.
-template <class Src>
-__device__ __forceinline__ void emit_final(TopkShared& S, const Src& src, uint32_t tau, uint32_t ties, int* out,
-                                           uint32_t out_base, int& scan_buf) {
-    uint32_t gt_seen = 0, eq_seen = 0;
-    const int cnt = src.count();
-    for (int e0 = 0; e0 < cnt; e0 += kTopkThreads) {
-        const int e = e0 + threadIdx.x;
-        uint32_t key = 0;
-        int idx = 0;
-        const bool in = src.get(e, key, idx);
-        const uint32_t gt = (in && key > tau) ? 1u : 0u;
-        const uint32_t eq = (in && key == tau) ? 1u : 0u;
-        uint32_t total;
-        const uint32_t ex = block_excl_scan(gt | (eq << 16), total, S.warp_sum[scan_buf]);
-        scan_buf ^= 1;
-        const uint32_t eq_before = eq_seen + (ex >> 16);
-        if (gt || (eq && eq_before < ties)) {
-            const uint32_t pos = out_base + gt_seen + (ex & 0xFFFFu) + min(eq_before, ties);
-            out[pos] = idx;
+// Stream float4 groups [g_lo, g_hi) of a row with n valid scores and compact the scores >= F0
+// into this warp's region, in index order.  Warp w takes the 128-byte pieces p with p % 4 == w.
+// Returns how many scores of this warp qualified (may exceed the region; the excess is dropped).
+__device__ __forceinline__ uint32_t stream_collect(TopkSmem& S, const float4* row4, int g_lo, int g_hi, int n,
+                                                   float F0, int region_base) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    // float4 offset inside a 128-float4 round: piece (lane/8)*4 + warp, float4 lane%8 of it
+    const int lane_off = (lane >> 3) * 32 + warp * 8 + (lane & 7);
+    uint32_t cnt = 0;
+    for (int g0 = g_lo; g0 < g_hi; g0 += kTkUnroll * 128) {
+        float4 v[kTkUnroll];
+#pragma unroll
+        for (int u = 0; u < kTkUnroll; ++u) {
+            const int g = g0 + u * 128 + lane_off;
+            v[u] = g < g_hi ? __ldcs(row4 + g) : make_float4(0.f, 0.f, 0.f, 0.f);
         }
+#pragma unroll
+        for (int u = 0; u < kTkUnroll; ++u) {
+            const int g = g0 + u * 128 + lane_off;
+            const float f[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+            uint32_t mask = 0;
+            if (g < g_hi) {
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    if (f[j] >= F0 && g * 4 + j < n) mask |= 1u << j;
+            }
+            const uint32_t c = __popc(mask);
+            const uint32_t incl = warp_incl_scan(c);
+            if (mask) {
+                uint32_t pos = cnt + incl - c;
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    if (mask & (1u << j)) {
+                        if (pos < (uint32_t)kTkRegion) {
+                            S.cand_key[region_base + pos] = score_key(f[j]);
+                            S.cand_idx[region_base + pos] = g * 4 + j;
+                        }
+                        ++pos;
+                    }
+            }
+            cnt += __shfl_sync(0xffffffffu, incl, 31);
+        }
+    }
+    return cnt;
+}
+
+// Exact top-k among the candidates in S's regions (every candidate key >= lo; their total is
+// >= k and includes every key of the row >= lo).  Returns false, writing nothing, when more
+// than kTkBins keys tie at the k-th key.
+__device__ __forceinline__ bool refine_and_emit(TopkSmem& S, uint32_t lo, int k, int* out) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int nreg = S.nreg;
+    uint32_t mx = 0;
+    for (int r = 0; r < nreg; ++r)
+        for (int e = tid; e < S.reg_cnt[r]; e += kTkThreads) mx = max(mx, S.cand_key[S.reg_off[r] + e] - lo);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    __syncthreads();
+    if (lane == 0) S.red[warp] = mx;
+    __syncthreads();
+    uint32_t R = 0;
+#pragma unroll
+    for (int w = 0; w < kTkWarps; ++w) R = max(R, S.red[w]);
+    int fixed = R ? 32 - __clz(R) : 0;  // every offset is < 2^fixed
+    uint32_t pv = 0, need = (uint32_t)k, T = 0;
+    if (fixed == 0) {
+        for (int r = 0; r < nreg; ++r) T += (uint32_t)S.reg_cnt[r];  // all candidates share one key
+    }
+    while (fixed > 0) {
+        const int sh = fixed > 10 ? fixed - 10 : 0;
+        const int nbins = 1 << (fixed - sh);
+        __syncthreads();
+        clear_hist(S, nbins);
+        __syncthreads();
+        for (int r = 0; r < nreg; ++r)
+            for (int e = tid; e < S.reg_cnt[r]; e += kTkThreads) {
+                const uint32_t d = S.cand_key[S.reg_off[r] + e] - lo;
+                const bool match = fixed >= 32 ? true : ((d >> fixed) == (pv >> fixed));
+                if (match) atomicAdd(&S.hist[(d >> sh) & (nbins - 1)], 1u);
+            }
+        __syncthreads();
+        find_threshold_bin(S, nbins, need);
+        need -= S.sel_gt;
+        T = S.hist[S.sel_bin];  // after the last round (sh == 0) a bin is a single key
+        pv |= S.sel_bin << sh;
+        fixed = sh;
+    }
+    __syncthreads();
+    const uint32_t tau = lo + pv;
+    const uint32_t ties = need;  // 1 <= ties <= T
+    if (T > (uint32_t)kTkBins && T != ties) return false;
+    // per-region counts of keys > tau and == tau
+    for (int r = warp; r < nreg; r += kTkWarps) {
+        uint32_t gt = 0, eq = 0;
+        for (int e = lane; e < S.reg_cnt[r]; e += 32) {
+            const uint32_t key = S.cand_key[S.reg_off[r] + e];
+            gt += key > tau;
+            eq += key == tau;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            gt += __shfl_xor_sync(0xffffffffu, gt, o);
+            eq += __shfl_xor_sync(0xffffffffu, eq, o);
+        }
+        if (lane == 0) S.reg_gt[r] = (int)gt, S.reg_eq[r] = (int)eq;
+    }
+    __syncthreads();
+    uint32_t* tie_idx = S.hist;  // reused: up to kTkBins tie indices
+    for (int r = warp; r < nreg; r += kTkWarps) {
+        uint32_t gbase = 0, ebase = 0;
+        for (int q = 0; q < r; ++q) gbase += (uint32_t)S.reg_gt[q], ebase += (uint32_t)S.reg_eq[q];
+        for (int e0 = 0; e0 < S.reg_cnt[r]; e0 += 32) {
+            const int e = e0 + lane;
+            const bool in = e < S.reg_cnt[r];
+            const uint32_t key = in ? S.cand_key[S.reg_off[r] + e] : 0u;
+            const int ix = in ? S.cand_idx[S.reg_off[r] + e] : 0;
+            const bool gt = in && key > tau, eq = in && key == tau;
+            const uint32_t bg = __ballot_sync(0xffffffffu, gt), be = __ballot_sync(0xffffffffu, eq);
+            const uint32_t below = (1u << lane) - 1u;
+            if (gt) out[gbase + __popc(bg & below)] = ix;
+            if (eq) {
+                const uint32_t p = ebase + __popc(be & below);
+                if (T == ties) out[(uint32_t)k - ties + p] = ix;
+                else tie_idx[p] = (uint32_t)ix;
+            }
+            gbase += __popc(bg);
+            ebase += __popc(be);
+        }
+    }
+    if (T != ties) {
+        // the `ties` lowest indices among the T tied keys, ascending
+        __syncthreads();
+        for (uint32_t a = tid; a < T; a += kTkThreads) {
+            const uint32_t ia = tie_idx[a];
+            uint32_t rank = 0;
+            for (uint32_t b = 0; b < T; ++b) rank += tie_idx[b] < ia;
+            if (rank < ties) out[(uint32_t)k - ties + rank] = (int)ia;
+        }
+    }
+    return true;
+}
+
+// Exact radix select over the row in global memory (the fallback): histogram passes of
+// 10 + 10 + 10 + 2 bits fix tau and the number of ties to keep, then one ordered pass writes
+// keys > tau and the lowest-index ties, ascending.
+__device__ __noinline__ void topk_global(TopkSmem& S, const float* row, int n, int k, int* out) {
+    const int tid = threadIdx.x;
+    uint32_t pval = 0, need = (uint32_t)k;
+    int fixed = 32;
+    while (fixed > 0) {
+        const int width = fixed >= 10 ? 10 : fixed;
+        const int sh = fixed - width;
+        const int nbins = 1 << width;
+        __syncthreads();
+        clear_hist(S, nbins);
+        __syncthreads();
+        for (int e = tid; e < n; e += kTkThreads) {
+            const uint32_t key = score_key(row[e]);
+            if (fixed >= 32 || (key >> fixed) == (pval >> fixed)) atomicAdd(&S.hist[(key >> sh) & (nbins - 1)], 1u);
+        }
+        __syncthreads();
+        find_threshold_bin(S, nbins, need);
+        need -= S.sel_gt;
+        pval |= S.sel_bin << sh;
+        fixed = sh;
+    }
+    const uint32_t tau = pval, ties = need;
+    uint32_t gt_seen = 0, eq_seen = 0;
+    for (int e0 = 0; e0 < n; e0 += kTkThreads) {
+        const int e = e0 + tid;
+        const uint32_t key = e < n ? score_key(row[e]) : 0u;
+        const uint32_t gt = (e < n && key > tau) ? 1u : 0u;
+        const uint32_t eq = (e < n && key == tau) ? 1u : 0u;
+        uint32_t total;
+        const uint32_t ex = block_excl_scan(S, gt | (eq << 16), total);
+        const uint32_t eq_before = eq_seen + (ex >> 16);
+        if (gt || (eq && eq_before < ties)) out[gt_seen + (ex & 0xFFFFu) + min(eq_before, ties)] = e;
         gt_seen += total & 0xFFFFu;
         eq_seen += total >> 16;
     }
 }
 
-// Two-pass radix select over the global row (the fallback path).
-__device__ __noinline__ void topk_two_pass(TopkShared& S, const float* row, int n, int k, int* out, int& scan_buf) {
-    const int tid = threadIdx.x;
-    const float4* row4 = reinterpret_cast<const float4*>(row);
-    // ---- pass 1: histogram of the top 12 key bits
-    clear_hist(S, kTopkBins);
-    __syncthreads();
-    const int n4 = (n + 3) >> 2;
-    for (int g = tid; g < n4; g += kTopkThreads) {
-        const float4 v = row4[g];
-        const int e = g * 4;
-        atomicAdd(&S.hist[score_key(v.x) >> 20], 1u);
-        if (e + 1 < n) atomicAdd(&S.hist[score_key(v.y) >> 20], 1u);
-        if (e + 2 < n) atomicAdd(&S.hist[score_key(v.z) >> 20], 1u);
-        if (e + 3 < n) atomicAdd(&S.hist[score_key(v.w) >> 20], 1u);
-    }
-    __syncthreads();
-    find_threshold_bin(S, kTopkBins, (uint32_t)k, scan_buf);
-    const uint32_t b0 = S.sel_bin;
-    const uint32_t gt0 = S.sel_gt;  // keys strictly above bin b0 (< k)
+__device__ __forceinline__ uint32_t rank_target(long long m, long long n, int k) {
+    // aim at rank 1.5k of the row, i.e. rank 1.5k * m / n of the m samples
+    return (uint32_t)max(1LL, min(m - 1, (3LL * k * m + 2LL * n - 1) / (2LL * n)));
+}
 
-    // ---- pass 2: emit keys above b0, collect candidates inside b0 (both in index order)
-    uint32_t sel_base = 0, cand_base = 0;
-    for (int g0 = 0; g0 < n4; g0 += kTopkThreads) {
-        const int g = g0 + tid;
-        uint32_t key[4] = {0, 0, 0, 0};
-        uint32_t nsel = 0, ncand = 0, selmask = 0, candmask = 0;
-        if (g < n4) {
-            const float4 v = __ldcs(row4 + g);
+// Sample s4 evenly spaced float4 of float4 range [g_lo, g_hi) into keys[base .. base + 4*s4).
+__device__ __forceinline__ void take_samples(uint32_t* keys, int base, const float4* row4, int g_lo, int g_hi, int n,
+                                             int s4) {
+    for (int i = threadIdx.x; i < s4; i += kTkThreads) {
+        const int g = g_lo + (int)(((long long)i * (g_hi - g_lo)) / s4);
+        uint32_t kk[4] = {0u, 0u, 0u, 0u};
+        if (g < g_hi) {
+            const float4 v = row4[g];
             const float f[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                if (g * 4 + j < n) {
-                    key[j] = score_key(f[j]);
-                    const uint32_t d = key[j] >> 20;
-                    if (d > b0) { selmask |= 1u << j; ++nsel; }
-                    else if (d == b0) { candmask |= 1u << j; ++ncand; }
-                }
-            }
+            for (int j = 0; j < 4; ++j) kk[j] = g * 4 + j < n ? score_key(f[j]) : 0u;
         }
-        uint32_t total;
-        const uint32_t ex = block_excl_scan(nsel | (ncand << 16), total, S.warp_sum[scan_buf]);
-        scan_buf ^= 1;
-        uint32_t ps = sel_base + (ex & 0xFFFFu), pc = cand_base + (ex >> 16);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            if (selmask & (1u << j)) out[ps++] = g * 4 + j;
-            if (candmask & (1u << j)) {
-                if (pc < (uint32_t)kTopkCap) {
-                    S.cand_key[pc] = key[j];
-                    S.cand_idx[pc] = g * 4 + j;
-                }
-                ++pc;
-            }
-        }
-        sel_base += total & 0xFFFFu;
-        cand_base += total >> 16;
-    }
-    __syncthreads();
-
-    // ---- refine inside bin b0: 12 more bits, then the last 8 bits
-    uint32_t need = (uint32_t)k - gt0;
-    uint32_t b1, b2;
-    const uint32_t p0 = b0 << 20;
-    if (cand_base <= (uint32_t)kTopkCap) {
-        const CandSource src{&S, (int)cand_base};
-        refine_round(S, src, 8, 12, 0xFFF00000u, p0, need, b1, scan_buf);
-        refine_round(S, src, 0, 8, 0xFFFFFF00u, p0 | (b1 << 8), need, b2, scan_buf);
-        emit_final(S, src, p0 | (b1 << 8) | b2, need, out, gt0, scan_buf);
-    } else {
-        const RowSource src{row, n, b0};
-        refine_round(S, src, 8, 12, 0xFFF00000u, p0, need, b1, scan_buf);
-        refine_round(S, src, 0, 8, 0xFFFFFF00u, p0 | (b1 << 8), need, b2, scan_buf);
-        emit_final(S, src, p0 | (b1 << 8) | b2, need, out, gt0, scan_buf);
+        for (int j = 0; j < 4; ++j) keys[base + 4 * i + j] = kk[j];
     }
 }
 
-// Block-wide max of a uint32.
-__device__ __forceinline__ uint32_t block_max_u32(TopkShared& S, uint32_t v) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v = max(v, __shfl_xor_sync(0xffffffffu, v, o));
-    __syncthreads();
-    if (lane == 0) S.red[warp] = v;
-    __syncthreads();
-    uint32_t m = 0;
-#pragma unroll
-    for (int w = 0; w < kTopkThreads / 32; ++w) m = max(m, S.red[w]);
-    return m;
+__device__ __forceinline__ int sample_count4(int n4, int parts) {
+    return min(kTkMaxSample4, max(256, n4 / 8)) / parts;  // ~n/32 scores in all
 }
 
-// Exact top-k among the m <= kTopkCap candidates (all keys >= lo), emitted in candidate order.
-__device__ __forceinline__ void refine_candidates(TopkShared& S, int m, uint32_t lo, int k, int* out, int& scan_buf) {
-    uint32_t kmax = 0;
-    for (int e = threadIdx.x; e < m; e += kTopkThreads) kmax = max(kmax, S.cand_key[e] - lo);
-    const uint32_t R = block_max_u32(S, kmax);
-    int fixed = R ? 32 - __clz(R) : 0;   // offsets are < 2^fixed; bits >= fixed are all zero
-    uint32_t pv = 0, need = (uint32_t)k;
-    while (fixed > 0) {
-        const int sh = fixed > 12 ? fixed - 12 : 0;
-        const int width = fixed - sh;
-        const int nbins = 1 << width;
-        clear_hist(S, nbins);
-        __syncthreads();
-        for (int e = threadIdx.x; e < m; e += kTopkThreads) {
-            const uint32_t d = S.cand_key[e] - lo;
-            const bool match = fixed >= 32 ? true : ((d >> fixed) == (pv >> fixed));
-            if (match) atomicAdd(&S.hist[(d >> sh) & (nbins - 1)], 1u);
-        }
-        __syncthreads();
-        find_threshold_bin(S, nbins, need, scan_buf);
-        need -= S.sel_gt;
-        pv |= S.sel_bin << sh;
-        fixed = sh;
-    }
-    const CandSource src{&S, m};
-    emit_final(S, src, lo + pv, need, out, 0u, scan_buf);
+// Second aim after a miss: the observed count c at rank rs scales about linearly with the rank.
+__device__ __forceinline__ uint32_t retarget(uint32_t rs, uint32_t c, long long m, int k) {
+    const long long want = (3LL * k) / 2;
+    const long long r2 = ((long long)rs * want + (c > 0 ? c : 1) - 1) / (c > 0 ? (long long)c : 1LL);
+    return (uint32_t)max(1LL, min(m - 1, r2));
 }
 
-__global__ void __launch_bounds__(kTopkThreads) topk_kernel(const TopkParams P) {
+__global__ void __launch_bounds__(kTkThreads) topk_kernel(const TopkParams P) {
     extern __shared__ __align__(1024) uint8_t topk_smem[];
-    TopkShared& S = *reinterpret_cast<TopkShared*>(topk_smem);
-    const int r = blockIdx.x;
-    const int tid = threadIdx.x;
-    long long n_ll = P.ctx_len ? (long long)P.ctx_len[r] + 1 : P.q_pos0 + r + 1;
-    if (n_ll > P.n_max || n_ll < 1) {
-        if (tid == 0) record_error(DSA_DEV_ERR_BOUNDS, 0x401);
-        n_ll = n_ll < 1 ? 1 : P.n_max;
-    }
-    const int n = (int)n_ll;
+    TopkSmem& S = *reinterpret_cast<TopkSmem*>(topk_smem);
+    const int r = blockIdx.x, tid = threadIdx.x, warp = tid >> 5;
+    const int n = (int)row_length(P, r, tid == 0);
     const int k = P.k;
     int* out = P.idx + (long long)r * k;
     if (n <= k) {
-        for (int j = tid; j < k; j += kTopkThreads) out[j] = j < n ? j : -1;
+        for (int j = tid; j < k; j += kTkThreads) out[j] = j < n ? j : -1;
         return;
     }
     const float* row = P.scores + (long long)r * P.ld;
     const float4* row4 = reinterpret_cast<const float4*>(row);
     const int n4 = (n + 3) >> 2;
-    int scan_buf = 0;
-
-    // ---- threshold estimate T0 from a sample (two 12-bit histogram rounds over ~1024 keys)
-    uint32_t T0 = 0;
-    if (n > kTopkCap) {
-        uint32_t sk[4] = {0, 0, 0, 0};
-        int sv = 0;
-        if (tid < kTopkSampleVec) {
-            const int g = (int)(((long long)tid * n4) / kTopkSampleVec);
-            const float4 v = row4[g];
-            const float f[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-                if (g * 4 + j < n) sk[j] = score_key(f[j]), sv |= 1 << j;
+    const int s4 = sample_count4(n4, 1);
+    const long long m = 4LL * s4;
+    uint32_t rs = (uint32_t)rank_target(m, n, k);
+    bool done = false;
+    for (int attempt = 0; attempt < 2 && !done; ++attempt) {
+        // ---- threshold estimate (rows of up to kTkCap scores keep them all)
+        uint32_t T0 = 0;
+        if (n > kTkCap) {
+            if (attempt > 0) __syncthreads();
+            take_samples(S.cand_key, 0, row4, 0, n4, n, s4);
+            T0 = sample_threshold(S, (int)m, rs);
         }
-        clear_hist(S, kTopkBins);
-        __syncthreads();
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-            if (sv & (1 << j)) atomicAdd(&S.hist[sk[j] >> 20], 1u);
-        __syncthreads();
-        // aim at rank 2k of the row: r_s = 2k * m / n of the ~m = 4*256 samples
-        const uint32_t rs = (uint32_t)min(4LL * kTopkSampleVec - 1,
-                                          (2LL * k * 4 * kTopkSampleVec + n - 1) / n);
-        find_threshold_bin(S, kTopkBins, rs, scan_buf);
-        const uint32_t b = S.sel_bin, need2 = rs - S.sel_gt;
-        clear_hist(S, kTopkBins);
-        __syncthreads();
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-            if ((sv & (1 << j)) && (sk[j] >> 20) == b) atomicAdd(&S.hist[(sk[j] >> 8) & 0xFFF], 1u);
-        __syncthreads();
-        find_threshold_bin(S, kTopkBins, need2, scan_buf);
-        T0 = (b << 20) | (S.sel_bin << 8);
-    }
-
-    // ---- single streaming pass: compact keys >= T0 in index order
-    uint32_t cbase = 0;
-    for (int g0 = 0; g0 < n4; g0 += kTopkUnroll * kTopkThreads) {
-        float4 v[kTopkUnroll];
-#pragma unroll
-        for (int u = 0; u < kTopkUnroll; ++u) {
-            const int g = g0 + u * kTopkThreads + tid;
-            v[u] = g < n4 ? __ldcs(row4 + g) : make_float4(0.f, 0.f, 0.f, 0.f);
+        // ---- one streaming pass: scores >= T0 into the 4 warp regions
+        const uint32_t c = stream_collect(S, row4, 0, n4, n, key_floor_float(T0), warp * kTkRegion);
+        if ((tid & 31) == 0) {
+            S.reg_off[warp] = warp * kTkRegion;
+            S.reg_cnt[warp] = (int)min(c, (uint32_t)kTkRegion);
+            S.reg_gt[warp] = (int)c;
         }
+        if (tid == 0) S.nreg = kTkWarps;
+        __syncthreads();
+        uint32_t total = 0;
+        bool fits = true;
 #pragma unroll
-        for (int u = 0; u < kTopkUnroll; ++u) {
-            const int g = g0 + u * kTopkThreads + tid;
-            const float f[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-            uint32_t key[4], mask = 0, cnt = 0;
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                key[j] = score_key(f[j]);
-                if (g * 4 + j < n && key[j] >= T0) mask |= 1u << j, ++cnt;
-            }
-            uint32_t total;
-            const uint32_t ex = block_excl_scan(cnt, total, S.warp_sum[scan_buf]);
-            scan_buf ^= 1;
-            uint32_t pos = cbase + ex;
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-                if (mask & (1u << j)) {
-                    if (pos < (uint32_t)kTopkCap) {
-                        S.cand_key[pos] = key[j];
-                        S.cand_idx[pos] = g * 4 + j;
-                    }
-                    ++pos;
-                }
-            cbase += total;
-            if (g0 + (u + 1) * kTopkThreads >= n4) break;  // uniform across the block
+        for (int w = 0; w < kTkWarps; ++w) {
+            total += (uint32_t)S.reg_gt[w];
+            fits = fits && S.reg_gt[w] <= kTkRegion;
+        }
+        fits = fits && total >= (uint32_t)k;
+        done = fits && refine_and_emit(S, T0, k, out);
+        if (!done) rs = retarget(rs, total, m, k);
+        if (tid == 0) {
+            atomicAdd(&g_counters[0], attempt == 0 ? 1ull : 0ull);
+            if (!done) atomicAdd(&g_counters[1 + 3 * attempt], 1ull);  // [1] first miss, [4] second miss
         }
     }
-    __syncthreads();
-    if (cbase >= (uint32_t)k && cbase <= (uint32_t)kTopkCap) {
-        refine_candidates(S, (int)cbase, T0, k, out, scan_buf);
-    } else {
-        topk_two_pass(S, row, n, k, out, scan_buf);
-    }
+    if (!done) topk_global(S, row, n, k, out);
 }
 
-// ---------------------------------------------------------------------------------------------
-// Few long rows (decode: B rows of ~131K keys): a cluster of kTopkCluster CTAs shares one row.
-// Each CTA samples and streams 1/kTopkCluster of the row; the sample histograms are summed and
-// the per-CTA candidate lists are gathered through distributed shared memory, so the row is
-// still read once from HBM but by kTopkCluster SMs.  CTA 0 of the cluster refines and writes
-// the row (or, if the estimate missed, runs the two-pass fallback over the whole row).
-constexpr int kTopkCluster = 8;
-
-namespace cg = cooperative_groups;
-
-// Sum the histograms of every CTA of the cluster into `merged` (a local array).
-__device__ __forceinline__ void cluster_merge_hist(TopkShared& S, uint32_t* merged) {
-    cg::cluster_group cluster = cg::this_cluster();
-    for (int b = threadIdx.x; b < kTopkBins; b += kTopkThreads) {
-        uint32_t sum = 0;
-#pragma unroll
-        for (int c = 0; c < kTopkCluster; ++c) sum += cluster.map_shared_rank(S.hist, c)[b];
-        merged[b] = sum;
-    }
-}
-
-__global__ void __launch_bounds__(kTopkThreads) topk_cluster_kernel(const TopkParams P) {
+// Few long rows (decode): a cluster of kTkCluster CTAs per row.  Each CTA samples and streams
+// 1/kTkCluster of the row; the sample keys and the candidate regions meet in CTA 0 through
+// distributed shared memory; CTA 0 refines and writes the row.
+__global__ void __launch_bounds__(kTkThreads) topk_cluster_kernel(const TopkParams P) {
     extern __shared__ __align__(1024) uint8_t topk_smem[];
-    TopkShared& S = *reinterpret_cast<TopkShared*>(topk_smem);
+    __shared__ int src_cnt[kTkMaxRegions];
+    TopkSmem& S = *reinterpret_cast<TopkSmem*>(topk_smem);
     cg::cluster_group cluster = cg::this_cluster();
     const int crank = (int)cluster.block_rank();
-    const int r = blockIdx.x / kTopkCluster;
-    const int tid = threadIdx.x;
-    long long n_ll = P.ctx_len ? (long long)P.ctx_len[r] + 1 : P.q_pos0 + r + 1;
-    if (n_ll > P.n_max || n_ll < 1) {
-        if (tid == 0 && crank == 0) record_error(DSA_DEV_ERR_BOUNDS, 0x402);
-        n_ll = n_ll < 1 ? 1 : P.n_max;
-    }
-    const int n = (int)n_ll;
+    const int r = blockIdx.x / kTkCluster, tid = threadIdx.x, warp = tid >> 5;
+    const int n = (int)row_length(P, r, tid == 0 && crank == 0);
     const int k = P.k;
     int* out = P.idx + (long long)r * k;
     if (n <= k) {  // uniform over the cluster
         if (crank == 0)
-            for (int j = tid; j < k; j += kTopkThreads) out[j] = j < n ? j : -1;
+            for (int j = tid; j < k; j += kTkThreads) out[j] = j < n ? j : -1;
         return;
     }
     const float* row = P.scores + (long long)r * P.ld;
     const float4* row4 = reinterpret_cast<const float4*>(row);
     const int n4 = (n + 3) >> 2;
-    const int seg = (n4 + kTopkCluster - 1) / kTopkCluster;
+    const int seg = (n4 + kTkCluster - 1) / kTkCluster;
     const int g_lo = min(n4, crank * seg), g_hi = min(n4, g_lo + seg);
-    int scan_buf = 0;
-    uint32_t* merged = S.cand_key;  // scratch until candidates are collected
+    TopkSmem* S0 = cluster.map_shared_rank(&S, 0);
 
-    // ---- threshold estimate over the whole row from kTopkSampleVec float4 samples
-    constexpr int kPer = kTopkSampleVec / kTopkCluster;
-    uint32_t sk[4] = {0, 0, 0, 0};
-    int sv = 0;
-    if (tid < kPer) {
-        const int gi = crank * kPer + tid;
-        const int g = (int)(((long long)gi * n4) / kTopkSampleVec);
-        const float4 v = row4[g];
-        const float f[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-            if (g * 4 + j < n) sk[j] = score_key(f[j]), sv |= 1 << j;
-    }
-    clear_hist(S, kTopkBins);
-    __syncthreads();
-#pragma unroll
-    for (int j = 0; j < 4; ++j)
-        if (sv & (1 << j)) atomicAdd(&S.hist[sk[j] >> 20], 1u);
-    cluster.sync();
-    cluster_merge_hist(S, merged);
-    cluster.sync();  // every CTA has read every histogram
-    for (int b = tid; b < kTopkBins; b += kTopkThreads) S.hist[b] = merged[b];
-    __syncthreads();
-    const uint32_t rs = (uint32_t)min(4LL * kTopkSampleVec - 1, (2LL * k * 4 * kTopkSampleVec + n - 1) / n);
-    find_threshold_bin(S, kTopkBins, rs, scan_buf);
-    const uint32_t b = S.sel_bin, need2 = rs - S.sel_gt;
-    __syncthreads();
-    clear_hist(S, kTopkBins);
-    __syncthreads();
-#pragma unroll
-    for (int j = 0; j < 4; ++j)
-        if ((sv & (1 << j)) && (sk[j] >> 20) == b) atomicAdd(&S.hist[(sk[j] >> 8) & 0xFFF], 1u);
-    cluster.sync();
-    cluster_merge_hist(S, merged);
-    cluster.sync();
-    for (int bb = tid; bb < kTopkBins; bb += kTopkThreads) S.hist[bb] = merged[bb];
-    __syncthreads();
-    find_threshold_bin(S, kTopkBins, need2, scan_buf);
-    const uint32_t T0 = (b << 20) | (S.sel_bin << 8);
-    __syncthreads();
-
-    // ---- stream this CTA's segment, compact keys >= T0 (index order) into the local list
-    uint32_t cbase = 0;
-    for (int g0 = g_lo; g0 < g_hi; g0 += kTopkUnroll * kTopkThreads) {
-        float4 v[kTopkUnroll];
-#pragma unroll
-        for (int u = 0; u < kTopkUnroll; ++u) {
-            const int g = g0 + u * kTopkThreads + tid;
-            v[u] = g < g_hi ? __ldcs(row4 + g) : make_float4(0.f, 0.f, 0.f, 0.f);
+    const int s4 = sample_count4(n4, kTkCluster);  // per CTA
+    const long long m = 4LL * s4 * kTkCluster;
+    uint32_t rs = (uint32_t)rank_target(m, n, k);
+    bool done = false;
+    for (int attempt = 0; attempt < 2; ++attempt) {
+        // ---- samples of every segment into CTA 0, which computes T0 and hands it to every CTA
+        take_samples(S0->cand_key, 4 * crank * s4, row4, g_lo, g_hi, n, s4);
+        cluster.sync();
+        if (crank == 0) {
+            const uint32_t t0 = sample_threshold(S, (int)m, rs);
+            if (tid < kTkCluster) cluster.map_shared_rank(&S, tid)->T0 = t0;
         }
-#pragma unroll
-        for (int u = 0; u < kTopkUnroll; ++u) {
-            const int g = g0 + u * kTopkThreads + tid;
-            const float f[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-            uint32_t key[4], mask = 0, cnt = 0;
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                key[j] = score_key(f[j]);
-                if (g < g_hi && g * 4 + j < n && key[j] >= T0) mask |= 1u << j, ++cnt;
+        cluster.sync();
+        const uint32_t T0 = S.T0;
+
+        // ---- stream this CTA's segment into its warp regions
+        const uint32_t c = stream_collect(S, row4, g_lo, g_hi, n, key_floor_float(T0), warp * kTkRegion);
+        if ((tid & 31) == 0) S.reg_gt[warp] = (int)c;
+        cluster.sync();
+
+        if (crank == 0) {
+            if (tid < kTkMaxRegions) src_cnt[tid] = cluster.map_shared_rank(&S, tid / kTkWarps)->reg_gt[tid % kTkWarps];
+            __syncthreads();
+            uint32_t total = 0;
+            bool fits = true;
+            for (int q = 0; q < kTkMaxRegions; ++q) {
+                total += (uint32_t)src_cnt[q];
+                fits = fits && src_cnt[q] <= kTkRegion;
             }
-            uint32_t total;
-            const uint32_t ex = block_excl_scan(cnt, total, S.warp_sum[scan_buf]);
-            scan_buf ^= 1;
-            uint32_t pos = cbase + ex;
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-                if (mask & (1u << j)) {
-                    if (pos < (uint32_t)kTopkCap) {
-                        S.cand_key[pos] = key[j];
-                        S.cand_idx[pos] = g * 4 + j;
+            fits = fits && total >= (uint32_t)k && total <= (uint32_t)kTkCap;
+            if (fits) {
+                // gather every region, CTA-major then warp: CTA 0's own regions are compacted in
+                // place (destination never above source; read, barrier, write per chunk)
+                int off = 0;
+                for (int q = 0; q < kTkMaxRegions; ++q) {
+                    const int cnt = src_cnt[q];
+                    const TopkSmem* Src = cluster.map_shared_rank(&S, q / kTkWarps);
+                    const int src_off = (q % kTkWarps) * kTkRegion;
+                    for (int e0 = 0; e0 < cnt; e0 += kTkThreads) {
+                        const int e = e0 + tid;
+                        uint32_t key = 0;
+                        int ix = 0;
+                        if (e < cnt) key = Src->cand_key[src_off + e], ix = Src->cand_idx[src_off + e];
+                        __syncthreads();
+                        if (e < cnt) S.cand_key[off + e] = key, S.cand_idx[off + e] = ix;
                     }
-                    ++pos;
+                    if (tid == 0) S.reg_off[q] = off, S.reg_cnt[q] = cnt;
+                    off += cnt;
                 }
-            cbase += total;
-            if (g0 + (u + 1) * kTopkThreads >= g_hi) break;
-        }
-    }
-    if (tid == 0) S.sel_gt = cbase;  // publish this CTA's candidate count
-    cluster.sync();
-
-    if (crank == 0) {
-        uint32_t counts[kTopkCluster], total = 0;
-        bool fits = true;
-#pragma unroll
-        for (int c = 0; c < kTopkCluster; ++c) {
-            counts[c] = cluster.map_shared_rank(&S.sel_gt, c)[0];
-            fits = fits && counts[c] <= (uint32_t)kTopkCap;
-            total += counts[c];
-        }
-        fits = fits && total >= (uint32_t)k && total <= (uint32_t)kTopkCap;
-        if (fits) {
-            uint32_t off = counts[0];
-            for (int c = 1; c < kTopkCluster; ++c) {
-                const uint32_t* pk = cluster.map_shared_rank(S.cand_key, c);
-                const int* pi = cluster.map_shared_rank(S.cand_idx, c);
-                for (uint32_t e = tid; e < counts[c]; e += kTopkThreads) {
-                    S.cand_key[off + e] = pk[e];
-                    S.cand_idx[off + e] = pi[e];
-                }
-                off += counts[c];
+                if (tid == 0) S.nreg = kTkMaxRegions;
+                __syncthreads();
+                done = refine_and_emit(S, T0, k, out);
+            }
+            if (tid == 0) {
+                atomicAdd(&g_counters[2], attempt == 0 ? 1ull : 0ull);
+                if (!done) atomicAdd(&g_counters[3 + 2 * attempt], 1ull);  // [3] first miss, [5] second miss
+                S.sel_gt = done ? 1u : 0u;
+                S.T0 = retarget(rs, total, m, k);
+            }
+            __syncthreads();
+            // tell every CTA whether to go again (and with which rank)
+            if (tid < kTkCluster) {
+                TopkSmem* D = cluster.map_shared_rank(&S, tid);
+                D->sel_bin = S.sel_gt;
+                D->red[0] = S.T0;
             }
         }
-        __syncthreads();
-        if (fits) refine_candidates(S, (int)total, T0, k, out, scan_buf);
-        else topk_two_pass(S, row, n, k, out, scan_buf);
+        cluster.sync();  // CTA 0's gather of every region is complete; the verdict is everywhere
+        done = S.sel_bin != 0u;
+        rs = S.red[0];
+        if (done) break;
     }
-    cluster.sync();  // peers keep their shared memory alive until CTA 0 has read it
+    if (crank == 0 && !done) topk_global(S, row, n, k, out);
+    cluster.sync();  // peers keep their shared memory alive until CTA 0 is done with it
 }
 
 }  // namespace dsa

@@ -159,6 +159,17 @@ dsa_status dsa_sync_status(dsa_stream_t stream);
 void dsa_profile_begin(void);
 dsa_status dsa_profile_end(int64_t *launches, double *total_ms);
 
+/*
+ * Diagnostic path counters, accumulated on the device since load or the last reset:
+ *   [0] top-k rows handled by the one-CTA-per-row kernel; [1] of those, rows whose first sampled
+ *   threshold missed (a second estimate and pass followed); [4] rows whose second estimate also
+ *   missed (exact radix select over the row); [2], [3], [5] the same for rows handled by a CTA
+ *   cluster.  Copies up to n counters (n <= DSA_NUM_COUNTERS) into out after synchronising the
+ *   device; if reset != 0 the counters are zeroed afterwards.  Returns DSA_ERR_CUDA on failure.
+ */
+#define DSA_NUM_COUNTERS 8
+dsa_status dsa_read_counters(int64_t *out, int n, int reset);
+
 /* Number of kernels the library has launched since it was loaded. */
 int64_t dsa_launch_count(void);
 

@@ -44,6 +44,9 @@ _SIGS = {
     "dsa_prefill": (_i, [_p, _p, _p, _p, _p, _p, _i64, _i, _i, _i, _i, _i, _i, _f, _p, _p, _p, _sz, _p]),
     "dsa_decode": (_i, [_p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _i, _i64, _i, _i, _i, _i, _i, _i, _f, _i,
                         _p, _p, _p, _sz, _p]),
+    "dsa_decode_noalloc": (_i, [_p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _i, _i64, _i, _i, _i, _i, _i, _i, _f, _i,
+                                _p, _p, _p]),
+    "dsa_decode_noalloc_scratch_bytes": (_sz, []),
     "dsa_workspace_size": (_sz, [_i, _i64, _i, _i, _i, _i]),
     "dsa_sync_status": (_i, [_p]),
     "dsa_profile_begin": (None, []),

@@ -356,6 +356,31 @@ int64_t prefill_ld(int64_t L) { return (int64_t)align_up((size_t)L, 4); }
 
 }  // namespace
 
+// ------------------------------------------------------------------ allocation-free decode
+// Scratch of dsa_decode_noalloc: a fixed array in the library's own device memory.  Every GPU on
+// which the library is loaded holds it until the process exits.  Host code must not pass the
+// array's name to a kernel (on the host it is only a stand-in for the symbol); its device
+// address is looked up once per device with cudaGetSymbolAddress.
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;  // 16 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[256] = {};
+
+// Device address of g_noalloc_scratch on the current device (looked up on first use).
+dsa_status noalloc_scratch(void** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 256) return DSA_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (!g_noalloc_addr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return DSA_ERR_CUDA;
+        g_noalloc_addr[dev] = p;
+    }
+    *out = g_noalloc_addr[dev];
+    return DSA_OK;
+}
+
 // ====================================================================== C ABI
 extern "C" {
 
@@ -572,6 +597,24 @@ dsa_status dsa_decode(const void* q, const void* qI, const void* w, const void* 
     }
     return DSA_OK;
 }
+
+dsa_status dsa_decode_noalloc(const void* q, const void* qI, const void* w, const void* k_new, const void* v_new,
+                              const void* kI_new, void* k_cache, void* v_cache, void* kI_cache, int32_t* ctx_len, int B,
+                              int64_t Lmax, int Hq, int Hkv, int D, int HI, int dI, int topk, float scale,
+                              int update_ctx, void* out, int32_t* idx_out, dsa_stream_t stream) {
+    if (B <= 0 || Lmax <= 0 || Hq <= 0 || topk <= 0 || Lmax > (int64_t)INT32_MAX || topk > kMaxTopk)
+        return DSA_ERR_INVALID_ARG;
+    // The same work as dsa_decode, with its workspace in the library's fixed scratch array.
+    if (decode_ws_layout(Lmax, B, Hq, topk, idx_out == nullptr).total > kNoAllocScratchBytes)
+        return DSA_ERR_WORKSPACE;
+    void* scratch = nullptr;
+    dsa_status st = noalloc_scratch(&scratch);
+    if (st != DSA_OK) return st;
+    return dsa_decode(q, qI, w, k_new, v_new, kI_new, k_cache, v_cache, kI_cache, ctx_len, B, Lmax, Hq, Hkv, D, HI,
+                      dI, topk, scale, update_ctx, out, idx_out, scratch, kNoAllocScratchBytes, stream);
+}
+
+size_t dsa_decode_noalloc_scratch_bytes(void) { return kNoAllocScratchBytes; }
 
 dsa_status dsa_sync_status(dsa_stream_t stream) {
     if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return DSA_ERR_CUDA;

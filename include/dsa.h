@@ -135,6 +135,34 @@ dsa_status dsa_decode(const void *q, const void *qI, const void *w, const void *
                       void *out, int32_t *idx_out, void *ws, size_t ws_bytes, dsa_stream_t stream);
 
 /*
+ * dsa_decode without a caller workspace: the same decode step, with every piece of scratch it
+ * needs (one fp32 score row per sequence, the index rows when idx_out is NULL, and the per-split
+ * attention partials) taken from a fixed array inside the library's own device memory.  The
+ * pages describe nothing like it: it exists for callers that cannot allocate device memory -- for
+ * example a plugin inside a serving process whose memory pool owns the whole GPU and offers no
+ * way to request workspace, or a caller that must not pay cudaMalloc's implicit device-wide
+ * synchronisation on a latency-critical path.
+ *   - The array holds dsa_decode_noalloc_scratch_bytes() = 16 MiB on every GPU where the library
+ *     is loaded, from load until the process exits.
+ *   - Sizes: the call returns DSA_ERR_WORKSPACE, launching nothing, when the step needs more than
+ *     that, i.e. when dsa_workspace_size(DSA_OP_DECODE, Lmax, B, Hq, HI, topk) (with idx_out NULL;
+ *     less when idx_out is given) exceeds 16 MiB.  B = 16 sequences of 131328 positions fit.
+ *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress) with
+ *     that device current; make that first call before any stream capture.
+ *   - All calls share the one array and it keeps the previous call's contents: no part of it has
+ *     to start at zero (every kernel writes the scratch it later reads), but two calls that
+ *     overlap on the GPU (different streams, or different threads) race on it.  Serialise them.
+ *   - Arguments, results and errors are otherwise those of dsa_decode.
+ */
+dsa_status dsa_decode_noalloc(const void *q, const void *qI, const void *w, const void *k_new, const void *v_new,
+                              const void *kI_new, void *k_cache, void *v_cache, void *kI_cache, int32_t *ctx_len,
+                              int B, int64_t Lmax, int Hq, int Hkv, int D, int HI, int dI, int topk, float scale,
+                              int update_ctx, void *out, int32_t *idx_out, dsa_stream_t stream);
+
+/* Size in bytes of the fixed scratch array used by dsa_decode_noalloc. */
+size_t dsa_decode_noalloc_scratch_bytes(void);
+
+/*
  * Bytes of workspace an entry point needs.  op: DSA_OP_*.  L: sequence length (prefill) or cache
  * capacity Lmax (decode); B: sequences (decode); Hq: query heads; HI: indexer heads; topk.
  * DSA_OP_PREFILL returns the recommended size (score rows of up to 4 GiB per chunk plus index

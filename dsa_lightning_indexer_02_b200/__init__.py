@@ -40,8 +40,13 @@ _SIGS = {
     "dsa_version": (_i, []),
     "dsa_index": (_i, [_p, _p, _p, _i, _i64, _i, _i, _i64, _p, _i64, _p]),
     "dsa_topk": (_i, [_p, _i64, _i, _i64, _i, _p, _p, _sz, _p]),
+    "dsa_topk_window": (_i, [_p, _i64, _i, _i64, _i, _i64, _p, _p]),
     "dsa_sparse_attn": (_i, [_p, _p, _p, _p, _i, _i64, _i64, _i, _i, _i, _i, _f, _p, _p, _p]),
     "dsa_prefill": (_i, [_p, _p, _p, _p, _p, _p, _i64, _i, _i, _i, _i, _i, _i, _f, _p, _p, _p, _sz, _p]),
+    "dsa_prefill_rows": (_i, [_p, _p, _p, _p, _p, _p, _i64, _i64, _i, _i, _i, _i, _i, _i, _i64, _f, _p, _p, _p,
+                              _sz, _p]),
+    "dsa_prefill_window": (_i, [_p, _p, _p, _p, _p, _p, _i64, _i, _i, _i, _i, _i, _i, _i64, _f, _p, _p, _p, _sz,
+                                _p]),
     "dsa_decode": (_i, [_p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _i, _i64, _i, _i, _i, _i, _i, _i, _f, _i,
                         _p, _p, _p, _sz, _p]),
     "dsa_decode_noalloc": (_i, [_p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _i, _i64, _i, _i, _i, _i, _i, _i, _f, _i,
@@ -127,12 +132,16 @@ def dsa_index(qI, kI, w, q_pos0: int, scores, stream=None) -> None:
     _check(st, "dsa_index")
 
 
-def dsa_topk(scores, q_pos0: int, k: int, idx, stream=None) -> None:
+def dsa_topk(scores, q_pos0: int, k: int, idx, window: int = 0, stream=None) -> None:
     import torch
     _need(scores, torch.float32, "scores", 2), _need(idx, torch.int32, "idx", 2)
     Lq = scores.shape[0]
     if idx.shape != (Lq, k):
         raise ValueError(f"idx must be [{Lq}, {k}]")
+    if window:
+        st = _lib.dsa_topk_window(_ptr(scores), scores.shape[1], Lq, q_pos0, k, window, _ptr(idx), _stream(stream))
+        _check(st, "dsa_topk_window")
+        return
     st = _lib.dsa_topk(_ptr(scores), scores.shape[1], Lq, q_pos0, k, _ptr(idx), None, 0, _stream(stream))
     _check(st, "dsa_topk")
 
@@ -151,7 +160,8 @@ def dsa_sparse_attn(q, k, v, idx, q_pos0: int, scale: float, out, lse=None, stre
     _check(st, "dsa_sparse_attn")
 
 
-def dsa_prefill(q, k, v, qI, kI, w, topk: int, scale: float, out, idx_out=None, ws=None, stream=None) -> None:
+def dsa_prefill(q, k, v, qI, kI, w, topk: int, scale: float, out, idx_out=None, ws=None, window: int = 0,
+                stream=None) -> None:
     import torch
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (qI, "qI"), (out, "out")):
         _need(t, torch.bfloat16, n, 3)
@@ -162,10 +172,38 @@ def dsa_prefill(q, k, v, qI, kI, w, topk: int, scale: float, out, idx_out=None, 
         ws = torch.empty(workspace_size(DSA_OP_PREFILL, L, 1, Hq, HI, topk), dtype=torch.uint8, device=q.device)
     if idx_out is not None:
         _need(idx_out, torch.int32, "idx_out", 2)
+    if window:
+        st = _lib.dsa_prefill_window(_ptr(q), _ptr(k), _ptr(v), _ptr(qI), _ptr(kI), _ptr(w), L, Hq, k.shape[1], D,
+                                     HI, dI, topk, window, float(scale), _ptr(out), _ptr(idx_out), _ptr(ws),
+                                     ws.numel() * ws.element_size(), _stream(stream))
+        _check(st, "dsa_prefill_window")
+        return
     st = _lib.dsa_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(qI), _ptr(kI), _ptr(w), L, Hq, k.shape[1], D, HI, dI,
                           topk, float(scale), _ptr(out), _ptr(idx_out), _ptr(ws), ws.numel() * ws.element_size(),
                           _stream(stream))
     _check(st, "dsa_prefill")
+
+
+def dsa_prefill_rows(q_rows, k, v, qI_rows, kI, w_rows, row0: int, topk: int, scale: float, out_rows,
+                     idx_rows=None, ws=None, window: int = 0, stream=None) -> None:
+    """Prefill of query rows row0 .. row0+len(q_rows)-1; k, v, kI cover at least those rows."""
+    import torch
+    for t, n in ((q_rows, "q_rows"), (k, "k"), (v, "v"), (qI_rows, "qI_rows"), (out_rows, "out_rows")):
+        _need(t, torch.bfloat16, n, 3)
+    _need(kI, torch.bfloat16, "kI", 2), _need(w_rows, torch.bfloat16, "w_rows", 2)
+    rows, Hq, D = q_rows.shape
+    HI, dI = qI_rows.shape[1], qI_rows.shape[2]
+    if k.shape[0] < row0 + rows or kI.shape[0] < row0 + rows:
+        raise ValueError("k/v/kI must cover rows up to row0 + rows")
+    if ws is None:
+        ws = torch.empty(workspace_size(DSA_OP_PREFILL, row0 + rows, 1, Hq, HI, topk), dtype=torch.uint8,
+                         device=q_rows.device)
+    if idx_rows is not None:
+        _need(idx_rows, torch.int32, "idx_rows", 2)
+    st = _lib.dsa_prefill_rows(_ptr(q_rows), _ptr(k), _ptr(v), _ptr(qI_rows), _ptr(kI), _ptr(w_rows), row0, rows, Hq,
+                               k.shape[1], D, HI, dI, topk, window, float(scale), _ptr(out_rows), _ptr(idx_rows),
+                               _ptr(ws), ws.numel() * ws.element_size(), _stream(stream))
+    _check(st, "dsa_prefill_rows")
 
 
 def dsa_decode(q, qI, w, k_new, v_new, kI_new, k_cache, v_cache, kI_cache, ctx_len, topk: int, scale: float, out,

@@ -17,7 +17,8 @@
 //     (m16n8k16, keys or head-dimension rows as M, 8 heads as N), so no MMA lane is wasted on
 //     the small head count; P^T goes from the accumulator layout to the operand layout with
 //     movmatrix; online softmax in fp32 (exp2 domain);
-//   - masked and padding slots (index -1) are zero-filled copies with logit -inf.
+//   - slots past the row's count and entries naming no key (index -1 or >= n_keys) are
+//     zero-filled copies with logit -inf.
 // With nsplit > 1 every CTA writes unnormalised partial results (O, running max, running sum)
 // for its slice of the index list; attn_combine_kernel merges them.
 #pragma once
@@ -48,12 +49,13 @@ struct AttnParams {
     float* lse;               // [T, Hq] natural-log LSE, may be null
     int nsplit;               // key splits per token
     float* part;              // nsplit > 1: [T, nsplit, Hq, D + 2]
+    long long window;         // > 0 (prefill): a row holds at most min(topk, window) keys
 };
 
 __host__ __device__ constexpr int attn_keys_per_stage(int hkv) { return 128 / hkv; }
 __host__ __device__ constexpr int attn_row_bytes(int hkv) { return hkv * kAttnD * 2 + 16; }
 __host__ __device__ constexpr int attn_smem_bytes(int hkv) {
-    return kAttnStages * attn_keys_per_stage(hkv) * attn_row_bytes(hkv) * 2 + kAttnIdxWin * 4;
+    return kAttnStages * attn_keys_per_stage(hkv) * attn_row_bytes(hkv) * 2 + kAttnIdxWin * 4 + kAttnStages * 128;
 }
 
 // NT: n-tiles of 8 query heads per KV group (G <= 8 * NT).
@@ -79,6 +81,7 @@ __global__ void __launch_bounds__(256) sparse_attn_kernel(const AttnParams P) {
         vb += (long long)t * P.kv_bstride;
     } else {
         n_ll = P.q_pos0 + t + 1;
+        if (P.window > 0 && n_ll > P.window) n_ll = P.window;
     }
     const int n_sel = (int)min((long long)P.topk, n_ll);
     const int per_split = (n_sel + P.nsplit - 1) / P.nsplit;
@@ -105,6 +108,8 @@ __global__ void __launch_bounds__(256) sparse_attn_kernel(const AttnParams P) {
     // ---- the index list, kAttnIdxWin entries at a time, in shared memory: the gathers of a stage
     // are issued without waiting on a global load of their indices
     int* sidx = reinterpret_cast<int*>(smem + kAttnStages * STAGE);
+    // per stage and key: 1 if the slot holds a usable key (in range, index in [0, n_keys))
+    uint8_t* svalid = reinterpret_cast<uint8_t*>(sidx + kAttnIdxWin);
     int win_off = 0;  // window covers slots [p_begin + win_off, p_begin + win_off + kAttnIdxWin)
     auto fill_window = [&]() {
         for (int i = threadIdx.x; i < kAttnIdxWin; i += nthreads) {
@@ -126,6 +131,7 @@ __global__ void __launch_bounds__(256) sparse_attn_kernel(const AttnParams P) {
             const int p = p0 + key;
             int s = (p < p_end) ? sidx[p - p_begin - win_off] : -1;
             bool ok = s >= 0 && s < P.n_keys;
+            if (ch == 0) svalid[buf * 128 + key] = ok ? 1 : 0;
             const long long off = (ok ? (long long)s : 0) * (Hkv * kAttnD) + ch * 8;
             cp_async_16(sk + key * RB + ch * 16, kb + off, ok);
             cp_async_16(sv + key * RB + ch * 16, vb + off, ok);
@@ -185,7 +191,10 @@ __global__ void __launch_bounds__(256) sparse_attn_kernel(const AttnParams P) {
                 }
             }
             // mask slots beyond this CTA's range; rows: key lane/4 (c0,c1) and lane/4+8 (c2,c3)
-            const bool v0 = pbase + (lane >> 2) < p_end, v1 = pbase + (lane >> 2) + 8 < p_end;
+            // masked: slots past this CTA's range and entries that name no key (e.g. -1 padding)
+            const uint8_t* vrow = svalid + (step % kAttnStages) * 128 + kt * 16;
+            const bool v0 = pbase + (lane >> 2) < p_end && vrow[lane >> 2];
+            const bool v1 = pbase + (lane >> 2) + 8 < p_end && vrow[(lane >> 2) + 8];
             uint32_t pb[NT][2];
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
@@ -329,11 +338,16 @@ __global__ void __launch_bounds__(256) sparse_attn_kernel(const AttnParams P) {
     }
 }
 
-// Merge split partials: one warp per (token, head).
+// Merge split partials: one warp per (token, head).  With advance_ctx (decode), block 0 also
+// moves every sequence's context length one position on (nothing later in the step reads it).
 __global__ void __launch_bounds__(128) attn_combine_kernel(const float* part, int T, int nsplit, int Hq,
-                                                           __nv_bfloat16* out, float* lse) {
+                                                           __nv_bfloat16* out, float* lse, int* advance_ctx,
+                                                           long long Lmax) {
     const int wid = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
+    if (advance_ctx && blockIdx.x == 0)
+        for (int b = threadIdx.x; b < T; b += blockDim.x)
+            if (advance_ctx[b] >= 0 && advance_ctx[b] < Lmax) advance_ctx[b] += 1;
     if (wid >= T * Hq) return;
     const int t = wid / Hq, h = wid % Hq;
     float mx = -INFINITY;

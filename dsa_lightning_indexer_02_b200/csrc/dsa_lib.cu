@@ -156,7 +156,8 @@ dsa_status launch_indexer_t(const CUtensorMap& mq, const CUtensorMap& mk, const 
 
 // Shared by dsa_index (P = 1) and the decode step (P = B, one query each).
 dsa_status run_indexer(const void* qI, const void* kI, const __nv_bfloat16* w, int P_, int Lq, int64_t q_pos0,
-                       const int* ctx_len, int64_t Lk, int HI, float* scores, int64_t ld, cudaStream_t s) {
+                       const int* ctx_len, int64_t Lk, int HI, float* scores, int64_t ld, cudaStream_t s,
+                       int64_t window = 0) {
     const bool decode = ctx_len != nullptr;
     const int BN = decode ? HI : 256;
     const int TB = BN / HI;
@@ -170,11 +171,13 @@ dsa_status run_indexer(const void* qI, const void* kI, const __nv_bfloat16* w, i
     P.scores = scores;
     P.ld = ld;
     P.num_qb = (Lq + TB - 1) / TB;
+    P.window = decode ? 0 : window;
     const int sms = num_sms();
     if (sms <= 0) return DSA_ERR_CUDA;
     const int64_t ktiles = (Lk + kIdxBM - 1) / kIdxBM;
     if (decode) {
-        int ns = std::max(1, (2 * sms + P_ - 1) / P_);
+        // about 4 units per SM, the same count on every SM when B divides 4*SMs
+        int ns = std::max(1, (4 * sms + P_ - 1) / P_);
         ns = (int)std::min<int64_t>(ns, ktiles);
         P.kt_per_split = (int)((ktiles + ns - 1) / ns);
         P.nsplit = (int)((ktiles + P.kt_per_split - 1) / P.kt_per_split);
@@ -215,15 +218,16 @@ dsa_status run_indexer(const void* qI, const void* kI, const __nv_bfloat16* w, i
 
 // ------------------------------------------------------------------ top-k launch
 dsa_status run_topk(const float* scores, int64_t ld, int rows, int64_t q_pos0, const int* ctx_len, int64_t n_max,
-                    int k, int* idx, cudaStream_t s) {
-    TopkParams P{scores, ld, rows, q_pos0, ctx_len, n_max, k, idx};
+                    int k, int* idx, cudaStream_t s, int64_t window = 0) {
+    TopkParams P{scores, ld, rows, q_pos0, ctx_len, n_max, k, idx, window};
     const int sms = num_sms();
     const int smem = (int)sizeof(TopkSmem);
     // Few long rows: a cluster of CTAs per row; otherwise one CTA per row.
     if ((long long)rows * kTkCluster <= 2LL * sms && n_max > 4LL * kTkCap) {
+        const int csmem = smem + kTkCap * 8;
         static bool cattr = false;
         if (!cattr) {
-            if (cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+            if (cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, csmem) !=
                 cudaSuccess)
                 return DSA_ERR_CUDA;
             cattr = true;
@@ -231,7 +235,7 @@ dsa_status run_topk(const float* scores, int64_t ld, int rows, int64_t q_pos0, c
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(rows * kTkCluster);
         cfg.blockDim = dim3(kTkThreads);
-        cfg.dynamicSmemBytes = smem;
+        cfg.dynamicSmemBytes = csmem;
         cfg.stream = s;
         cudaLaunchAttribute attr[1];
         attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -411,17 +415,22 @@ dsa_status dsa_index(const void* qI, const void* kI, const void* w, int Lq, int6
                        ld_scores, reinterpret_cast<cudaStream_t>(stream));
 }
 
+dsa_status dsa_topk_window(const float* scores, int64_t ld_scores, int Lq, int64_t q_pos0, int k, int64_t window,
+                           int32_t* idx, dsa_stream_t stream) {
+    if (!scores || !idx) return DSA_ERR_INVALID_ARG;
+    if (!aligned16(scores) || !aligned16(idx)) return DSA_ERR_INVALID_ARG;
+    if (Lq <= 0 || q_pos0 < 0 || ld_scores % 4 != 0 || ld_scores < q_pos0 + Lq) return DSA_ERR_INVALID_ARG;
+    if (k <= 0 || window < 0) return DSA_ERR_INVALID_ARG;
+    if (k > kMaxTopk || q_pos0 + Lq > (int64_t)INT32_MAX) return DSA_ERR_UNSUPPORTED;
+    return run_topk(scores, ld_scores, Lq, q_pos0, nullptr, q_pos0 + Lq, k, idx,
+                    reinterpret_cast<cudaStream_t>(stream), window);
+}
+
 dsa_status dsa_topk(const float* scores, int64_t ld_scores, int Lq, int64_t q_pos0, int k, int32_t* idx, void* ws,
                     size_t ws_bytes, dsa_stream_t stream) {
     (void)ws;
     (void)ws_bytes;
-    if (!scores || !idx) return DSA_ERR_INVALID_ARG;
-    if (!aligned16(scores) || !aligned16(idx)) return DSA_ERR_INVALID_ARG;
-    if (Lq <= 0 || q_pos0 < 0 || ld_scores % 4 != 0 || ld_scores < q_pos0 + Lq) return DSA_ERR_INVALID_ARG;
-    if (k <= 0) return DSA_ERR_INVALID_ARG;
-    if (k > kMaxTopk || q_pos0 + Lq > (int64_t)INT32_MAX) return DSA_ERR_UNSUPPORTED;
-    return run_topk(scores, ld_scores, Lq, q_pos0, nullptr, q_pos0 + Lq, k, idx,
-                    reinterpret_cast<cudaStream_t>(stream));
+    return dsa_topk_window(scores, ld_scores, Lq, q_pos0, k, 0, idx, stream);
 }
 
 dsa_status dsa_sparse_attn(const void* q, const void* k, const void* v, const int32_t* idx, int Lq, int64_t Lk,
@@ -476,26 +485,29 @@ size_t dsa_workspace_size(int op, int64_t L, int B, int Hq, int HI, int topk) {
     }
 }
 
-dsa_status dsa_prefill(const void* q, const void* k, const void* v, const void* qI, const void* kI, const void* w,
-                       int64_t L, int Hq, int Hkv, int D, int HI, int dI, int topk, float scale, void* out,
-                       int32_t* idx_out, void* ws, size_t ws_bytes, dsa_stream_t stream) {
+dsa_status dsa_prefill_rows(const void* q, const void* k, const void* v, const void* qI, const void* kI,
+                            const void* w, int64_t row0, int64_t rows, int Hq, int Hkv, int D, int HI, int dI,
+                            int topk, int64_t window, float scale, void* out, int32_t* idx_out, void* ws,
+                            size_t ws_bytes, dsa_stream_t stream) {
     if (!q || !k || !v || !qI || !kI || !w || !out) return DSA_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(qI) || !aligned16(kI) || !aligned16(w) ||
         !aligned16(out) || (idx_out && !aligned16(idx_out)))
         return DSA_ERR_INVALID_ARG;
-    if (L <= 0 || topk <= 0 || HI <= 0 || dI <= 0 || !(scale == scale)) return DSA_ERR_INVALID_ARG;
+    if (row0 < 0 || rows <= 0 || topk <= 0 || HI <= 0 || dI <= 0 || window < 0 || !(scale == scale))
+        return DSA_ERR_INVALID_ARG;
     dsa_status st = check_attn_shape(Hq, Hkv, D);
     if (st != DSA_OK) return st;
-    if (dI != kIdxBK || !hi_supported_prefill(HI) || topk > kMaxTopk || L * HI > (int64_t)INT32_MAX)
+    const int64_t Lk = row0 + rows;  // keys the last row needs
+    if (dI != kIdxBK || !hi_supported_prefill(HI) || topk > kMaxTopk || Lk * HI > (int64_t)INT32_MAX)
         return DSA_ERR_UNSUPPORTED;
     if (!ws || !aligned16(ws)) return DSA_ERR_WORKSPACE;
-    const int64_t ld = prefill_ld(L);
+    const int64_t ld = prefill_ld(Lk);
     const int TB = 256 / HI;
     const size_t per_row = (size_t)ld * 4 + (idx_out ? 0 : (size_t)topk * 4);
     int64_t C = (int64_t)((ws_bytes > 512 ? ws_bytes - 512 : 0) / per_row);  // 512: alignment slack
-    C = std::min<int64_t>(C, L);
+    C = std::min<int64_t>(C, rows);
     if (C >= TB) C = C / TB * TB;
-    if (C < std::min<int64_t>(L, TB)) return DSA_ERR_WORKSPACE;
+    if (C < std::min<int64_t>(rows, TB)) return DSA_ERR_WORKSPACE;
     float* scores = static_cast<float*>(ws);
     int32_t* idx_ws = idx_out ? nullptr
                               : reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) +
@@ -505,12 +517,13 @@ dsa_status dsa_prefill(const void* q, const void* k, const void* v, const void* 
     const auto* qIb = static_cast<const __nv_bfloat16*>(qI);
     const auto* wb = static_cast<const __nv_bfloat16*>(w);
     auto* ob = static_cast<__nv_bfloat16*>(out);
-    for (int64_t c0 = 0; c0 < L; c0 += C) {
-        const int rows = (int)std::min<int64_t>(C, L - c0);
+    for (int64_t c0 = 0; c0 < rows; c0 += C) {   // c0: offset inside the row range
+        const int n = (int)std::min<int64_t>(C, rows - c0);
+        const int64_t t0 = row0 + c0;            // absolute position of the chunk's first row
         int32_t* idx_c = idx_out ? idx_out + c0 * topk : idx_ws;
-        st = run_indexer(qIb + c0 * HI * dI, kI, wb + c0 * HI, 1, rows, c0, nullptr, c0 + rows, HI, scores, ld, s);
+        st = run_indexer(qIb + c0 * HI * dI, kI, wb + c0 * HI, 1, n, t0, nullptr, t0 + n, HI, scores, ld, s, window);
         if (st != DSA_OK) return st;
-        st = run_topk(scores, ld, rows, c0, nullptr, c0 + rows, topk, idx_c, s);
+        st = run_topk(scores, ld, n, t0, nullptr, t0 + n, topk, idx_c, s, window);
         if (st != DSA_OK) return st;
         AttnParams P{};
         P.q = qb + c0 * Hq * D;
@@ -518,18 +531,35 @@ dsa_status dsa_prefill(const void* q, const void* k, const void* v, const void* 
         P.v = static_cast<const __nv_bfloat16*>(v);
         P.idx = idx_c;
         P.topk = topk;
-        P.T = rows;
-        P.q_pos0 = c0;
-        P.n_keys = L;
+        P.T = n;
+        P.q_pos0 = t0;
+        P.n_keys = Lk;
         P.Hq = Hq;
         P.Hkv = Hkv;
         P.scale_log2 = scale * 1.4426950408889634f;
         P.out = ob + c0 * Hq * D;
         P.nsplit = 1;
+        P.window = window;
         st = run_attn(P, s);
         if (st != DSA_OK) return st;
     }
     return DSA_OK;
+}
+
+dsa_status dsa_prefill_window(const void* q, const void* k, const void* v, const void* qI, const void* kI,
+                              const void* w, int64_t L, int Hq, int Hkv, int D, int HI, int dI, int topk,
+                              int64_t window, float scale, void* out, int32_t* idx_out, void* ws, size_t ws_bytes,
+                              dsa_stream_t stream) {
+    if (L <= 0) return DSA_ERR_INVALID_ARG;
+    return dsa_prefill_rows(q, k, v, qI, kI, w, 0, L, Hq, Hkv, D, HI, dI, topk, window, scale, out, idx_out, ws,
+                            ws_bytes, stream);
+}
+
+dsa_status dsa_prefill(const void* q, const void* k, const void* v, const void* qI, const void* kI, const void* w,
+                       int64_t L, int Hq, int Hkv, int D, int HI, int dI, int topk, float scale, void* out,
+                       int32_t* idx_out, void* ws, size_t ws_bytes, dsa_stream_t stream) {
+    return dsa_prefill_window(q, k, v, qI, kI, w, L, Hq, Hkv, D, HI, dI, topk, 0, scale, out, idx_out, ws, ws_bytes,
+                              stream);
 }
 
 dsa_status dsa_decode(const void* q, const void* qI, const void* w, const void* k_new, const void* v_new,
@@ -587,10 +617,10 @@ dsa_status dsa_decode(const void* q, const void* qI, const void* w, const void* 
     if (P.nsplit > 1) {
         LaunchScope ls(K_COMBINE, s);
         const int warps = B * Hq;
-        attn_combine_kernel<<<(warps + 3) / 4, 128, 0, s>>>(part, B, P.nsplit, Hq, P.out, nullptr);
+        attn_combine_kernel<<<(warps + 3) / 4, 128, 0, s>>>(part, B, P.nsplit, Hq, P.out, nullptr,
+                                                            update_ctx ? ctx_len : nullptr, Lmax);
         if ((st = launch_status()) != DSA_OK) return st;
-    }
-    if (update_ctx) {
+    } else if (update_ctx) {
         LaunchScope ls(K_ADVANCE, s);
         decode_advance_kernel<<<(B + 127) / 128, 128, 0, s>>>(ctx_len, B, Lmax);
         if ((st = launch_status()) != DSA_OK) return st;

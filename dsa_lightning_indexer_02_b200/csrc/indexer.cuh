@@ -44,6 +44,7 @@ struct IndexerParams {
     int num_units;              // P * num_qb * nsplit
     uint32_t q_box_bytes;       // bytes one Q TMA box brings
     uint32_t k_box_bytes;       // bytes one kI TMA box brings
+    long long window;           // > 0 (prefill): keys s <= t - window are not needed (not scored)
 };
 
 struct IndexerUnit {
@@ -72,7 +73,8 @@ __device__ __forceinline__ IndexerUnit indexer_unit(const IndexerParams& P, int 
     const long long t_last = r.tq0 + r.rows - 1;
     const int nkt = (int)(t_last / kIdxBM) + 1;
     if (P.nsplit == 1) {
-        r.kt0 = 0;
+        // sliding window: the block's first token needs keys from tq0 - window + 1 on
+        r.kt0 = P.window > 0 ? (int)(max(0LL, r.tq0 - P.window + 1) / kIdxBM) : 0;
         r.kt1 = nkt;
     } else {
         r.kt0 = split * P.kt_per_split;
@@ -116,11 +118,23 @@ __device__ __forceinline__ float head_sum(const float* v, const float* w) {
         float2 acc[NA];
 #pragma unroll
         for (int i = 0; i < NA; ++i) acc[i] = make_float2(0.f, 0.f);
+        if constexpr (N % 4 == 0) {
+            // weights four at a time: one 16-byte shared load (a warp-wide broadcast) per 4 heads
 #pragma unroll
-        for (int p = 0; p < NP; ++p) {
-            const float2 x = make_float2(fmaxf(v[2 * p], 0.f), fmaxf(v[2 * p + 1], 0.f));
-            const float2 ww = *reinterpret_cast<const float2*>(w + 2 * p);
-            acc[p % NA] = ffma2(x, ww, acc[p % NA]);
+            for (int q = 0; q < N / 4; ++q) {
+                const float4 w4 = *reinterpret_cast<const float4*>(w + 4 * q);
+                const float2 x0 = make_float2(fmaxf(v[4 * q], 0.f), fmaxf(v[4 * q + 1], 0.f));
+                const float2 x1 = make_float2(fmaxf(v[4 * q + 2], 0.f), fmaxf(v[4 * q + 3], 0.f));
+                acc[(2 * q) % NA] = ffma2(x0, make_float2(w4.x, w4.y), acc[(2 * q) % NA]);
+                acc[(2 * q + 1) % NA] = ffma2(x1, make_float2(w4.z, w4.w), acc[(2 * q + 1) % NA]);
+            }
+        } else {
+#pragma unroll
+            for (int p = 0; p < NP; ++p) {
+                const float2 x = make_float2(fmaxf(v[2 * p], 0.f), fmaxf(v[2 * p + 1], 0.f));
+                const float2 ww = *reinterpret_cast<const float2*>(w + 2 * p);
+                acc[p % NA] = ffma2(x, ww, acc[p % NA]);
+            }
         }
         float r = 0.f;
 #pragma unroll
@@ -133,17 +147,21 @@ __device__ __forceinline__ float head_sum(const float* v, const float* w) {
 template <int N>
 __device__ __forceinline__ void head_sum_acc(const float* v, const float* w, float2 (&carry)[4]) {
 #pragma unroll
-    for (int p = 0; p < N / 2; ++p) {
-        const float2 x = make_float2(fmaxf(v[2 * p], 0.f), fmaxf(v[2 * p + 1], 0.f));
-        const float2 ww = *reinterpret_cast<const float2*>(w + 2 * p);
-        carry[p % 4] = ffma2(x, ww, carry[p % 4]);
+    for (int q = 0; q < N / 4; ++q) {
+        const float4 w4 = *reinterpret_cast<const float4*>(w + 4 * q);
+        const float2 x0 = make_float2(fmaxf(v[4 * q], 0.f), fmaxf(v[4 * q + 1], 0.f));
+        const float2 x1 = make_float2(fmaxf(v[4 * q + 2], 0.f), fmaxf(v[4 * q + 3], 0.f));
+        carry[(2 * q) % 4] = ffma2(x0, make_float2(w4.x, w4.y), carry[(2 * q) % 4]);
+        carry[(2 * q + 1) % 4] = ffma2(x1, make_float2(w4.z, w4.w), carry[(2 * q + 1) % 4]);
     }
 }
 
 template <int HI, int BN, int STAGES>
 struct IndexerCfg {
     static constexpr int TB = BN / HI;
-    static constexpr int NWG = (BN >= 128 && BN / 2 >= HI) ? 2 : 1;
+    // epilogue warpgroups: each owns BN/NWG columns (whole tokens); more warps hide the latency
+    // of the per-token reduction chains
+    static constexpr int NWG = (BN >= 256 && BN / 4 >= HI) ? 4 : (BN >= 128 && BN / 2 >= HI) ? 2 : 1;
     static constexpr int COLS_WG = BN / NWG;
     static constexpr int CHUNK = COLS_WG >= 32 ? 32 : 16;
     static constexpr int NCHUNK = COLS_WG / CHUNK;

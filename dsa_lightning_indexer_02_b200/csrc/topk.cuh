@@ -15,16 +15,18 @@
 //            its own shared-memory region with warp-level scans -- no block barrier per load;
 //   refine   if every region fits and the total is >= k, the candidates contain the exact
 //            top-k: radix rounds over the key offsets from T0 (first round scaled to the
-//            candidates' key range) give the exact k-th key tau and the number r of keys equal
-//            to tau to keep;
-//   emit     keys > tau are written region by region; the keys == tau are ranked by index and
-//            the r lowest kept.
+//            candidates' key range) narrow the bin that holds the k-th key until it is small;
+//   emit     keys above that bin are written region by region; the bin's few members are ranked
+//            by (key desc, index asc) and the best ones complete the row.
 // If the candidates miss the window [k, capacity], the estimate is redone once, aimed using the
 // observed count, and the row streamed again.  Rows that still miss (or where more than 1024
 // keys tie at tau) take an exact radix select over the row itself (10-bit rounds, then one
 // ordered pass): slower, and rare.
-// Output order: keys > tau region by region (each region ascending), then the kept ties
-// ascending.
+// Output order: keys above the boundary bin region by region (each region ascending), then the
+// boundary bin's kept members by (key desc, index asc).
+// Sliding window (SW-DSA, page "DSA注意力机制：多模态学习中的强化推理新范式", showapi.com,
+// section 1.4: the selection is restricted to a local window): with window W > 0 only keys
+// s > t - W compete; everything else is unchanged.
 #pragma once
 
 #include <cooperative_groups.h>
@@ -54,13 +56,17 @@ struct TopkParams {
     long long n_max;      // upper bound on n (keys addressable in a row)
     int k;
     int* idx;             // [rows, k]
+    long long window;     // > 0: only the last `window` keys of a row (s > t - window) compete
 };
 
 struct TopkSmem {
     uint32_t hist[kTkBins];
     uint32_t cand_key[kTkCap];  // also holds the sample keys before streaming
     int cand_idx[kTkCap];
-    int reg_off[kTkMaxRegions], reg_cnt[kTkMaxRegions], reg_gt[kTkMaxRegions], reg_eq[kTkMaxRegions];
+    // candidate regions: keys/indices may live in this CTA's or (cluster) another CTA's shared memory
+    const uint32_t* reg_kp[kTkMaxRegions];
+    const int* reg_ip[kTkMaxRegions];
+    int reg_cnt[kTkMaxRegions], reg_gt[kTkMaxRegions], reg_eq[kTkMaxRegions];
     int nreg;
     uint32_t red[kTkWarps];
     uint32_t sel_bin, sel_gt;
@@ -85,6 +91,11 @@ __device__ __forceinline__ long long row_length(const TopkParams& P, int r, bool
         n = n < 1 ? 1 : P.n_max;
     }
     return n;
+}
+
+// First key of row r's candidate range: 0, or n - window under a sliding window.
+__device__ __forceinline__ int row_first_key(const TopkParams& P, int n) {
+    return (P.window > 0 && (long long)n > P.window) ? (int)(n - P.window) : 0;
 }
 
 // Inclusive warp prefix sum.
@@ -178,16 +189,22 @@ __device__ __forceinline__ uint32_t sample_threshold(TopkSmem& S, int m, uint32_
     return (b1 << 22) | (S.sel_bin << 12);
 }
 
-// Stream float4 groups [g_lo, g_hi) of a row with n valid scores and compact the scores >= F0
-// into this warp's region, in index order.  Warp w takes the 128-byte pieces p with p % 4 == w.
+// Stream float4 groups [g_lo, g_hi) of a row whose keys e_lo <= e < n compete and compact the
+// scores >= F0 into this warp's region, in index order.  Warp w takes the 128-byte pieces p
+// (keys 32p .. 32p+31 of the row) with p % 4 == w: region w.
 // Returns how many scores of this warp qualified (may exceed the region; the excess is dropped).
-__device__ __forceinline__ uint32_t stream_collect(TopkSmem& S, const float4* row4, int g_lo, int g_hi, int n,
-                                                   float F0, int region_base) {
+__device__ __forceinline__ uint32_t stream_collect(TopkSmem& S, const float4* row4, int g_lo, int g_hi, int e_lo,
+                                                   int n, float F0, int region_base) {
+    const int g_first = g_lo;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     // float4 offset inside a 128-float4 round: piece (lane/8)*4 + warp, float4 lane%8 of it
     const int lane_off = (lane >> 3) * 32 + warp * 8 + (lane & 7);
     uint32_t cnt = 0;
-    for (int g0 = g_lo; g0 < g_hi; g0 += kTkUnroll * 128) {
+    // pieces are numbered from the start of the row: start at a multiple of 4 pieces (32 float4)
+    // so that warp w takes exactly the pieces p with p % 4 == w (keys below g_lo are masked)
+    g_lo &= ~31;
+    constexpr int kStep = kTkUnroll * 128;  // float4 per iteration
+    for (int g0 = g_lo; g0 < g_hi; g0 += kStep) {
         float4 v[kTkUnroll];
 #pragma unroll
         for (int u = 0; u < kTkUnroll; ++u) {
@@ -202,7 +219,7 @@ __device__ __forceinline__ uint32_t stream_collect(TopkSmem& S, const float4* ro
             if (g < g_hi) {
 #pragma unroll
                 for (int j = 0; j < 4; ++j)
-                    if (f[j] >= F0 && g * 4 + j < n) mask |= 1u << j;
+                    if (f[j] >= F0 && g * 4 + j < n && g * 4 + j >= e_lo && g >= g_first) mask |= 1u << j;
             }
             const uint32_t c = __popc(mask);
             const uint32_t incl = warp_incl_scan(c);
@@ -225,14 +242,18 @@ __device__ __forceinline__ uint32_t stream_collect(TopkSmem& S, const float4* ro
 }
 
 // Exact top-k among the candidates in S's regions (every candidate key >= lo; their total is
-// >= k and includes every key of the row >= lo).  Returns false, writing nothing, when more
-// than kTkBins keys tie at the k-th key.
+// >= k and includes every key of the row >= lo).  Radix rounds over the key offsets narrow down
+// the bin holding the k-th key until it holds at most kTkSmallBin candidates (or one key value);
+// keys above that bin are all kept, and the bin's members are ranked by (key desc, index asc).
+// Returns false, writing nothing, when more than kTkBins candidates share the last bin.
+constexpr int kTkSmallBin = 64;
+
 __device__ __forceinline__ bool refine_and_emit(TopkSmem& S, uint32_t lo, int k, int* out) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int nreg = S.nreg;
     uint32_t mx = 0;
     for (int r = 0; r < nreg; ++r)
-        for (int e = tid; e < S.reg_cnt[r]; e += kTkThreads) mx = max(mx, S.cand_key[S.reg_off[r] + e] - lo);
+        for (int e = tid; e < S.reg_cnt[r]; e += kTkThreads) mx = max(mx, S.reg_kp[r][e] - lo);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
     __syncthreads();
@@ -242,10 +263,9 @@ __device__ __forceinline__ bool refine_and_emit(TopkSmem& S, uint32_t lo, int k,
 #pragma unroll
     for (int w = 0; w < kTkWarps; ++w) R = max(R, S.red[w]);
     int fixed = R ? 32 - __clz(R) : 0;  // every offset is < 2^fixed
-    uint32_t pv = 0, need = (uint32_t)k, T = 0;
-    if (fixed == 0) {
-        for (int r = 0; r < nreg; ++r) T += (uint32_t)S.reg_cnt[r];  // all candidates share one key
-    }
+    uint32_t pv = 0, need = (uint32_t)k, cnt_b = 0;
+    if (fixed == 0)
+        for (int r = 0; r < nreg; ++r) cnt_b += (uint32_t)S.reg_cnt[r];  // one key value for all
     while (fixed > 0) {
         const int sh = fixed > 10 ? fixed - 10 : 0;
         const int nbins = 1 << (fixed - sh);
@@ -254,76 +274,80 @@ __device__ __forceinline__ bool refine_and_emit(TopkSmem& S, uint32_t lo, int k,
         __syncthreads();
         for (int r = 0; r < nreg; ++r)
             for (int e = tid; e < S.reg_cnt[r]; e += kTkThreads) {
-                const uint32_t d = S.cand_key[S.reg_off[r] + e] - lo;
+                const uint32_t d = S.reg_kp[r][e] - lo;
                 const bool match = fixed >= 32 ? true : ((d >> fixed) == (pv >> fixed));
                 if (match) atomicAdd(&S.hist[(d >> sh) & (nbins - 1)], 1u);
             }
         __syncthreads();
         find_threshold_bin(S, nbins, need);
         need -= S.sel_gt;
-        T = S.hist[S.sel_bin];  // after the last round (sh == 0) a bin is a single key
+        cnt_b = S.hist[S.sel_bin];
         pv |= S.sel_bin << sh;
         fixed = sh;
+        if (cnt_b <= (uint32_t)kTkSmallBin) break;  // uniform: every thread read the same count
     }
     __syncthreads();
-    const uint32_t tau = lo + pv;
-    const uint32_t ties = need;  // 1 <= ties <= T
-    if (T > (uint32_t)kTkBins && T != ties) return false;
-    // per-region counts of keys > tau and == tau
-    for (int r = warp; r < nreg; r += kTkWarps) {
-        uint32_t gt = 0, eq = 0;
-        for (int e = lane; e < S.reg_cnt[r]; e += 32) {
-            const uint32_t key = S.cand_key[S.reg_off[r] + e];
-            gt += key > tau;
-            eq += key == tau;
+    // boundary bin: offsets d with d >> fixed == pv >> fixed; kept outright: d >> fixed > pv >> fixed
+    if (cnt_b > (uint32_t)(kTkBins / 2)) return false;
+    const uint32_t bin = fixed >= 32 ? 0u : (pv >> fixed);
+    auto above = [&](uint32_t d) { return fixed < 32 && (d >> fixed) > bin; };
+    auto in_bin = [&](uint32_t d) { return fixed >= 32 || (d >> fixed) == bin; };
+    // the bin's members (key, index) into a small list; their order does not matter
+    uint32_t* bkey = S.hist;  // reused: up to kTkBins / 2 members
+    uint32_t* bidx = S.hist + kTkBins / 2;
+    if (tid == 0) S.sel_bin = 0;
+    __syncthreads();
+    for (int r = 0; r < nreg; ++r)
+        for (int e = tid; e < S.reg_cnt[r]; e += kTkThreads) {
+            const uint32_t key = S.reg_kp[r][e];
+            if (in_bin(key - lo)) {
+                const uint32_t p = atomicAdd(&S.sel_bin, 1u);
+                bkey[p] = key;
+                bidx[p] = (uint32_t)S.reg_ip[r][e];
+            }
         }
+    __syncthreads();
+    // kept: above the bin, or in it with rank < need by (key desc, index asc)
+    auto kept = [&](uint32_t key, uint32_t ix) {
+        const uint32_t d = key - lo;
+        if (above(d)) return true;
+        if (!in_bin(d)) return false;
+        uint32_t rank = 0;
+        for (uint32_t b2 = 0; b2 < cnt_b; ++b2) {
+            const uint32_t kb = bkey[b2];
+            rank += (kb > key) || (kb == key && bidx[b2] < ix);
+        }
+        return rank < need;
+    };
+    // write the kept keys region by region, each region in its own (ascending) order
+    for (int r = warp; r < nreg; r += kTkWarps) {
+        uint32_t c = 0;
+        for (int e = lane; e < S.reg_cnt[r]; e += 32) c += kept(S.reg_kp[r][e], (uint32_t)S.reg_ip[r][e]);
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            gt += __shfl_xor_sync(0xffffffffu, gt, o);
-            eq += __shfl_xor_sync(0xffffffffu, eq, o);
-        }
-        if (lane == 0) S.reg_gt[r] = (int)gt, S.reg_eq[r] = (int)eq;
+        for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+        if (lane == 0) S.reg_gt[r] = (int)c;
     }
     __syncthreads();
-    uint32_t* tie_idx = S.hist;  // reused: up to kTkBins tie indices
     for (int r = warp; r < nreg; r += kTkWarps) {
-        uint32_t gbase = 0, ebase = 0;
-        for (int q = 0; q < r; ++q) gbase += (uint32_t)S.reg_gt[q], ebase += (uint32_t)S.reg_eq[q];
+        uint32_t base = 0;
+        for (int q = 0; q < r; ++q) base += (uint32_t)S.reg_gt[q];
         for (int e0 = 0; e0 < S.reg_cnt[r]; e0 += 32) {
             const int e = e0 + lane;
             const bool in = e < S.reg_cnt[r];
-            const uint32_t key = in ? S.cand_key[S.reg_off[r] + e] : 0u;
-            const int ix = in ? S.cand_idx[S.reg_off[r] + e] : 0;
-            const bool gt = in && key > tau, eq = in && key == tau;
-            const uint32_t bg = __ballot_sync(0xffffffffu, gt), be = __ballot_sync(0xffffffffu, eq);
-            const uint32_t below = (1u << lane) - 1u;
-            if (gt) out[gbase + __popc(bg & below)] = ix;
-            if (eq) {
-                const uint32_t p = ebase + __popc(be & below);
-                if (T == ties) out[(uint32_t)k - ties + p] = ix;
-                else tie_idx[p] = (uint32_t)ix;
-            }
-            gbase += __popc(bg);
-            ebase += __popc(be);
-        }
-    }
-    if (T != ties) {
-        // the `ties` lowest indices among the T tied keys, ascending
-        __syncthreads();
-        for (uint32_t a = tid; a < T; a += kTkThreads) {
-            const uint32_t ia = tie_idx[a];
-            uint32_t rank = 0;
-            for (uint32_t b = 0; b < T; ++b) rank += tie_idx[b] < ia;
-            if (rank < ties) out[(uint32_t)k - ties + rank] = (int)ia;
+            const int ix = in ? S.reg_ip[r][e] : 0;
+            const bool keep = in && kept(S.reg_kp[r][e], (uint32_t)ix);
+            const uint32_t bk = __ballot_sync(0xffffffffu, keep);
+            if (keep) out[base + __popc(bk & ((1u << lane) - 1u))] = ix;
+            base += __popc(bk);
         }
     }
     return true;
 }
 
 // Exact radix select over the row in global memory (the fallback): histogram passes of
-// 10 + 10 + 10 + 2 bits fix tau and the number of ties to keep, then one ordered pass writes
-// keys > tau and the lowest-index ties, ascending.
-__device__ __noinline__ void topk_global(TopkSmem& S, const float* row, int n, int k, int* out) {
+// 10 + 10 + 10 + 2 bits fix tau and the number of ties to keep, a scan finds the last kept tie,
+// then the kept keys are written in the same order as the fast path (region by region).
+__device__ __noinline__ void topk_global(TopkSmem& S, const float* row, int lo, int n, int k, int* out) {
     const int tid = threadIdx.x;
     uint32_t pval = 0, need = (uint32_t)k;
     int fixed = 32;
@@ -334,7 +358,7 @@ __device__ __noinline__ void topk_global(TopkSmem& S, const float* row, int n, i
         __syncthreads();
         clear_hist(S, nbins);
         __syncthreads();
-        for (int e = tid; e < n; e += kTkThreads) {
+        for (int e = lo + tid; e < n; e += kTkThreads) {
             const uint32_t key = score_key(row[e]);
             if (fixed >= 32 || (key >> fixed) == (pval >> fixed)) atomicAdd(&S.hist[(key >> sh) & (nbins - 1)], 1u);
         }
@@ -345,18 +369,38 @@ __device__ __noinline__ void topk_global(TopkSmem& S, const float* row, int n, i
         fixed = sh;
     }
     const uint32_t tau = pval, ties = need;
-    uint32_t gt_seen = 0, eq_seen = 0;
-    for (int e0 = 0; e0 < n; e0 += kTkThreads) {
+    // the kept ties are the `ties` lowest-index keys equal to tau: count ties per 32-key piece in
+    // index order to find the last kept tie's index
+    uint32_t eq_seen = 0;
+    int tie_end = n;  // keys == tau with index < tie_end are kept
+    for (int e0 = lo; e0 < n; e0 += kTkThreads) {
         const int e = e0 + tid;
-        const uint32_t key = e < n ? score_key(row[e]) : 0u;
-        const uint32_t gt = (e < n && key > tau) ? 1u : 0u;
-        const uint32_t eq = (e < n && key == tau) ? 1u : 0u;
+        const uint32_t eq = (e < n && score_key(row[e]) == tau) ? 1u : 0u;
         uint32_t total;
-        const uint32_t ex = block_excl_scan(S, gt | (eq << 16), total);
-        const uint32_t eq_before = eq_seen + (ex >> 16);
-        if (gt || (eq && eq_before < ties)) out[gt_seen + (ex & 0xFFFFu) + min(eq_before, ties)] = e;
-        gt_seen += total & 0xFFFFu;
-        eq_seen += total >> 16;
+        const uint32_t ex = block_excl_scan(S, eq, total);
+        if (eq && eq_seen + ex == ties - 1) S.sel_gt = (uint32_t)e + 1;  // the last kept tie
+        __syncthreads();
+        eq_seen += total;
+        if (eq_seen >= ties) {
+            tie_end = (int)S.sel_gt;
+            break;
+        }
+    }
+    // emit region by region (region = (e >> 5) & 3), ascending within a region
+    uint32_t written = 0;
+    for (int region = 0; region < 4; ++region) {
+        for (int p0 = (lo >> 5); p0 * 32 < n; p0 += kTkThreads / 32) {
+            // warp w handles piece p = p0 + w if it belongs to this region
+            const int p = p0 + (tid >> 5);
+            const int e = p * 32 + (tid & 31);
+            const bool mine = (p & 3) == region;
+            const uint32_t key = (mine && e >= lo && e < n) ? score_key(row[e]) : 0u;
+            const bool keep = mine && e >= lo && e < n && (key > tau || (key == tau && e < tie_end));
+            uint32_t total;
+            const uint32_t ex = block_excl_scan(S, keep ? 1u : 0u, total);
+            if (keep) out[written + ex] = e;
+            written += total;
+        }
     }
 }
 
@@ -365,20 +409,30 @@ __device__ __forceinline__ uint32_t rank_target(long long m, long long n, int k)
     return (uint32_t)max(1LL, min(m - 1, (3LL * k * m + 2LL * n - 1) / (2LL * n)));
 }
 
-// Sample s4 evenly spaced float4 of float4 range [g_lo, g_hi) into keys[base .. base + 4*s4).
-__device__ __forceinline__ void take_samples(uint32_t* keys, int base, const float4* row4, int g_lo, int g_hi, int n,
-                                             int s4) {
-    for (int i = threadIdx.x; i < s4; i += kTkThreads) {
-        const int g = g_lo + (int)(((long long)i * (g_hi - g_lo)) / s4);
-        uint32_t kk[4] = {0u, 0u, 0u, 0u};
-        if (g < g_hi) {
-            const float4 v = row4[g];
-            const float f[4] = {v.x, v.y, v.z, v.w};
+// Sample s4 evenly spaced float4 of float4 range [g_lo, g_hi) into keys[base .. base + 4*s4); all
+// of a thread's loads are issued before any is used.
+__device__ __forceinline__ void take_samples(uint32_t* keys, int base, const float4* row4, int g_lo, int g_hi, int e_lo,
+                                             int n, int s4) {
+    constexpr int kPer = kTkMaxSample4 / kTkThreads;
+    float4 v[kPer];
+    int gg[kPer];
+    // position of sample i: g_lo + floor(i * span / s4), via a 32.32 fixed-point step
+    const unsigned long long step = ((unsigned long long)(g_hi - g_lo) << 32) / (unsigned)max(s4, 1);
 #pragma unroll
-            for (int j = 0; j < 4; ++j) kk[j] = g * 4 + j < n ? score_key(f[j]) : 0u;
-        }
+    for (int u = 0; u < kPer; ++u) {
+        const int i = threadIdx.x + u * kTkThreads;
+        gg[u] = g_lo + (int)(((unsigned long long)i * step) >> 32);
+        v[u] = (i < s4 && gg[u] < g_hi) ? row4[gg[u]] : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
 #pragma unroll
-        for (int j = 0; j < 4; ++j) keys[base + 4 * i + j] = kk[j];
+    for (int u = 0; u < kPer; ++u) {
+        const int i = threadIdx.x + u * kTkThreads;
+        if (i >= s4) continue;
+        const int g = gg[u];
+        const float f[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            keys[base + 4 * i + j] = (g < g_hi && g * 4 + j < n && g * 4 + j >= e_lo) ? score_key(f[j]) : 0u;
     }
 }
 
@@ -393,36 +447,38 @@ __device__ __forceinline__ uint32_t retarget(uint32_t rs, uint32_t c, long long 
     return (uint32_t)max(1LL, min(m - 1, r2));
 }
 
-__global__ void __launch_bounds__(kTkThreads) topk_kernel(const TopkParams P) {
+__global__ void __launch_bounds__(kTkThreads, 6) topk_kernel(const TopkParams P) {
     extern __shared__ __align__(1024) uint8_t topk_smem[];
     TopkSmem& S = *reinterpret_cast<TopkSmem*>(topk_smem);
     const int r = blockIdx.x, tid = threadIdx.x, warp = tid >> 5;
     const int n = (int)row_length(P, r, tid == 0);
+    const int lo = row_first_key(P, n), ne = n - lo;  // competing keys: [lo, n)
     const int k = P.k;
     int* out = P.idx + (long long)r * k;
-    if (n <= k) {
-        for (int j = tid; j < k; j += kTkThreads) out[j] = j < n ? j : -1;
+    if (ne <= k) {
+        for (int j = tid; j < k; j += kTkThreads) out[j] = j < ne ? lo + j : -1;
         return;
     }
     const float* row = P.scores + (long long)r * P.ld;
     const float4* row4 = reinterpret_cast<const float4*>(row);
-    const int n4 = (n + 3) >> 2;
-    const int s4 = sample_count4(n4, 1);
+    const int n4 = (n + 3) >> 2, g0 = lo >> 2;
+    const int s4 = sample_count4(n4 - g0, 1);
     const long long m = 4LL * s4;
-    uint32_t rs = (uint32_t)rank_target(m, n, k);
+    uint32_t rs = (uint32_t)rank_target(m, ne, k);
     bool done = false;
     for (int attempt = 0; attempt < 2 && !done; ++attempt) {
         // ---- threshold estimate (rows of up to kTkCap scores keep them all)
         uint32_t T0 = 0;
-        if (n > kTkCap) {
+        if (ne > kTkCap) {
             if (attempt > 0) __syncthreads();
-            take_samples(S.cand_key, 0, row4, 0, n4, n, s4);
+            take_samples(S.cand_key, 0, row4, g0, n4, lo, n, s4);
             T0 = sample_threshold(S, (int)m, rs);
         }
         // ---- one streaming pass: scores >= T0 into the 4 warp regions
-        const uint32_t c = stream_collect(S, row4, 0, n4, n, key_floor_float(T0), warp * kTkRegion);
+        const uint32_t c = stream_collect(S, row4, g0, n4, lo, n, key_floor_float(T0), warp * kTkRegion);
         if ((tid & 31) == 0) {
-            S.reg_off[warp] = warp * kTkRegion;
+            S.reg_kp[warp] = S.cand_key + warp * kTkRegion;
+            S.reg_ip[warp] = S.cand_idx + warp * kTkRegion;
             S.reg_cnt[warp] = (int)min(c, (uint32_t)kTkRegion);
             S.reg_gt[warp] = (int)c;
         }
@@ -443,12 +499,13 @@ __global__ void __launch_bounds__(kTkThreads) topk_kernel(const TopkParams P) {
             if (!done) atomicAdd(&g_counters[1 + 3 * attempt], 1ull);  // [1] first miss, [4] second miss
         }
     }
-    if (!done) topk_global(S, row, n, k, out);
+    if (!done) topk_global(S, row, lo, n, k, out);
 }
 
 // Few long rows (decode): a cluster of kTkCluster CTAs per row.  Each CTA samples and streams
-// 1/kTkCluster of the row; the sample keys and the candidate regions meet in CTA 0 through
-// distributed shared memory; CTA 0 refines and writes the row.
+// 1/kTkCluster of the row; the sample keys go to CTA 0, which sets the threshold, gathers every
+// CTA's candidate regions through distributed shared memory, then refines and writes the row.
+// Dynamic shared memory: sizeof(TopkSmem) + kTkCap * 8 bytes (CTA 0's gather buffer).
 __global__ void __launch_bounds__(kTkThreads) topk_cluster_kernel(const TopkParams P) {
     extern __shared__ __align__(1024) uint8_t topk_smem[];
     __shared__ int src_cnt[kTkMaxRegions];
@@ -457,27 +514,29 @@ __global__ void __launch_bounds__(kTkThreads) topk_cluster_kernel(const TopkPara
     const int crank = (int)cluster.block_rank();
     const int r = blockIdx.x / kTkCluster, tid = threadIdx.x, warp = tid >> 5;
     const int n = (int)row_length(P, r, tid == 0 && crank == 0);
+    const int lo = row_first_key(P, n), ne = n - lo;  // competing keys: [lo, n)
     const int k = P.k;
     int* out = P.idx + (long long)r * k;
-    if (n <= k) {  // uniform over the cluster
+    if (ne <= k) {  // uniform over the cluster
         if (crank == 0)
-            for (int j = tid; j < k; j += kTkThreads) out[j] = j < n ? j : -1;
+            for (int j = tid; j < k; j += kTkThreads) out[j] = j < ne ? lo + j : -1;
         return;
     }
     const float* row = P.scores + (long long)r * P.ld;
     const float4* row4 = reinterpret_cast<const float4*>(row);
-    const int n4 = (n + 3) >> 2;
-    const int seg = (n4 + kTkCluster - 1) / kTkCluster;
-    const int g_lo = min(n4, crank * seg), g_hi = min(n4, g_lo + seg);
+    const int n4 = (n + 3) >> 2, gw = lo >> 2;
+    // segments of whole groups of 4 pieces (32 float4), so regions keep their meaning across CTAs
+    const int seg = ((n4 - (gw & ~31) + kTkCluster - 1) / kTkCluster + 31) & ~31;
+    const int g_lo = min(n4, max(gw, (gw & ~31) + crank * seg)), g_hi = min(n4, (gw & ~31) + (crank + 1) * seg);
     TopkSmem* S0 = cluster.map_shared_rank(&S, 0);
 
-    const int s4 = sample_count4(n4, kTkCluster);  // per CTA
+    const int s4 = sample_count4(n4 - gw, kTkCluster);  // per CTA
     const long long m = 4LL * s4 * kTkCluster;
-    uint32_t rs = (uint32_t)rank_target(m, n, k);
+    uint32_t rs = (uint32_t)rank_target(m, ne, k);
     bool done = false;
     for (int attempt = 0; attempt < 2; ++attempt) {
         // ---- samples of every segment into CTA 0, which computes T0 and hands it to every CTA
-        take_samples(S0->cand_key, 4 * crank * s4, row4, g_lo, g_hi, n, s4);
+        take_samples(S0->cand_key, 4 * crank * s4, row4, g_lo, g_hi, lo, n, s4);
         cluster.sync();
         if (crank == 0) {
             const uint32_t t0 = sample_threshold(S, (int)m, rs);
@@ -487,7 +546,7 @@ __global__ void __launch_bounds__(kTkThreads) topk_cluster_kernel(const TopkPara
         const uint32_t T0 = S.T0;
 
         // ---- stream this CTA's segment into its warp regions
-        const uint32_t c = stream_collect(S, row4, g_lo, g_hi, n, key_floor_float(T0), warp * kTkRegion);
+        const uint32_t c = stream_collect(S, row4, g_lo, g_hi, lo, n, key_floor_float(T0), warp * kTkRegion);
         if ((tid & 31) == 0) S.reg_gt[warp] = (int)c;
         cluster.sync();
 
@@ -502,25 +561,36 @@ __global__ void __launch_bounds__(kTkThreads) topk_cluster_kernel(const TopkPara
             }
             fits = fits && total >= (uint32_t)k && total <= (uint32_t)kTkCap;
             if (fits) {
-                // gather every region, CTA-major then warp: CTA 0's own regions are compacted in
-                // place (destination never above source; read, barrier, write per chunk)
-                int off = 0;
-                for (int q = 0; q < kTkMaxRegions; ++q) {
-                    const int cnt = src_cnt[q];
-                    const TopkSmem* Src = cluster.map_shared_rank(&S, q / kTkWarps);
-                    const int src_off = (q % kTkWarps) * kTkRegion;
-                    for (int e0 = 0; e0 < cnt; e0 += kTkThreads) {
-                        const int e = e0 + tid;
-                        uint32_t key = 0;
-                        int ix = 0;
-                        if (e < cnt) key = Src->cand_key[src_off + e], ix = Src->cand_idx[src_off + e];
-                        __syncthreads();
-                        if (e < cnt) S.cand_key[off + e] = key, S.cand_idx[off + e] = ix;
+                // gather every CTA's regions into a local buffer, region-major (region w of CTA 0,
+                // of CTA 1, ...), in one flattened pass so the remote loads overlap; region w of
+                // the row then stays one ascending run, as in the one-CTA kernel
+                uint32_t* gkey = reinterpret_cast<uint32_t*>(topk_smem + sizeof(TopkSmem));
+                int* gidx = reinterpret_cast<int*>(gkey + kTkCap);
+                __shared__ int src_pre[kTkMaxRegions + 1];
+                if (tid == 0) {
+                    int acc = 0;
+                    for (int q = 0; q < kTkMaxRegions; ++q) {  // q = warp * kTkCluster + cta
+                        src_pre[q] = acc;
+                        acc += src_cnt[(q % kTkCluster) * kTkWarps + q / kTkCluster];
                     }
-                    if (tid == 0) S.reg_off[q] = off, S.reg_cnt[q] = cnt;
-                    off += cnt;
+                    src_pre[kTkMaxRegions] = acc;
                 }
-                if (tid == 0) S.nreg = kTkMaxRegions;
+                __syncthreads();
+#pragma unroll 4
+                for (int f = tid; f < (int)total; f += kTkThreads) {
+                    int q = 0;
+                    while (q + 1 < kTkMaxRegions && src_pre[q + 1] <= f) ++q;
+                    const int e = f - src_pre[q];
+                    const TopkSmem* Src = cluster.map_shared_rank(&S, q % kTkCluster);
+                    gkey[f] = Src->cand_key[(q / kTkCluster) * kTkRegion + e];
+                    gidx[f] = Src->cand_idx[(q / kTkCluster) * kTkRegion + e];
+                }
+                if (tid < kTkWarps) {
+                    S.reg_kp[tid] = gkey + src_pre[tid * kTkCluster];
+                    S.reg_ip[tid] = gidx + src_pre[tid * kTkCluster];
+                    S.reg_cnt[tid] = src_pre[(tid + 1) * kTkCluster] - src_pre[tid * kTkCluster];
+                }
+                if (tid == 0) S.nreg = kTkWarps;
                 __syncthreads();
                 done = refine_and_emit(S, T0, k, out);
             }
@@ -543,7 +613,7 @@ __global__ void __launch_bounds__(kTkThreads) topk_cluster_kernel(const TopkPara
         rs = S.red[0];
         if (done) break;
     }
-    if (crank == 0 && !done) topk_global(S, row, n, k, out);
+    if (crank == 0 && !done) topk_global(S, row, lo, n, k, out);
     cluster.sync();  // peers keep their shared memory alive until CTA 0 is done with it
 }
 

@@ -75,14 +75,25 @@ dsa_status dsa_index(const void *qI, const void *kI, const void *w, int Lq, int6
  * Step 2 -- per-row top-k.  Row i holds n_i = q_pos0+i+1 valid scores (row i at
  * scores + i*ld_scores, ld_scores a multiple of 4 and >= q_pos0+Lq).
  *   idx     int32 [Lq, k]: the min(k, n_i) keys with the largest scores (equal scores: lower key
- *           index first), then -1 padding.  Exact and deterministic; the order within a row is
- *           fixed (keys above the threshold bin by ascending index, then the remaining selected
- *           keys by ascending index) but callers should treat a row as a set.
+ *           index first), then -1 padding.  Exact and deterministic: a row's output depends
+ *           only on that row's scores (not on Lq, chunking or the kernel variant).  Order within
+ *           a row: the selected keys grouped by region ((index / 32) mod 4, regions 0..3 in turn),
+ *           ascending within a region; callers may treat a row as a set.
  *   ws, ws_bytes  unused (may be NULL/0); kept so callers can pass a workspace uniformly.
  * Cites: page gsyq.cn section 一 (top 2048 per token), section 八 (deterministic top-k).
  */
 dsa_status dsa_topk(const float *scores, int64_t ld_scores, int Lq, int64_t q_pos0, int k, int32_t *idx,
                     void *ws, size_t ws_bytes, dsa_stream_t stream);
+
+/*
+ * Step 2 with a sliding window (SW-DSA: page "DSA注意力机制：多模态学习中的强化推理新范式",
+ * showapi.com, section 1.4, restricts the selection to a local window).  As dsa_topk, except
+ * that row i (query position t = q_pos0+i) selects among keys max(0, t-window+1) .. t only:
+ * the min(k, min(window, t+1)) best of them, -1 padded.  window = 0 means no window (identical to
+ * dsa_topk); window < 0 is invalid.
+ */
+dsa_status dsa_topk_window(const float *scores, int64_t ld_scores, int Lq, int64_t q_pos0, int k, int64_t window,
+                           int32_t *idx, dsa_stream_t stream);
 
 /*
  * Step 3 -- sparse attention over selected keys (prefill layout).
@@ -113,6 +124,31 @@ dsa_status dsa_sparse_attn(const void *q, const void *k, const void *v, const in
 dsa_status dsa_prefill(const void *q, const void *k, const void *v, const void *qI, const void *kI, const void *w,
                        int64_t L, int Hq, int Hkv, int D, int HI, int dI, int topk, float scale, void *out,
                        int32_t *idx_out, void *ws, size_t ws_bytes, dsa_stream_t stream);
+
+/*
+ * Steps 1-3 for the query rows row0 .. row0+rows-1 of one causal sequence (chunked prefill, or
+ * one rank's share of a sequence whose rows are spread over GPUs).  Row-local arrays:
+ *   q bf16 [rows, Hq, D]; qI bf16 [rows, HI, dI]; w bf16 [rows, HI]; out bf16 [rows, Hq, D];
+ *   idx_out int32 [rows, topk] or NULL.  Whole-sequence arrays, at least row0+rows positions:
+ *   k, v bf16 [.., Hkv, D]; kI bf16 [.., dI].  window as in dsa_prefill_window (0 = none).
+ *   ws      workspace for score rows of length row0+rows (see dsa_workspace_size with
+ *           L = row0+rows).
+ * Processing consecutive row ranges gives exactly dsa_prefill's results for those rows.
+ */
+dsa_status dsa_prefill_rows(const void *q, const void *k, const void *v, const void *qI, const void *kI,
+                            const void *w, int64_t row0, int64_t rows, int Hq, int Hkv, int D, int HI, int dI,
+                            int topk, int64_t window, float scale, void *out, int32_t *idx_out, void *ws,
+                            size_t ws_bytes, dsa_stream_t stream);
+
+/*
+ * dsa_prefill with a sliding window of `window` keys per query (SW-DSA, see dsa_topk_window): the
+ * indexer skips key tiles that lie wholly before every window of a query block, top-k selects
+ * within the window, attention runs over the selected keys.  window = 0: identical to dsa_prefill.
+ */
+dsa_status dsa_prefill_window(const void *q, const void *k, const void *v, const void *qI, const void *kI,
+                              const void *w, int64_t L, int Hq, int Hkv, int D, int HI, int dI, int topk,
+                              int64_t window, float scale, void *out, int32_t *idx_out, void *ws, size_t ws_bytes,
+                              dsa_stream_t stream);
 
 /*
  * One decode step for B sequences, each with one new token (the pages' decode path: page

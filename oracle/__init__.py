@@ -37,9 +37,9 @@ def _load():
         lib = ctypes.CDLL(_SO)
         p, i64, i32, f64 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_double
         lib.oracle_index_rows.argtypes = [p, p, p, p, i64, i32, i32, p, i64]
-        lib.oracle_topk_rows.argtypes = [p, i64, p, i64, i32, p, p]
+        lib.oracle_topk_rows.argtypes = [p, i64, p, p, i64, i32, p, p]
         lib.oracle_sparse_attn_rows.argtypes = [p, p, p, p, i64, i32, i32, i32, i32, f64, p, p]
-        lib.oracle_dsa_rows.argtypes = [p, p, p, p, p, p, p, i64, i32, i32, i32, i32, i32, i32, f64,
+        lib.oracle_dsa_rows.argtypes = [p, p, p, p, p, p, p, i64, i32, i32, i32, i32, i32, i32, i64, f64,
                                         p, p, p, p, i64, p, p]
         lib.oracle_num_threads.restype = i32
         for f in ("oracle_index_rows", "oracle_topk_rows", "oracle_sparse_attn_rows",
@@ -75,15 +75,20 @@ def index_rows(qI: np.ndarray, w: np.ndarray, kI: np.ndarray, t_rows) -> np.ndar
     return scores
 
 
-def topk_rows(scores: np.ndarray, n_valid, k: int):
-    """(idx int32 [rows, k] ordered by (score desc, index asc), -1 padded; tau float64 [rows])."""
+def topk_rows(scores: np.ndarray, n_valid, k: int, window: int = 0):
+    """(idx int32 [rows, k] ordered by (score desc, index asc), -1 padded; tau float64 [rows]).
+
+    With window > 0 only keys n-window .. n-1 of a row with n valid keys compete."""
     scores = _c(scores, np.float64)
     n_valid = _c(np.atleast_1d(n_valid), np.int64)
     nr, ld = scores.shape
     assert n_valid.size == nr and int(n_valid.max(initial=0)) <= ld
+    first = None
+    if window > 0:
+        first = _c(np.maximum(0, n_valid - window), np.int64)
     idx = np.empty((nr, k), dtype=np.int32)
     tau = np.empty(nr)
-    _load().oracle_topk_rows(_ptr(scores), ld, _ptr(n_valid), nr, k, _ptr(idx), _ptr(tau))
+    _load().oracle_topk_rows(_ptr(scores), ld, _ptr(n_valid), _ptr(first), nr, k, _ptr(idx), _ptr(tau))
     return idx, tau
 
 
@@ -106,12 +111,13 @@ def sparse_attn_rows(q: np.ndarray, k: np.ndarray, v: np.ndarray, idx: np.ndarra
 
 
 def dsa_rows(q_rows, qI_rows, w_rows, k, v, kI, t_rows, topk: int, scale: float,
-             keep_scores: bool = False) -> dict:
+             keep_scores: bool = False, window: int = 0) -> dict:
     """All three steps for query positions t_rows of one causal sequence.
 
     q_rows/qI_rows/w_rows hold the rows of those positions only; k, v, kI hold the whole prefix.
     Returns idx, out, lse, tau (score of the last selected key), absmax (max |score| of the row)
-    and, with keep_scores, the score rows (NaN beyond t).
+    and, with keep_scores, the score rows (NaN beyond t).  window > 0: sliding-window top-k over
+    keys t-window+1 .. t (the scores and absmax still cover the whole causal row).
     """
     t_rows = _c(np.atleast_1d(t_rows), np.int64)
     nr = t_rows.size
@@ -130,7 +136,7 @@ def dsa_rows(q_rows, qI_rows, w_rows, k, v, kI, t_rows, topk: int, scale: float,
     ld = int(t_rows.max()) + 1
     scores = np.full((nr, ld), np.nan) if keep_scores else None
     _load().oracle_dsa_rows(_ptr(q_rows), _ptr(qI_rows), _ptr(w_rows), _ptr(k), _ptr(v), _ptr(kI),
-                            _ptr(t_rows), nr, Hq, Hkv, D, HI, dI, topk, float(scale), _ptr(idx),
+                            _ptr(t_rows), nr, Hq, Hkv, D, HI, dI, topk, int(window), float(scale), _ptr(idx),
                             _ptr(out), _ptr(lse), _ptr(scores), ld, _ptr(tau), _ptr(absmax))
     res = {"idx": idx, "out": out, "lse": lse, "tau": tau, "absmax": absmax}
     if keep_scores:

@@ -75,16 +75,17 @@ static int by_score_then_index(const void *pa, const void *pb) {
     return (a->idx > b->idx) - (a->idx < b->idx);
 }
 
-/* Step 2 for one row: idx[0..k) = first min(k, n) keys in that order, then -1.
- * Returns the score of the last selected key (the k-th score when n >= k). */
-static double topk_row(const double *scores, int64_t n, int k, int32_t *idx) {
-    scored_key *buf = (scored_key *)malloc((size_t)(n > 0 ? n : 1) * sizeof(scored_key));
-    for (int64_t s = 0; s < n; ++s) {
-        buf[s].score = scores[s];
-        buf[s].idx = (int32_t)s;
+/* Step 2 for one row, keys lo..n-1 competing: idx[0..k) = first min(k, n-lo) of them in that
+ * order, then -1.  Returns the score of the last selected key (the k-th score when n-lo >= k). */
+static double topk_row(const double *scores, int64_t lo, int64_t n, int k, int32_t *idx) {
+    int64_t c = n - lo;
+    scored_key *buf = (scored_key *)malloc((size_t)(c > 0 ? c : 1) * sizeof(scored_key));
+    for (int64_t s = lo; s < n; ++s) {
+        buf[s - lo].score = scores[s];
+        buf[s - lo].idx = (int32_t)s;
     }
-    qsort(buf, (size_t)n, sizeof(scored_key), by_score_then_index);
-    int64_t m = n < k ? n : k;
+    qsort(buf, (size_t)c, sizeof(scored_key), by_score_then_index);
+    int64_t m = c < k ? c : k;
     for (int64_t j = 0; j < m; ++j) idx[j] = buf[j].idx;
     for (int64_t j = m; j < k; ++j) idx[j] = -1;
     double tau = m > 0 ? buf[m - 1].score : 0.0;
@@ -146,13 +147,14 @@ void oracle_index_rows(const uint16_t *qI, const uint16_t *w, const uint16_t *kI
         index_row(qI + r * HI * dI, w + r * HI, kI, t_rows[r] + 1, HI, dI, scores + r * ld);
 }
 
-/* Step 2.  n_valid[r] keys per row (t + 1 for a causal row).  tau[r] (nullable) receives the
- * score of the last selected key. */
-void oracle_topk_rows(const double *scores, int64_t ld, const int64_t *n_valid, int64_t nr, int k, int32_t *idx,
-                      double *tau) {
+/* Step 2.  n_valid[r] keys per row (t + 1 for a causal row); with first[r] (nullable) only keys
+ * first[r] .. n_valid[r]-1 compete (a sliding window).  tau[r] (nullable) receives the score of
+ * the last selected key. */
+void oracle_topk_rows(const double *scores, int64_t ld, const int64_t *n_valid, const int64_t *first, int64_t nr,
+                      int k, int32_t *idx, double *tau) {
 #pragma omp parallel for schedule(dynamic, 1)
     for (int64_t r = 0; r < nr; ++r) {
-        double t = topk_row(scores + r * ld, n_valid[r], k, idx + r * k);
+        double t = topk_row(scores + r * ld, first ? first[r] : 0, n_valid[r], k, idx + r * k);
         if (tau) tau[r] = t;
     }
 }
@@ -168,12 +170,13 @@ void oracle_sparse_attn_rows(const uint16_t *q, const uint16_t *kc, const uint16
 }
 
 /* Steps 1-3 for a set of rows of one causal sequence, without keeping more than one score row
- * per thread.  scores (nullable) [nr, ld] keeps the score rows; tau [nr] (nullable); absmax[nr]
+ * per thread.  window > 0: only keys t-window+1 .. t compete in step 2 (sliding-window DSA,
+ * page "DSA注意力机制：多模态学习中的强化推理新范式", showapi.com, section 1.4).  scores (nullable) [nr, ld] keeps the score rows; tau [nr] (nullable); absmax[nr]
  * (nullable) receives max_s |score(t, s)|. */
 void oracle_dsa_rows(const uint16_t *q, const uint16_t *qI, const uint16_t *w, const uint16_t *kc,
                      const uint16_t *vc, const uint16_t *kI, const int64_t *t_rows, int64_t nr, int Hq, int Hkv,
-                     int D, int HI, int dI, int k, double scale, int32_t *idx, double *out, double *lse,
-                     double *scores, int64_t ld, double *tau, double *absmax) {
+                     int D, int HI, int dI, int k, int64_t window, double scale, int32_t *idx, double *out,
+                     double *lse, double *scores, int64_t ld, double *tau, double *absmax) {
 #pragma omp parallel for schedule(dynamic, 1)
     for (int64_t r = 0; r < nr; ++r) {
         int64_t n = t_rows[r] + 1;
@@ -184,7 +187,8 @@ void oracle_dsa_rows(const uint16_t *q, const uint16_t *qI, const uint16_t *w, c
             for (int64_t s = 0; s < n; ++s) m = fabs(row[s]) > m ? fabs(row[s]) : m;
             absmax[r] = m;
         }
-        double t = topk_row(row, n, k, idx + r * k);
+        int64_t lo = (window > 0 && n > window) ? n - window : 0;
+        double t = topk_row(row, lo, n, k, idx + r * k);
         if (tau) tau[r] = t;
         attend_row(q + r * Hq * D, kc, vc, idx + r * k, k, Hq, Hkv, D, scale, out + r * Hq * D,
                    lse ? lse + r * Hq : NULL);

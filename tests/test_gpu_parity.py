@@ -320,3 +320,81 @@ def test_profile_and_launch_counter(cuda_ok, tiny):
     assert dsa.launch_count() - n0 == 3
     assert prof["indexer"]["launches"] == 1 and prof["topk"]["launches"] == 1 and prof["sparse_attn"]["launches"] == 1
     assert all(v["ms"] > 0 for k, v in prof.items() if v["launches"])
+
+
+@pytest.mark.parametrize("W", [1, 100, 3000])
+def test_topk_window_exact_on_oracle_scores(cuda_ok, tiny, W):
+    """Sliding-window top-k (SW-DSA) on the oracle's fp32 scores equals the oracle's, exactly."""
+    cfg, x, ref = tiny
+    L = cfg.L
+    s32 = np.nan_to_num(ref["scores"], nan=0.0).astype(np.float32)
+    idx = torch.empty((L, cfg.k), dtype=torch.int32, device="cuda")
+    dsa.dsa_topk(torch.from_numpy(s32).cuda(), 0, cfg.k, idx, window=W)
+    assert dsa.sync_status() == dsa.DSA_OK
+    want, _ = oracle.topk_rows(s32.astype(np.float64), np.arange(L) + 1, cfg.k, window=W)
+    got = idx.cpu().numpy()
+    for r in range(L):
+        assert sorted(got[r].tolist()) == sorted(want[r].tolist()), r
+
+
+@pytest.mark.parametrize("name,W", [("tiny", 300), ("32k", 4096), ("32k", 40000)])
+def test_prefill_window_sampled_rows(cuda_ok, name, W):
+    cfg = synth.CONFIGS[name]
+    x = synth.inputs(cfg, 0, cfg.L)
+    L = cfg.L
+    out = torch.empty((L, cfg.Hq, cfg.D), dtype=torch.bfloat16, device="cuda")
+    idx = torch.empty((L, cfg.k), dtype=torch.int32, device="cuda")
+    d = {n: dev(a) for n, a in x.items()}
+    dsa.dsa_prefill(d["q"], d["k"], d["v"], d["qI"], d["kI"], d["w"], cfg.k, cfg.scale, out, idx, window=W)
+    assert dsa.sync_status() == dsa.DSA_OK
+    rows = np.unique(np.concatenate([[0, W - 2, W - 1, W, W + 1, L - 1], synth.sample_rows(13, L, seed=5)]))
+    rows = rows[(rows >= 0) & (rows < L)]
+    ref = oracle.dsa_rows(x["q"][rows], x["qI"][rows], x["w"][rows], x["k"], x["v"], x["kI"], rows, cfg.k,
+                          cfg.scale, keep_scores=True, window=W)
+    gi = idx.cpu().numpy()[rows]
+    n_win = np.minimum(rows + 1, W)
+    for r, t in enumerate(rows):                       # every selected key inside the window
+        sel = gi[r][gi[r] >= 0]
+        assert len(sel) == min(cfg.k, n_win[r]) and sel.min() >= t - W + 1 and sel.max() <= t
+    mm = index_set_mismatch(gi, ref["idx"], ref["scores"], ref["tau"], ref["absmax"], rows + 1)
+    assert mm["out_of_band"] == 0, mm
+    own, _ = oracle.sparse_attn_rows(x["q"][rows], x["k"], x["v"], gi, cfg.scale)
+    assert_output_ok(bf16_tensor_to_f64(out[torch.from_numpy(rows).cuda()]), own, f"window {W}")
+
+
+def test_attention_skips_padding_entries_inside_the_count(cuda_ok):
+    """Entries that name no key (-1, or >= Lk) are skipped wherever they sit in the list."""
+    rng = np.random.default_rng(13)
+    L, Hq, Hkv, topk = 300, 8, 2, 64
+    tq, tk, tv = (torch.from_numpy(rng.standard_normal(sh).astype(np.float32)).to(torch.bfloat16)
+                  for sh in ((L, Hq, 128), (L, Hkv, 128), (L, Hkv, 128)))
+    bits = [t.view(torch.int16).numpy().view(np.uint16) for t in (tq, tk, tv)]
+    idx = np.full((L, topk), -1, dtype=np.int32)
+    for t in range(L):
+        m = min(topk, t + 1)
+        idx[t, :m] = rng.choice(t + 1, size=m, replace=False)
+        holes = rng.choice(m, size=m // 4, replace=False)
+        idx[t, holes[: len(holes) // 2]] = -1
+        idx[t, holes[len(holes) // 2:]] = L + 7            # out of range
+    out = torch.empty((L, Hq, 128), dtype=torch.bfloat16, device="cuda")
+    dsa.dsa_sparse_attn(tq.cuda(), tk.cuda(), tv.cuda(), torch.from_numpy(idx).cuda(), 0, 0.0883883, out)
+    assert dsa.sync_status() == dsa.DSA_OK
+    clean = np.where(idx >= L, -1, idx).astype(np.int32)
+    want, _ = oracle.sparse_attn_rows(bits[0], bits[1], bits[2], clean, 0.0883883)
+    assert_output_ok(bf16_tensor_to_f64(out), want, "holes")
+
+
+def test_prefill_rows_ranges_reproduce_prefill(cuda_ok, c32k):
+    """Consecutive row ranges through dsa_prefill_rows (row-local q/qI/w/out) give exactly the
+    indices and outputs of one dsa_prefill over the whole sequence."""
+    cfg, x = c32k
+    out_full, idx_full = run_prefill(cfg, x)
+    d = {n: dev(a) for n, a in x.items()}
+    out = torch.empty_like(out_full)
+    idx = torch.empty_like(idx_full)
+    for r0, r1 in ((0, 777), (777, 9000), (9000, 20001), (20001, cfg.L)):
+        dsa.dsa_prefill_rows(d["q"][r0:r1], d["k"][:r1], d["v"][:r1], d["qI"][r0:r1], d["kI"][:r1], d["w"][r0:r1],
+                             r0, cfg.k, cfg.scale, out[r0:r1], idx[r0:r1])
+    assert dsa.sync_status() == dsa.DSA_OK
+    assert torch.equal(idx, idx_full)
+    assert torch.equal(out.view(torch.int16), out_full.view(torch.int16))

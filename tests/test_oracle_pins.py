@@ -247,3 +247,27 @@ def test_golden_regression_fixture():
         assert sorted(res["idx"][r][res["idx"][r] >= 0].tolist()) == row["idx_sorted"]
         assert res["tau"][r] == pytest.approx(row["tau"], rel=1e-12)
         np.testing.assert_allclose(res["out"][r, :, :4].ravel(), row["out_head_d0_3"], rtol=1e-10, atol=1e-12)
+
+
+def test_sliding_window_topk_brute_force():
+    """SW-DSA: with window W only keys t-W+1..t compete; W >= t+1 is the full causal row and
+    W = 1 keeps the query's own key."""
+    rng = np.random.default_rng(9)
+    L, HI, dI, k = 60, 2, 16, 9
+    base = rand_bf16(rng, (5, dI))
+    kI = base[rng.integers(0, 5, size=L)]                     # ties again
+    qI, w = rand_bf16(rng, (L, HI, dI)), rand_bf16(rng, (L, HI))
+    scores = oracle.index_rows(qI, w, kI, np.arange(L))
+    full = np.nan_to_num(scores, nan=-np.inf)
+    for W in (1, 7, 20, 1000):
+        idx, _ = oracle.topk_rows(full, np.arange(L) + 1, k, window=W)
+        for t in range(L):
+            lo = max(0, t - W + 1)
+            order = sorted(range(lo, t + 1), key=lambda s: (-scores[t, s], s))[:k]
+            assert list(idx[t][:len(order)]) == order and np.all(idx[t][len(order):] == -1)
+    idx_w, _ = oracle.topk_rows(full, np.arange(L) + 1, k, window=L + 1)
+    idx_f, _ = oracle.topk_rows(full, np.arange(L) + 1, k)
+    assert np.array_equal(idx_w, idx_f)
+    res = oracle.dsa_rows(rand_bf16(rng, (L, 2, 16)), qI, w, rand_bf16(rng, (L, 1, 16)), rand_bf16(rng, (L, 1, 16)),
+                          kI, np.arange(L), k, 0.25, window=1)
+    assert np.array_equal(res["idx"][:, 0], np.arange(L)) and np.all(res["idx"][:, 1:] == -1)

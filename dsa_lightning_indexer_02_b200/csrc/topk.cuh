@@ -65,7 +65,7 @@ struct TopkSmem {
     int cand_idx[kTkCap];
     // candidate regions: keys/indices may live in this CTA's or (cluster) another CTA's shared memory
     const uint32_t* reg_kp[kTkMaxRegions];
-    const int* reg_ip[kTkMaxRegions];
+    int* reg_ip[kTkMaxRegions];
     int reg_cnt[kTkMaxRegions], reg_gt[kTkMaxRegions], reg_eq[kTkMaxRegions];
     int nreg;
     uint32_t red[kTkWarps];
@@ -292,9 +292,12 @@ __device__ __forceinline__ bool refine_and_emit(TopkSmem& S, uint32_t lo, int k,
     const uint32_t bin = fixed >= 32 ? 0u : (pv >> fixed);
     auto above = [&](uint32_t d) { return fixed < 32 && (d >> fixed) > bin; };
     auto in_bin = [&](uint32_t d) { return fixed >= 32 || (d >> fixed) == bin; };
-    // the bin's members (key, index) into a small list; their order does not matter
-    uint32_t* bkey = S.hist;  // reused: up to kTkBins / 2 members
-    uint32_t* bidx = S.hist + kTkBins / 2;
+    // the bin's members: (key, location) into a small list, order irrelevant; each is ranked once
+    // by (key desc, index asc) and the ones not kept are marked (index -1) in place, so that the
+    // passes below test a candidate in O(1)
+    uint32_t* bkey = S.hist;                      // reused: up to kTkBins / 2 members
+    uint32_t* bloc = S.hist + kTkBins / 2;        // region << 16 | position
+    auto loc_idx = [&](uint32_t l) { return S.reg_ip[l >> 16][l & 0xFFFFu]; };
     if (tid == 0) S.sel_bin = 0;
     __syncthreads();
     for (int r = 0; r < nreg; ++r)
@@ -303,26 +306,41 @@ __device__ __forceinline__ bool refine_and_emit(TopkSmem& S, uint32_t lo, int k,
             if (in_bin(key - lo)) {
                 const uint32_t p = atomicAdd(&S.sel_bin, 1u);
                 bkey[p] = key;
-                bidx[p] = (uint32_t)S.reg_ip[r][e];
+                bloc[p] = ((uint32_t)r << 16) | (uint32_t)e;
             }
         }
     __syncthreads();
-    // kept: above the bin, or in it with rank < need by (key desc, index asc)
-    auto kept = [&](uint32_t key, uint32_t ix) {
-        const uint32_t d = key - lo;
-        if (above(d)) return true;
-        if (!in_bin(d)) return false;
-        uint32_t rank = 0;
-        for (uint32_t b2 = 0; b2 < cnt_b; ++b2) {
-            const uint32_t kb = bkey[b2];
-            rank += (kb > key) || (kb == key && bidx[b2] < ix);
+    bool drop[(kTkBins / 2 + kTkThreads - 1) / kTkThreads];
+#pragma unroll
+    for (int j = 0; j < (int)(sizeof(drop) / sizeof(drop[0])); ++j) {
+        const uint32_t a = tid + j * kTkThreads;
+        drop[j] = false;
+        if (a < cnt_b) {
+            const uint32_t ka = bkey[a];
+            const int ia = loc_idx(bloc[a]);
+            uint32_t rank = 0;
+            for (uint32_t b2 = 0; b2 < cnt_b; ++b2) {
+                const uint32_t kb = bkey[b2];
+                rank += (kb > ka) || (kb == ka && loc_idx(bloc[b2]) < ia);
+            }
+            drop[j] = rank >= need;
         }
-        return rank < need;
+    }
+    __syncthreads();  // every rank used the original indices
+#pragma unroll
+    for (int j = 0; j < (int)(sizeof(drop) / sizeof(drop[0])); ++j) {
+        const uint32_t a = tid + j * kTkThreads;
+        if (a < cnt_b && drop[j]) S.reg_ip[bloc[a] >> 16][bloc[a] & 0xFFFFu] = -1;
+    }
+    __syncthreads();
+    auto kept = [&](uint32_t key, int ix) {
+        const uint32_t d = key - lo;
+        return above(d) || (in_bin(d) && ix >= 0);
     };
     // write the kept keys region by region, each region in its own (ascending) order
     for (int r = warp; r < nreg; r += kTkWarps) {
         uint32_t c = 0;
-        for (int e = lane; e < S.reg_cnt[r]; e += 32) c += kept(S.reg_kp[r][e], (uint32_t)S.reg_ip[r][e]);
+        for (int e = lane; e < S.reg_cnt[r]; e += 32) c += kept(S.reg_kp[r][e], S.reg_ip[r][e]);
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
         if (lane == 0) S.reg_gt[r] = (int)c;
@@ -335,7 +353,7 @@ __device__ __forceinline__ bool refine_and_emit(TopkSmem& S, uint32_t lo, int k,
             const int e = e0 + lane;
             const bool in = e < S.reg_cnt[r];
             const int ix = in ? S.reg_ip[r][e] : 0;
-            const bool keep = in && kept(S.reg_kp[r][e], (uint32_t)ix);
+            const bool keep = in && kept(S.reg_kp[r][e], ix);
             const uint32_t bk = __ballot_sync(0xffffffffu, keep);
             if (keep) out[base + __popc(bk & ((1u << lane) - 1u))] = ix;
             base += __popc(bk);
@@ -578,8 +596,10 @@ __global__ void __launch_bounds__(kTkThreads) topk_cluster_kernel(const TopkPara
                 __syncthreads();
 #pragma unroll 4
                 for (int f = tid; f < (int)total; f += kTkThreads) {
-                    int q = 0;
-                    while (q + 1 < kTkMaxRegions && src_pre[q + 1] <= f) ++q;
+                    int q = 0;  // last q with src_pre[q] <= f (binary search)
+#pragma unroll
+                    for (int step = kTkMaxRegions / 2; step > 0; step >>= 1)
+                        if (q + step < kTkMaxRegions && src_pre[q + step] <= f) q += step;
                     const int e = f - src_pre[q];
                     const TopkSmem* Src = cluster.map_shared_rank(&S, q % kTkCluster);
                     gkey[f] = Src->cand_key[(q / kTkCluster) * kTkRegion + e];

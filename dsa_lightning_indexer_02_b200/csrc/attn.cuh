@@ -8,17 +8,20 @@
 // The work is a gather: per token, 2048 keys x Hkv x 128 x (K and V) x 2 bytes = 4 MiB at the
 // 32/4/128 shape against 32 x 128 x 2048 x 4 flop, i.e. 8 flop per byte, far below the ridge
 // of the tensor cores.  The kernel therefore spends its effort on the memory side:
-//   - one CTA per (token, key split); each selected key's K and V rows for all KV heads are
-//     one contiguous Hkv*256-byte span, gathered with coalesced 16-byte cp.async copies into a
-//     3-stage shared-memory ring (rows padded by 16 bytes: conflict-free ldmatrix);
-//   - 2 warps per KV group; a warp owns its group's G query heads (GQA head packing: the
-//     K/V tile it reads from shared memory serves all G heads at once);
+//   - one CTA per (token, key split), two CTAs per SM for up to 8 heads per KV group; each selected key's K and V rows for
+//     all KV heads are one contiguous Hkv*256-byte span, and a producer warp moves each of them
+//     with one bulk copy (the copy engine, not the load/store units, tracks the bytes in
+//     flight) into a ring of 16-key stages; an mbarrier per stage counts the bytes in, another
+//     counts the consumer warps out (rows padded by 16 bytes: conflict-free ldmatrix);
+//   - 8/Hkv consumer warps per KV group, taking the group's stages in turn; a warp owns its
+//     group's G query heads (GQA head packing: the K/V tile it reads from shared memory
+//     serves all G heads at once);
 //   - S^T[keys x heads] = K . Q^T and O^T += V^T . P^T on warp-level bf16 MMAs
 //     (m16n8k16, keys or head-dimension rows as M, 8 heads as N), so no MMA lane is wasted on
 //     the small head count; P^T goes from the accumulator layout to the operand layout with
 //     movmatrix; online softmax in fp32 (exp2 domain);
-//   - slots past the row's count and entries naming no key (index -1 or >= n_keys) are
-//     zero-filled copies with logit -inf.
+//   - slots past the row's count and entries naming no key (index -1 or >= n_keys) copy a
+//     zero row and get logit -inf.
 // With nsplit > 1 every CTA writes unnormalised partial results (O, running max, running sum)
 // for its slice of the index list; attn_combine_kernel merges them.
 #pragma once
@@ -28,9 +31,14 @@
 namespace dsa {
 
 constexpr int kAttnD = 128;
-constexpr int kAttnStages = 3;
-constexpr int kAttnWPG = 2;  // warps per KV group
-constexpr int kAttnIdxWin = 2048;  // index-list window kept in shared memory
+constexpr int kAttnKS = 16;             // keys per stage
+constexpr int kAttnCW = 8;              // consumer warps (Hkv groups x 8/Hkv warps)
+constexpr int kAttnThreads = (kAttnCW + 1) * 32;
+constexpr int kAttnMaxStages = 16;
+constexpr int kAttnStageBudget = 100 * 1024;  // ring bytes per CTA: two CTAs per SM
+
+// Rows of zeros that stand in for slots naming no key (Hkv * 256 bytes at most).
+__device__ __align__(128) uint8_t g_attn_zero_row[4 * kAttnD * 2];
 
 struct AttnParams {
     const __nv_bfloat16* q;   // [T, Hq, D]
@@ -52,23 +60,39 @@ struct AttnParams {
     long long window;         // > 0 (prefill): a row holds at most min(topk, window) keys
 };
 
-__host__ __device__ constexpr int attn_keys_per_stage(int hkv) { return 128 / hkv; }
 __host__ __device__ constexpr int attn_row_bytes(int hkv) { return hkv * kAttnD * 2 + 16; }
-__host__ __device__ constexpr int attn_smem_bytes(int hkv) {
-    return kAttnStages * attn_keys_per_stage(hkv) * attn_row_bytes(hkv) * 2 + kAttnIdxWin * 4 + kAttnStages * 128;
+__host__ __device__ constexpr int attn_stage_bytes(int hkv) { return kAttnKS * attn_row_bytes(hkv) * 2; }
+__host__ __device__ constexpr int attn_stages(int hkv) {
+    return kAttnStageBudget / attn_stage_bytes(hkv) < kAttnMaxStages ? kAttnStageBudget / attn_stage_bytes(hkv)
+                                                                     : kAttnMaxStages;
+}
+// per consumer warp after the loop: [NT][36][32] floats (O fragments, m, l) for the merge
+__host__ __device__ constexpr int attn_xch_bytes(int nt) { return kAttnCW * nt * 36 * 32 * 4; }
+__host__ __device__ constexpr int attn_ring_bytes(int hkv, int nt) {
+    return attn_stages(hkv) * attn_stage_bytes(hkv) > attn_xch_bytes(nt) ? attn_stages(hkv) * attn_stage_bytes(hkv)
+                                                                         : attn_xch_bytes(nt);
+}
+// ring (or merge area) | full[NS], empty[NS] mbarriers | abort flag | valid flags [NS][16]
+__host__ __device__ constexpr int attn_smem_bytes(int hkv, int nt) {
+    return attn_ring_bytes(hkv, nt) + attn_stages(hkv) * 16 + 16 + attn_stages(hkv) * kAttnKS;
 }
 
 // NT: n-tiles of 8 query heads per KV group (G <= 8 * NT).
 template <int NT>
-__global__ void __launch_bounds__(256) sparse_attn_kernel(const AttnParams P) {
+__global__ void __launch_bounds__(kAttnThreads, NT == 1 ? 2 : 1) sparse_attn_kernel(const AttnParams P) {
     extern __shared__ __align__(1024) uint8_t smem[];
     const int Hkv = P.Hkv, G = P.Hq / P.Hkv;
-    const int KS = attn_keys_per_stage(Hkv);        // keys per stage (all groups)
+    const int WPG = kAttnCW / Hkv;                  // consumer warps per KV group
     const int RB = attn_row_bytes(Hkv);             // padded row bytes (K or V of one key)
-    const int STAGE = KS * RB * 2;                  // K rows then V rows
-    const int nthreads = blockDim.x;
+    const int STAGE = attn_stage_bytes(Hkv);        // K rows then V rows
+    const int NS = attn_stages(Hkv);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int grp = warp / kAttnWPG, wsub = warp % kAttnWPG;
+    const int grp = warp / WPG, wsub = warp % WPG;  // consumer warps only
+
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + attn_ring_bytes(Hkv, NT));
+    uint64_t* empty = full + NS;
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + NS);
+    uint8_t* svalid = reinterpret_cast<uint8_t*>(empty + NS) + 16;
 
     const int t = blockIdx.x / P.nsplit;
     const int split = blockIdx.x % P.nsplit;
@@ -88,100 +112,101 @@ __global__ void __launch_bounds__(256) sparse_attn_kernel(const AttnParams P) {
     const int p_begin = split * per_split;
     const int p_end = min(n_sel, p_begin + per_split);
     const int* idx_row = P.idx + (long long)t * P.topk;
-    const int nsteps = p_end > p_begin ? (p_end - p_begin + KS - 1) / KS : 0;
+    const int nsteps = p_end > p_begin ? (p_end - p_begin + kAttnKS - 1) / kAttnKS : 0;
 
-    // ---- Q^T fragments (B operand, K = head dim, N = 8 heads): head lane/4, dims 2*(lane%4)+{0,1}(+8)
-    uint32_t qf[NT][8][2];
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-        const int hl = nt * 8 + (lane >> 2);
-        const bool hv = hl < G;
-        const __nv_bfloat16* qrow = P.q + ((long long)t * P.Hq + grp * G + (hv ? hl : 0)) * kAttnD;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-            const int d = kk * 16 + 2 * (lane & 3);
-            qf[nt][kk][0] = hv ? *reinterpret_cast<const uint32_t*>(qrow + d) : 0u;
-            qf[nt][kk][1] = hv ? *reinterpret_cast<const uint32_t*>(qrow + d + 8) : 0u;
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < NS; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], Hkv);
         }
+        *abort_flag = 0;
+        fence_mbar_init();
     }
-
-    // ---- the index list, kAttnIdxWin entries at a time, in shared memory: the gathers of a stage
-    // are issued without waiting on a global load of their indices
-    int* sidx = reinterpret_cast<int*>(smem + kAttnStages * STAGE);
-    // per stage and key: 1 if the slot holds a usable key (in range, index in [0, n_keys))
-    uint8_t* svalid = reinterpret_cast<uint8_t*>(sidx + kAttnIdxWin);
-    int win_off = 0;  // window covers slots [p_begin + win_off, p_begin + win_off + kAttnIdxWin)
-    auto fill_window = [&]() {
-        for (int i = threadIdx.x; i < kAttnIdxWin; i += nthreads) {
-            const int p = p_begin + win_off + i;
-            sidx[i] = p < p_end ? __ldg(idx_row + p) : -1;
-        }
-    };
-    fill_window();
     __syncthreads();
 
-    // ---- async gather of one stage: KS keys x (all KV heads) of K and V
-    const int chunks_per_row = Hkv * kAttnD * 2 / 16;
-    auto load_stage = [&](int step, int buf) {
-        uint8_t* sk = smem + buf * STAGE;
-        uint8_t* sv = sk + KS * RB;
-        const int p0 = p_begin + step * KS;
-        for (int c = threadIdx.x; c < KS * chunks_per_row; c += nthreads) {
-            const int key = c / chunks_per_row, ch = c % chunks_per_row;
-            const int p = p0 + key;
-            int s = (p < p_end) ? sidx[p - p_begin - win_off] : -1;
-            bool ok = s >= 0 && s < P.n_keys;
-            if (ch == 0) svalid[buf * 128 + key] = ok ? 1 : 0;
-            const long long off = (ok ? (long long)s : 0) * (Hkv * kAttnD) + ch * 8;
-            cp_async_16(sk + key * RB + ch * 16, kb + off, ok);
-            cp_async_16(sv + key * RB + ch * 16, vb + off, ok);
-        }
-    };
-
     float o[NT][8][4];  // O^T: [d-tile][4] per n-tile; rows = head dims, cols = heads
+    float m_run[NT][2], l_run[NT][2];  // per owned head (cols 2*(lane%4)+{0,1})
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
+    for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
         for (int dt = 0; dt < 8; ++dt)
 #pragma unroll
             for (int i = 0; i < 4; ++i) o[nt][dt][i] = 0.f;
-    float m_run[NT][2], l_run[NT][2];  // per owned head (cols 2*(lane%4)+{0,1})
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) m_run[nt][0] = m_run[nt][1] = -INFINITY, l_run[nt][0] = l_run[nt][1] = 0.f;
-
-#pragma unroll
-    for (int s = 0; s < kAttnStages - 1; ++s) {
-        if (s < nsteps) load_stage(s, s);
-        cp_async_commit();
+        m_run[nt][0] = m_run[nt][1] = -INFINITY, l_run[nt][0] = l_run[nt][1] = 0.f;
     }
 
-    const int tiles_per_warp = KS / 16 / kAttnWPG;  // 16-key tiles this warp takes per stage
-    for (int step = 0; step < nsteps; ++step) {
-        cp_async_wait<kAttnStages - 2>();
-        __syncthreads();
-        const int ls = step + kAttnStages - 1;
-        if (ls < nsteps) {
-            if (ls * KS >= win_off + kAttnIdxWin) {  // uniform: next window of the index list
-                win_off += kAttnIdxWin;
-                fill_window();
-                __syncthreads();
+    if (warp == kAttnCW) {
+        // ------------------------------------------------------------ producer warp
+        // Lane l holds the index of slot p_begin + 32 c + l for the current chunk c of two
+        // stages; the next chunk's indices are loaded one chunk ahead.
+        const int rowb = Hkv * kAttnD * 2;
+        const int key = lane & 15;
+        const bool is_v = lane >= 16;
+        auto ld_idx = [&](int c) {
+            const int p = p_begin + 32 * c + lane;
+            return p < p_end ? __ldg(idx_row + p) : -1;
+        };
+        int cur = ld_idx(0), nxt = ld_idx(1);
+        int issued = 0;
+        bool ok = true;
+        for (int step = 0; step < nsteps; ++step) {
+            const int buf = step % NS;
+            // every lane waits (and so acquires); the warp leaves together if any lane gave up
+            ok = __all_sync(0xffffffffu, wait_parity(&empty[buf], ((step / NS) & 1) ^ 1, 0x401, abort_flag));
+            if (!ok) break;
+            const int s = __shfl_sync(0xffffffffu, cur, (step & 1) * 16 + key);
+            const int p = p_begin + step * kAttnKS + key;
+            const bool kv_ok = p < p_end && s >= 0 && s < P.n_keys;
+            if (!is_v) svalid[buf * kAttnKS + key] = kv_ok ? 1 : 0;
+            __syncwarp();
+            if (lane == 0) mbar_arrive_expect_tx(&full[buf], 2 * kAttnKS * rowb);
+            __syncwarp();
+            const __nv_bfloat16* src = (is_v ? vb : kb) + (long long)(kv_ok ? s : 0) * (Hkv * kAttnD);
+            uint8_t* dst = smem + buf * STAGE + (is_v ? kAttnKS * RB : 0) + key * RB;
+            bulk_load(dst, kv_ok ? static_cast<const void*>(src) : static_cast<const void*>(g_attn_zero_row), rowb,
+                      &full[buf]);
+            issued = step + 1;
+            if (step & 1) {
+                cur = nxt;
+                nxt = ld_idx((step >> 1) + 2);
             }
-            load_stage(ls, ls % kAttnStages);
         }
-        cp_async_commit();
+        if (!ok) {
+            // let the copies already issued land before the CTA leaves (bounded waits)
+            for (int b = 0; b < NS && b < issued; ++b) {
+                const int last = issued - 1 - ((issued - 1 - b) % NS);
+                wait_parity(&full[b], (last / NS) & 1, 0x402, nullptr);
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ consumer warps
+        // ---- Q^T fragments (B operand, K = head dim, N = 8 heads): head lane/4, dims 2*(lane%4)+{0,1}(+8)
+        uint32_t qf[NT][8][2];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            const int hl = nt * 8 + (lane >> 2);
+            const bool hv = hl < G;
+            const __nv_bfloat16* qrow = P.q + ((long long)t * P.Hq + grp * G + (hv ? hl : 0)) * kAttnD;
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                const int d = kk * 16 + 2 * (lane & 3);
+                qf[nt][kk][0] = hv ? *reinterpret_cast<const uint32_t*>(qrow + d) : 0u;
+                qf[nt][kk][1] = hv ? *reinterpret_cast<const uint32_t*>(qrow + d + 8) : 0u;
+            }
+        }
 
-        const uint8_t* sk = smem + (step % kAttnStages) * STAGE;
-        const uint8_t* sv = sk + KS * RB;
-        for (int tt = 0; tt < tiles_per_warp; ++tt) {
-            const int kt = wsub * tiles_per_warp + tt;       // 16-key tile inside the stage
-            const int pbase = p_begin + step * KS + kt * 16;  // index-list slot of its first key
+        for (int step = wsub; step < nsteps; step += WPG) {
+            const int buf = step % NS;
+            if (!__all_sync(0xffffffffu, wait_parity(&full[buf], (step / NS) & 1, 0x403, abort_flag))) break;
+            const uint8_t* sk = smem + buf * STAGE;
+            const uint8_t* sv = sk + kAttnKS * RB;
             // S^T = K Q^T : 16 keys x 8 heads per n-tile
             float sacc[NT][4];
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) sacc[nt][0] = sacc[nt][1] = sacc[nt][2] = sacc[nt][3] = 0.f;
             {
                 const int mi = lane >> 3, ri = lane & 7;
-                const uint8_t* arow = sk + (kt * 16 + (mi & 1) * 8 + ri) * RB + (grp * kAttnD + (mi >> 1) * 8) * 2;
+                const uint8_t* arow = sk + ((mi & 1) * 8 + ri) * RB + (grp * kAttnD + (mi >> 1) * 8) * 2;
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     uint32_t a[4];
@@ -190,11 +215,10 @@ __global__ void __launch_bounds__(256) sparse_attn_kernel(const AttnParams P) {
                     for (int nt = 0; nt < NT; ++nt) mma_16816(sacc[nt], a, qf[nt][kk][0], qf[nt][kk][1]);
                 }
             }
-            // mask slots beyond this CTA's range; rows: key lane/4 (c0,c1) and lane/4+8 (c2,c3)
-            // masked: slots past this CTA's range and entries that name no key (e.g. -1 padding)
-            const uint8_t* vrow = svalid + (step % kAttnStages) * 128 + kt * 16;
-            const bool v0 = pbase + (lane >> 2) < p_end && vrow[lane >> 2];
-            const bool v1 = pbase + (lane >> 2) + 8 < p_end && vrow[(lane >> 2) + 8];
+            // masked: slots past this CTA's range and entries that name no key (e.g. -1 padding);
+            // rows: key lane/4 (c0,c1) and lane/4+8 (c2,c3)
+            const bool v0 = svalid[buf * kAttnKS + (lane >> 2)] != 0;
+            const bool v1 = svalid[buf * kAttnKS + (lane >> 2) + 8] != 0;
             uint32_t pb[NT][2];
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
@@ -236,7 +260,7 @@ __global__ void __launch_bounds__(256) sparse_attn_kernel(const AttnParams P) {
             // O^T += V^T P^T : A = V^T (16 dims x 16 keys) via transposing ldmatrix
             {
                 const int mi = lane >> 3, ri = lane & 7;
-                const uint8_t* vrow = sv + (kt * 16 + (mi >> 1) * 8 + ri) * RB + (grp * kAttnD + (mi & 1) * 8) * 2;
+                const uint8_t* vrow = sv + ((mi >> 1) * 8 + ri) * RB + (grp * kAttnD + (mi & 1) * 8) * 2;
 #pragma unroll
                 for (int dt = 0; dt < 8; ++dt) {
                     uint32_t a[4];
@@ -245,11 +269,12 @@ __global__ void __launch_bounds__(256) sparse_attn_kernel(const AttnParams P) {
                     for (int nt = 0; nt < NT; ++nt) mma_16816(o[nt][dt], a, pb[nt][0], pb[nt][1]);
                 }
             }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[buf]);
         }
     }
-    cp_async_wait<0>();
 
-    // ---- finish: full row sums, merge the kAttnWPG warps of a group through shared memory
+    // ---- finish: full row sums, merge the WPG consumer warps of a group through shared memory
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
@@ -260,10 +285,10 @@ __global__ void __launch_bounds__(256) sparse_attn_kernel(const AttnParams P) {
             l += __shfl_xor_sync(0xffffffffu, l, 16);
             l_run[nt][j] = l;
         }
-    __syncthreads();  // stage buffers are free now
+    __syncthreads();  // every issued copy was consumed (or waited for): the ring is free now
     // per warp: [NT][8][4] O values per lane + m, l per owned head
     float* xch = reinterpret_cast<float*>(smem) + (size_t)warp * (NT * 36 * 32);
-    if (wsub != 0) {
+    if (warp < kAttnCW && wsub != 0) {
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
@@ -277,9 +302,9 @@ __global__ void __launch_bounds__(256) sparse_attn_kernel(const AttnParams P) {
         }
     }
     __syncthreads();
-    if (wsub == 0) {
-#pragma unroll
-        for (int w2 = 1; w2 < kAttnWPG; ++w2) {
+    if (warp < kAttnCW && wsub == 0) {
+#pragma unroll 1
+        for (int w2 = 1; w2 < WPG; ++w2) {
             const float* x2 = reinterpret_cast<const float*>(smem) + (size_t)(warp + w2) * (NT * 36 * 32);
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {

@@ -262,17 +262,17 @@ dsa_status run_topk(const float* scores, int64_t ld, int rows, int64_t q_pos0, c
 // ------------------------------------------------------------------ attention launch
 template <int NT>
 dsa_status launch_attn_t(const AttnParams& P, cudaStream_t s) {
-    const int smem = attn_smem_bytes(P.Hkv);
+    const int smem = attn_smem_bytes(P.Hkv, NT);
     auto kern = sparse_attn_kernel<NT>;
-    static int attr_bytes = 0;
-    if (attr_bytes < smem) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, attn_smem_bytes(1)) !=
-            cudaSuccess)
+    static bool attr_set = false;
+    if (!attr_set) {
+        const int most = std::max(attn_smem_bytes(1, NT), std::max(attn_smem_bytes(2, NT), attn_smem_bytes(4, NT)));
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, most) != cudaSuccess)
             return DSA_ERR_CUDA;
-        attr_bytes = attn_smem_bytes(1);
+        attr_set = true;
     }
     LaunchScope ls(K_ATTN, s);
-    kern<<<P.T * P.nsplit, P.Hkv * kAttnWPG * 32, smem, s>>>(P);
+    kern<<<P.T * P.nsplit, kAttnThreads, smem, s>>>(P);
     return launch_status();
 }
 

@@ -106,6 +106,18 @@ __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
     return d;
 }
 
+// ReLU is split across two pipes.  Heads h with (h & 2) == 0 take max(x, 0) on the integer/ALU
+// pipe; heads with (h & 2) != 0 take x + |x| = 2 max(x, 0) on the floating-point pipe, and their
+// weights are stored halved (exact: a power-of-two scale), so w * max(x, 0) is reproduced to the
+// bit for every finite x.  One pipe alone would issue one ReLU per MMA output element and cap
+// the epilogue at the tensor-core rate.
+__device__ __forceinline__ float2 relu_pair_alu(float a, float b) { return make_float2(fmaxf(a, 0.f), fmaxf(b, 0.f)); }
+__device__ __forceinline__ float2 relu2_pair_fma(float a, float b) { return make_float2(a + fabsf(a), b + fabsf(b)); }
+// Scale that the stored weight of head h carries (see above); heads come in groups of four only
+// when the head count is a multiple of four.
+template <int HI>
+__device__ __forceinline__ float weight_store_scale(int h) { return (HI % 4 == 0 && (h & 2)) ? 0.5f : 1.f; }
+
 // sum_h w[h] * max(v[h], 0) over N >= 1 heads, with independent partial sums (no long
 // dependent FMA chain) on packed fp32 pairs.
 template <int N>
@@ -123,8 +135,8 @@ __device__ __forceinline__ float head_sum(const float* v, const float* w) {
 #pragma unroll
             for (int q = 0; q < N / 4; ++q) {
                 const float4 w4 = *reinterpret_cast<const float4*>(w + 4 * q);
-                const float2 x0 = make_float2(fmaxf(v[4 * q], 0.f), fmaxf(v[4 * q + 1], 0.f));
-                const float2 x1 = make_float2(fmaxf(v[4 * q + 2], 0.f), fmaxf(v[4 * q + 3], 0.f));
+                const float2 x0 = relu_pair_alu(v[4 * q], v[4 * q + 1]);
+                const float2 x1 = relu2_pair_fma(v[4 * q + 2], v[4 * q + 3]);
                 acc[(2 * q) % NA] = ffma2(x0, make_float2(w4.x, w4.y), acc[(2 * q) % NA]);
                 acc[(2 * q + 1) % NA] = ffma2(x1, make_float2(w4.z, w4.w), acc[(2 * q + 1) % NA]);
             }
@@ -149,8 +161,8 @@ __device__ __forceinline__ void head_sum_acc(const float* v, const float* w, flo
 #pragma unroll
     for (int q = 0; q < N / 4; ++q) {
         const float4 w4 = *reinterpret_cast<const float4*>(w + 4 * q);
-        const float2 x0 = make_float2(fmaxf(v[4 * q], 0.f), fmaxf(v[4 * q + 1], 0.f));
-        const float2 x1 = make_float2(fmaxf(v[4 * q + 2], 0.f), fmaxf(v[4 * q + 3], 0.f));
+        const float2 x0 = relu_pair_alu(v[4 * q], v[4 * q + 1]);
+        const float2 x1 = relu2_pair_fma(v[4 * q + 2], v[4 * q + 3]);
         carry[(2 * q) % 4] = ffma2(x0, make_float2(w4.x, w4.y), carry[(2 * q) % 4]);
         carry[(2 * q + 1) % 4] = ffma2(x1, make_float2(w4.z, w4.w), carry[(2 * q + 1) % 4]);
     }
@@ -319,7 +331,8 @@ __global__ void __launch_bounds__(IndexerCfg<HI, BN, STAGES>::THREADS, 1)
                 const int tok = c / HI;
                 float wv = 0.f;
                 if (tok < U.rows)
-                    wv = __bfloat162float(P.w[((long long)U.p * P.Lq + (long long)U.qb * C::TB + tok) * HI + (c % HI)]);
+                    wv = __bfloat162float(P.w[((long long)U.p * P.Lq + (long long)U.qb * C::TB + tok) * HI + (c % HI)]) *
+                         weight_store_scale<HI>(c % HI);
                 w_s[cc] = wv;
             }
             __syncwarp();

@@ -197,34 +197,55 @@ __device__ __forceinline__ uint32_t stream_collect(TopkSmem& S, const float4* ro
                                                    int n, float F0, int region_base) {
     const int g_first = g_lo;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const uint32_t lanes_below = (1u << lane) - 1u;
     // float4 offset inside a 128-float4 round: piece (lane/8)*4 + warp, float4 lane%8 of it
     const int lane_off = (lane >> 3) * 32 + warp * 8 + (lane & 7);
+    // float4 groups whose four keys all lie in [e_lo, n): [g_in_lo, g_in_hi)
+    const int g_in_lo = max(g_first, (e_lo + 3) >> 2), g_in_hi = min(g_hi, n >> 2);
     uint32_t cnt = 0;
     // pieces are numbered from the start of the row: start at a multiple of 4 pieces (32 float4)
     // so that warp w takes exactly the pieces p with p % 4 == w (keys below g_lo are masked)
     g_lo &= ~31;
     constexpr int kStep = kTkUnroll * 128;  // float4 per iteration
     for (int g0 = g_lo; g0 < g_hi; g0 += kStep) {
+        // warp-uniform: every float4 of this iteration is in range, so only the score is tested
+        const bool interior = g0 >= g_in_lo && g0 + kStep <= g_in_hi;
         float4 v[kTkUnroll];
 #pragma unroll
         for (int u = 0; u < kTkUnroll; ++u) {
             const int g = g0 + u * 128 + lane_off;
-            v[u] = g < g_hi ? __ldcs(row4 + g) : make_float4(0.f, 0.f, 0.f, 0.f);
+            v[u] = (interior || g < g_hi) ? __ldcs(row4 + g) : make_float4(0.f, 0.f, 0.f, 0.f);
         }
 #pragma unroll
         for (int u = 0; u < kTkUnroll; ++u) {
             const int g = g0 + u * 128 + lane_off;
             const float f[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
             uint32_t mask = 0;
-            if (g < g_hi) {
+            if (interior) {
+#pragma unroll
+                for (int j = 0; j < 4; ++j) mask |= (f[j] >= F0 ? 1u : 0u) << j;
+            } else if (g < g_hi) {
 #pragma unroll
                 for (int j = 0; j < 4; ++j)
                     if (f[j] >= F0 && g * 4 + j < n && g * 4 + j >= e_lo && g >= g_first) mask |= 1u << j;
             }
+            // compaction in (lane, j) order = index order: the exclusive prefix of the per-lane
+            // counts from ballots (one ballot when no lane has more than one candidate)
             const uint32_t c = __popc(mask);
-            const uint32_t incl = warp_incl_scan(c);
+            const uint32_t any = __ballot_sync(0xffffffffu, c != 0);
+            if (any == 0) continue;
+            uint32_t excl, tot;
+            if (__ballot_sync(0xffffffffu, c > 1) == 0) {
+                excl = __popc(any & lanes_below);
+                tot = __popc(any);
+            } else {
+                const uint32_t b0 = __ballot_sync(0xffffffffu, c & 1u), b1 = __ballot_sync(0xffffffffu, c & 2u),
+                               b2 = __ballot_sync(0xffffffffu, c & 4u);
+                excl = __popc(b0 & lanes_below) + 2 * __popc(b1 & lanes_below) + 4 * __popc(b2 & lanes_below);
+                tot = __popc(b0) + 2 * __popc(b1) + 4 * __popc(b2);
+            }
             if (mask) {
-                uint32_t pos = cnt + incl - c;
+                uint32_t pos = cnt + excl;
 #pragma unroll
                 for (int j = 0; j < 4; ++j)
                     if (mask & (1u << j)) {
@@ -235,7 +256,7 @@ __device__ __forceinline__ uint32_t stream_collect(TopkSmem& S, const float4* ro
                         ++pos;
                     }
             }
-            cnt += __shfl_sync(0xffffffffu, incl, 31);
+            cnt += tot;
         }
     }
     return cnt;

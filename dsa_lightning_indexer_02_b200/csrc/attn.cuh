@@ -8,14 +8,19 @@
 // The work is a gather: per token, 2048 keys x Hkv x 128 x (K and V) x 2 bytes = 4 MiB at the
 // 32/4/128 shape against 32 x 128 x 2048 x 4 flop, i.e. 8 flop per byte, far below the ridge
 // of the tensor cores.  The kernel therefore spends its effort on the memory side:
-//   - one CTA per (token, key split), two CTAs per SM for up to 8 heads per KV group; each selected key's K and V rows for
-//     all KV heads are one contiguous Hkv*256-byte span, and a producer warp moves each of them
-//     with one bulk copy (the copy engine, not the load/store units, tracks the bytes in
-//     flight) into a ring of 16-key stages; an mbarrier per stage counts the bytes in, another
-//     counts the consumer warps out (rows padded by 16 bytes: conflict-free ldmatrix);
-//   - 8/Hkv consumer warps per KV group, taking the group's stages in turn; a warp owns its
-//     group's G query heads (GQA head packing: the K/V tile it reads from shared memory
-//     serves all G heads at once);
+//   - one CTA per (token, key split), two CTAs per SM for up to 8 heads per KV group; each
+//     selected key's K and V rows for all KV heads are one contiguous Hkv*256-byte span, moved
+//     with one bulk copy into a ring of 3 stages of 64/Hkv keys (rows padded by 16 bytes:
+//     conflict-free ldmatrix).  The copies are issued by 3 producer warps, warp i owning ring
+//     slot i: the rate at which one warp issues bulk copies, not the memory system, bounds a
+//     single producer, so each SM runs six;
+//   - an mbarrier per slot counts the bytes in, another the 4 consumer warps out.  Every waiter
+//     waits for every phase of the barriers it uses (the consumers for every stage, producer i
+//     for every refill of slot i): copies land out of order, and a parity wait that skipped a
+//     phase could mistake an older completion for the one it wants;
+//   - consumer warp w takes 16-key tile w % (4/Hkv) of every stage for KV group w / (4/Hkv) and
+//     owns the group's G query heads (GQA head packing: the K/V tile it reads from shared
+//     memory serves all G heads at once);
 //   - S^T[keys x heads] = K . Q^T and O^T += V^T . P^T on warp-level bf16 MMAs
 //     (m16n8k16, keys or head-dimension rows as M, 8 heads as N), so no MMA lane is wasted on
 //     the small head count; P^T goes from the accumulator layout to the operand layout with
@@ -31,11 +36,10 @@
 namespace dsa {
 
 constexpr int kAttnD = 128;
-constexpr int kAttnKS = 16;             // keys per stage
-constexpr int kAttnCW = 8;              // consumer warps (Hkv groups x 8/Hkv warps)
-constexpr int kAttnThreads = (kAttnCW + 1) * 32;
-constexpr int kAttnMaxStages = 16;
-constexpr int kAttnStageBudget = 100 * 1024;  // ring bytes per CTA: two CTAs per SM
+constexpr int kAttnCW = 4;              // consumer warps, one 16-key tile of every stage each
+constexpr int kAttnNS = 3;              // ring slots = producer warps
+constexpr int kAttnThreads = (kAttnCW + kAttnNS) * 32;
+constexpr int kAttnMaxKS = 64;          // keys per stage at Hkv = 1
 
 // Rows of zeros that stand in for slots naming no key (Hkv * 256 bytes at most).
 __device__ __align__(128) uint8_t g_attn_zero_row[4 * kAttnD * 2];
@@ -60,21 +64,17 @@ struct AttnParams {
     long long window;         // > 0 (prefill): a row holds at most min(topk, window) keys
 };
 
+__host__ __device__ constexpr int attn_stage_keys(int hkv) { return 16 * (kAttnCW / hkv); }
 __host__ __device__ constexpr int attn_row_bytes(int hkv) { return hkv * kAttnD * 2 + 16; }
-__host__ __device__ constexpr int attn_stage_bytes(int hkv) { return kAttnKS * attn_row_bytes(hkv) * 2; }
-__host__ __device__ constexpr int attn_stages(int hkv) {
-    return kAttnStageBudget / attn_stage_bytes(hkv) < kAttnMaxStages ? kAttnStageBudget / attn_stage_bytes(hkv)
-                                                                     : kAttnMaxStages;
-}
+__host__ __device__ constexpr int attn_stage_bytes(int hkv) { return attn_stage_keys(hkv) * attn_row_bytes(hkv) * 2; }
 // per consumer warp after the loop: [NT][36][32] floats (O fragments, m, l) for the merge
 __host__ __device__ constexpr int attn_xch_bytes(int nt) { return kAttnCW * nt * 36 * 32 * 4; }
 __host__ __device__ constexpr int attn_ring_bytes(int hkv, int nt) {
-    return attn_stages(hkv) * attn_stage_bytes(hkv) > attn_xch_bytes(nt) ? attn_stages(hkv) * attn_stage_bytes(hkv)
-                                                                         : attn_xch_bytes(nt);
+    return kAttnNS * attn_stage_bytes(hkv) > attn_xch_bytes(nt) ? kAttnNS * attn_stage_bytes(hkv) : attn_xch_bytes(nt);
 }
-// ring (or merge area) | full[NS], empty[NS] mbarriers | abort flag | valid flags [NS][16]
+// ring (or merge area) | full[NS], empty[NS] mbarriers | abort flag | valid flags [NS][64]
 __host__ __device__ constexpr int attn_smem_bytes(int hkv, int nt) {
-    return attn_ring_bytes(hkv, nt) + attn_stages(hkv) * 16 + 16 + attn_stages(hkv) * kAttnKS;
+    return attn_ring_bytes(hkv, nt) + kAttnNS * 16 + 16 + kAttnNS * kAttnMaxKS;
 }
 
 // NT: n-tiles of 8 query heads per KV group (G <= 8 * NT).
@@ -83,16 +83,16 @@ __global__ void __launch_bounds__(kAttnThreads, NT == 1 ? 2 : 1) sparse_attn_ker
     extern __shared__ __align__(1024) uint8_t smem[];
     const int Hkv = P.Hkv, G = P.Hq / P.Hkv;
     const int WPG = kAttnCW / Hkv;                  // consumer warps per KV group
+    const int KS = attn_stage_keys(Hkv);            // keys per stage
     const int RB = attn_row_bytes(Hkv);             // padded row bytes (K or V of one key)
     const int STAGE = attn_stage_bytes(Hkv);        // K rows then V rows
-    const int NS = attn_stages(Hkv);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int grp = warp / WPG, wsub = warp % WPG;  // consumer warps only
 
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + attn_ring_bytes(Hkv, NT));
-    uint64_t* empty = full + NS;
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + NS);
-    uint8_t* svalid = reinterpret_cast<uint8_t*>(empty + NS) + 16;
+    uint64_t* empty = full + kAttnNS;
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + kAttnNS);
+    uint8_t* svalid = reinterpret_cast<uint8_t*>(empty + kAttnNS) + 16;
 
     const int t = blockIdx.x / P.nsplit;
     const int split = blockIdx.x % P.nsplit;
@@ -112,12 +112,12 @@ __global__ void __launch_bounds__(kAttnThreads, NT == 1 ? 2 : 1) sparse_attn_ker
     const int p_begin = split * per_split;
     const int p_end = min(n_sel, p_begin + per_split);
     const int* idx_row = P.idx + (long long)t * P.topk;
-    const int nsteps = p_end > p_begin ? (p_end - p_begin + kAttnKS - 1) / kAttnKS : 0;
+    const int nsteps = p_end > p_begin ? (p_end - p_begin + KS - 1) / KS : 0;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < NS; ++i) {
+        for (int i = 0; i < kAttnNS; ++i) {
             mbar_init(&full[i], 1);
-            mbar_init(&empty[i], Hkv);
+            mbar_init(&empty[i], kAttnCW);
         }
         *abort_flag = 0;
         fence_mbar_init();
@@ -135,48 +135,58 @@ __global__ void __launch_bounds__(kAttnThreads, NT == 1 ? 2 : 1) sparse_attn_ker
         m_run[nt][0] = m_run[nt][1] = -INFINITY, l_run[nt][0] = l_run[nt][1] = 0.f;
     }
 
-    if (warp == kAttnCW) {
-        // ------------------------------------------------------------ producer warp
-        // Lane l holds the index of slot p_begin + 32 c + l for the current chunk c of two
-        // stages; the next chunk's indices are loaded one chunk ahead.
+    if (warp >= kAttnCW) {
+        // ------------------------------------------------------------ producer warp: ring slot `slot`
+        // Copy c of a stage (c < 2*KS: K rows, then V rows) goes to lane c % 32; the stage's
+        // indices are loaded one refill ahead.
+        const int slot = warp - kAttnCW;
         const int rowb = Hkv * kAttnD * 2;
-        const int key = lane & 15;
-        const bool is_v = lane >= 16;
-        auto ld_idx = [&](int c) {
-            const int p = p_begin + 32 * c + lane;
-            return p < p_end ? __ldg(idx_row + p) : -1;
+        const int ncp = (2 * KS) / 32;  // copies per lane: 1, 2 or 4
+        auto ld_idx = [&](int step, int i) {
+            const int key = (lane + 32 * i) % KS;
+            const int p = p_begin + step * KS + key;
+            return (step < nsteps && p < p_end) ? __ldg(idx_row + p) : -1;
         };
-        int cur = ld_idx(0), nxt = ld_idx(1);
-        int issued = 0;
+        int pre[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) pre[i] = i < ncp ? ld_idx(slot, i) : -1;
+        int fills = 0;
         bool ok = true;
-        for (int step = 0; step < nsteps; ++step) {
-            const int buf = step % NS;
+        for (int step = slot; step < nsteps; step += kAttnNS, ++fills) {
             // every lane waits (and so acquires); the warp leaves together if any lane gave up
-            ok = __all_sync(0xffffffffu, wait_parity(&empty[buf], ((step / NS) & 1) ^ 1, 0x401, abort_flag));
+            ok = __all_sync(0xffffffffu, wait_parity(&empty[slot], (fills & 1) ^ 1, 0x401, abort_flag));
             if (!ok) break;
-            const int s = __shfl_sync(0xffffffffu, cur, (step & 1) * 16 + key);
-            const int p = p_begin + step * kAttnKS + key;
-            const bool kv_ok = p < p_end && s >= 0 && s < P.n_keys;
-            if (!is_v) svalid[buf * kAttnKS + key] = kv_ok ? 1 : 0;
+            int cur[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                cur[i] = pre[i];
+                pre[i] = i < ncp ? ld_idx(step + kAttnNS, i) : -1;
+            }
+            bool kv_ok[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int c = lane + 32 * i, key = c % KS;
+                kv_ok[i] = i < ncp && p_begin + step * KS + key < p_end && cur[i] >= 0 && cur[i] < P.n_keys;
+                if (i < ncp && c < KS) svalid[slot * kAttnMaxKS + key] = kv_ok[i] ? 1 : 0;
+            }
             __syncwarp();
-            if (lane == 0) mbar_arrive_expect_tx(&full[buf], 2 * kAttnKS * rowb);
+            if (lane == 0) mbar_arrive_expect_tx(&full[slot], 2 * KS * rowb);
             __syncwarp();
-            const __nv_bfloat16* src = (is_v ? vb : kb) + (long long)(kv_ok ? s : 0) * (Hkv * kAttnD);
-            uint8_t* dst = smem + buf * STAGE + (is_v ? kAttnKS * RB : 0) + key * RB;
-            bulk_load(dst, kv_ok ? static_cast<const void*>(src) : static_cast<const void*>(g_attn_zero_row), rowb,
-                      &full[buf]);
-            issued = step + 1;
-            if (step & 1) {
-                cur = nxt;
-                nxt = ld_idx((step >> 1) + 2);
+            uint8_t* st = smem + slot * STAGE;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                if (i >= ncp) break;
+                const int c = lane + 32 * i, key = c % KS;
+                const bool is_v = c >= KS;
+                const __nv_bfloat16* src = (is_v ? vb : kb) + (long long)(kv_ok[i] ? cur[i] : 0) * (Hkv * kAttnD);
+                bulk_load(st + (is_v ? KS * RB : 0) + key * RB,
+                          kv_ok[i] ? static_cast<const void*>(src) : static_cast<const void*>(g_attn_zero_row), rowb,
+                          &full[slot]);
             }
         }
-        if (!ok) {
-            // let the copies already issued land before the CTA leaves (bounded waits)
-            for (int b = 0; b < NS && b < issued; ++b) {
-                const int last = issued - 1 - ((issued - 1 - b) % NS);
-                wait_parity(&full[b], (last / NS) & 1, 0x402, nullptr);
-            }
+        if (!ok && fills > 0) {
+            // let this slot's last copies land before the CTA leaves (bounded wait)
+            wait_parity(&full[slot], (fills - 1) & 1, 0x402, nullptr);
         }
     } else {
         // ------------------------------------------------------------ consumer warps
@@ -195,15 +205,17 @@ __global__ void __launch_bounds__(kAttnThreads, NT == 1 ? 2 : 1) sparse_attn_ker
             }
         }
 
-        for (int step = wsub; step < nsteps; step += WPG) {
-            const int buf = step % NS;
-            if (!__all_sync(0xffffffffu, wait_parity(&full[buf], (step / NS) & 1, 0x403, abort_flag))) break;
-            const uint8_t* sk = smem + buf * STAGE;
-            const uint8_t* sv = sk + kAttnKS * RB;
-            // S^T = K Q^T : 16 keys x 8 heads per n-tile
-            float sacc[NT][4];
+        for (int step = 0; step < nsteps; ++step) {
+            const int buf = step % kAttnNS;
+            if (!__all_sync(0xffffffffu, wait_parity(&full[buf], (step / kAttnNS) & 1, 0x403, abort_flag))) break;
+            const uint8_t* sk = smem + buf * STAGE + wsub * 16 * RB;  // this warp's 16-key tile
+            const uint8_t* sv = sk + KS * RB;
+            // S^T = K Q^T : 16 keys x 8 heads per n-tile, two independent accumulation chains
+            float sacc[NT][4], sacc2[NT][4];
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt) sacc[nt][0] = sacc[nt][1] = sacc[nt][2] = sacc[nt][3] = 0.f;
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) sacc[nt][i] = sacc2[nt][i] = 0.f;
             {
                 const int mi = lane >> 3, ri = lane & 7;
                 const uint8_t* arow = sk + ((mi & 1) * 8 + ri) * RB + (grp * kAttnD + (mi >> 1) * 8) * 2;
@@ -212,13 +224,21 @@ __global__ void __launch_bounds__(kAttnThreads, NT == 1 ? 2 : 1) sparse_attn_ker
                     uint32_t a[4];
                     ldmatrix_x4(a, arow + kk * 32);
 #pragma unroll
-                    for (int nt = 0; nt < NT; ++nt) mma_16816(sacc[nt], a, qf[nt][kk][0], qf[nt][kk][1]);
+                    for (int nt = 0; nt < NT; ++nt) {
+                        if (kk & 1) mma_16816(sacc2[nt], a, qf[nt][kk][0], qf[nt][kk][1]);
+                        else mma_16816(sacc[nt], a, qf[nt][kk][0], qf[nt][kk][1]);
+                    }
                 }
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) sacc[nt][i] += sacc2[nt][i];
             }
             // masked: slots past this CTA's range and entries that name no key (e.g. -1 padding);
             // rows: key lane/4 (c0,c1) and lane/4+8 (c2,c3)
-            const bool v0 = svalid[buf * kAttnKS + (lane >> 2)] != 0;
-            const bool v1 = svalid[buf * kAttnKS + (lane >> 2) + 8] != 0;
+            const uint8_t* vflag = svalid + buf * kAttnMaxKS + wsub * 16;
+            const bool v0 = vflag[lane >> 2] != 0;
+            const bool v1 = vflag[(lane >> 2) + 8] != 0;
             uint32_t pb[NT][2];
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {

@@ -335,9 +335,11 @@ __global__ void selftest_timeout_kernel(unsigned long long limit_ns) {
     }
 }
 
+// Key splits per sequence for the decode attention: enough CTAs for two per SM (the kernel's
+// residency), so every SM keeps two rings of K/V copies in flight.
 int decode_attn_splits(int B) {
     const int sms = std::max(1, num_sms());
-    return std::max(1, std::min(kMaxDecodeSplits, sms / std::max(1, B)));
+    return std::max(1, std::min(kMaxDecodeSplits, 2 * sms / std::max(1, B)));
 }
 
 struct DecodeWs {

@@ -169,24 +169,64 @@ __device__ __forceinline__ void clear_hist(TopkSmem& S, int nbins) {
     for (int b = threadIdx.x; b < nbins; b += kTkThreads) S.hist[b] = 0;
 }
 
-// T0 from m sample keys in S.cand_key[0, m): the key at rank rs, truncated to its top 20 bits
-// (two 10-bit rounds).  Every sample key >= T0 is counted, so at least rs samples are >= T0.
+// T0 from m sample keys in S.cand_key[0, m): a lower bound on the key at rank rs (counted from
+// the top), found with two histogram rounds of 1024 bins over the samples' own key range
+// [kmin, kmax] (key 0 marks a masked sample and counts with the lowest bin).  Round 1 bins
+// have width 2^sh1, the smallest power of two that covers the range; round 2 splits the bin
+// holding rank rs again into up to 1024 parts.  Every sample key >= T0 is counted, so at least
+// rs samples are >= T0.  Bins that follow the data (rather than fixed top bits of the key) keep
+// the shared-memory atomics spread out when the scores sit in a narrow range.
 __device__ __forceinline__ uint32_t sample_threshold(TopkSmem& S, int m, uint32_t rs) {
-    clear_hist(S, kTkBins);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+    for (int e = threadIdx.x; e < m; e += kTkThreads) {
+        const uint32_t key = S.cand_key[e];
+        if (key) {
+            kmin = min(kmin, key);
+            kmax = max(kmax, key);
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
+        kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
+    }
+    if (lane == 0) {
+        S.hist[warp] = kmin;
+        S.hist[kTkWarps + warp] = kmax;
+    }
     __syncthreads();
-    for (int e = threadIdx.x; e < m; e += kTkThreads) atomicAdd(&S.hist[S.cand_key[e] >> 22], 1u);
+#pragma unroll
+    for (int w = 0; w < kTkWarps; ++w) {
+        kmin = min(kmin, S.hist[w]);
+        kmax = max(kmax, S.hist[kTkWarps + w]);
+    }
     __syncthreads();
-    find_threshold_bin(S, kTkBins, rs);
-    const uint32_t b1 = S.sel_bin, need = rs - S.sel_gt;
+    if (kmin > kmax) kmin = kmax = 0u;  // every sample masked
+    const uint32_t span = kmax - kmin;
+    const int sh1 = (span >> 10) ? 32 - __clz(span >> 10) : 0;  // (span >> sh1) < 1024
     clear_hist(S, kTkBins);
     __syncthreads();
     for (int e = threadIdx.x; e < m; e += kTkThreads) {
         const uint32_t key = S.cand_key[e];
-        if ((key >> 22) == b1) atomicAdd(&S.hist[(key >> 12) & 0x3FF], 1u);
+        atomicAdd(&S.hist[(key > kmin ? key - kmin : 0u) >> sh1], 1u);
+    }
+    __syncthreads();
+    find_threshold_bin(S, kTkBins, rs);
+    const uint32_t b1 = S.sel_bin, need = rs - S.sel_gt;
+    if (sh1 == 0) return kmin + b1;  // bins of single key values: exact
+    const int sh2 = sh1 > 10 ? sh1 - 10 : 0;
+    const uint32_t base = b1 << sh1;
+    clear_hist(S, kTkBins);
+    __syncthreads();
+    for (int e = threadIdx.x; e < m; e += kTkThreads) {
+        const uint32_t key = S.cand_key[e];
+        const uint32_t d = key > kmin ? key - kmin : 0u;
+        if ((d >> sh1) == b1) atomicAdd(&S.hist[(d - base) >> sh2], 1u);
     }
     __syncthreads();
     find_threshold_bin(S, kTkBins, need);
-    return (b1 << 22) | (S.sel_bin << 12);
+    return kmin + base + (S.sel_bin << sh2);
 }
 
 // Stream float4 groups [g_lo, g_hi) of a row whose keys e_lo <= e < n compete and compact the

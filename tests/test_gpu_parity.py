@@ -362,6 +362,29 @@ def test_prefill_window_sampled_rows(cuda_ok, name, W):
     assert_output_ok(bf16_tensor_to_f64(out[torch.from_numpy(rows).cuda()]), own, f"window {W}")
 
 
+def test_sparse_attn_random_gather_beyond_l2(cuda_ok):
+    """K/V far larger than L2 (2 x 268 MB) and uniformly random indices: most row copies miss L2
+    and land out of order, the case in which a pipeline that confused barrier phases would read
+    a stage before its copies arrived (or stall)."""
+    g = torch.Generator().manual_seed(14)
+    Lk, T, Hq, Hkv, topk = 262144, 4096, 32, 4, 2048
+    q0 = Lk - T
+    tq = torch.randn((T, Hq, 128), generator=g).to(torch.bfloat16)
+    tk = torch.randn((Lk, Hkv, 128), generator=g).to(torch.bfloat16)
+    tv = torch.randn((Lk, Hkv, 128), generator=g).to(torch.bfloat16)
+    t_abs = torch.arange(q0, Lk, dtype=torch.int64)
+    idx = (torch.rand((T, topk), generator=g, dtype=torch.float64) * (t_abs[:, None] + 1).double()).long()
+    idx = idx.clamp_max(t_abs[:, None]).to(torch.int32)
+    out = torch.empty((T, Hq, 128), dtype=torch.bfloat16, device="cuda")
+    for _ in range(2):
+        dsa.dsa_sparse_attn(tq.cuda(), tk.cuda(), tv.cuda(), idx.cuda(), q0, 0.0883883, out)
+        assert dsa.sync_status() == dsa.DSA_OK
+    rows = np.linspace(0, T - 1, 48).astype(np.int64)
+    bits = [t.view(torch.int16).numpy().view(np.uint16) for t in (tq, tk, tv)]
+    want, _ = oracle.sparse_attn_rows(bits[0][rows], bits[1], bits[2], idx.numpy()[rows], 0.0883883)
+    assert_output_ok(bf16_tensor_to_f64(out)[rows], want, "random gather")
+
+
 def test_attention_skips_padding_entries_inside_the_count(cuda_ok):
     """Entries that name no key (-1, or >= Lk) are skipped wherever they sit in the list."""
     rng = np.random.default_rng(13)

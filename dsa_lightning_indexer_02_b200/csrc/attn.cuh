@@ -266,12 +266,15 @@ __global__ void __launch_bounds__(kAttnThreads, NT == 1 ? 2 : 1) sparse_attn_ker
                 const float p2 = exp2f(z[2] - base[0]), p3 = exp2f(z[3] - base[1]);
                 l_run[nt][0] = l_run[nt][0] * alpha[0] + p0 + p2;
                 l_run[nt][1] = l_run[nt][1] * alpha[1] + p1 + p3;
+                // rescale only when some running max moved (alpha == 1 leaves O unchanged)
+                if (__any_sync(0xffffffffu, alpha[0] != 1.f || alpha[1] != 1.f)) {
 #pragma unroll
-                for (int dt = 0; dt < 8; ++dt) {
-                    o[nt][dt][0] *= alpha[0];
-                    o[nt][dt][1] *= alpha[1];
-                    o[nt][dt][2] *= alpha[0];
-                    o[nt][dt][3] *= alpha[1];
+                    for (int dt = 0; dt < 8; ++dt) {
+                        o[nt][dt][0] *= alpha[0];
+                        o[nt][dt][1] *= alpha[1];
+                        o[nt][dt][2] *= alpha[0];
+                        o[nt][dt][3] *= alpha[1];
+                    }
                 }
                 // P^T (keys x heads) -> B operand layout (keys as K, heads as N)
                 pb[nt][0] = movmatrix_trans(pack_bf16x2(p0, p1));

@@ -178,6 +178,7 @@ __device__ __forceinline__ void clear_hist(TopkSmem& S, int nbins) {
 // the shared-memory atomics spread out when the scores sit in a narrow range.
 __device__ __forceinline__ uint32_t sample_threshold(TopkSmem& S, int m, uint32_t rs) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    __syncthreads();  // the samples were written by other threads
     uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
     for (int e = threadIdx.x; e < m; e += kTkThreads) {
         const uint32_t key = S.cand_key[e];
@@ -209,7 +210,7 @@ __device__ __forceinline__ uint32_t sample_threshold(TopkSmem& S, int m, uint32_
     __syncthreads();
     for (int e = threadIdx.x; e < m; e += kTkThreads) {
         const uint32_t key = S.cand_key[e];
-        atomicAdd(&S.hist[(key > kmin ? key - kmin : 0u) >> sh1], 1u);
+        atomicAdd(&S.hist[min((key > kmin ? key - kmin : 0u) >> sh1, (uint32_t)kTkBins - 1u)], 1u);
     }
     __syncthreads();
     find_threshold_bin(S, kTkBins, rs);
@@ -222,7 +223,7 @@ __device__ __forceinline__ uint32_t sample_threshold(TopkSmem& S, int m, uint32_
     for (int e = threadIdx.x; e < m; e += kTkThreads) {
         const uint32_t key = S.cand_key[e];
         const uint32_t d = key > kmin ? key - kmin : 0u;
-        if ((d >> sh1) == b1) atomicAdd(&S.hist[(d - base) >> sh2], 1u);
+        if (min(d >> sh1, (uint32_t)kTkBins - 1u) == b1) atomicAdd(&S.hist[min((d - base) >> sh2, (uint32_t)kTkBins - 1u)], 1u);
     }
     __syncthreads();
     find_threshold_bin(S, kTkBins, need);

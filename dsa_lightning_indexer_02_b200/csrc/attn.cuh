@@ -40,6 +40,7 @@ constexpr int kAttnCW = 4;              // consumer warps, one 16-key tile of ev
 constexpr int kAttnNS = 3;              // ring slots = producer warps
 constexpr int kAttnThreads = (kAttnCW + kAttnNS) * 32;
 constexpr int kAttnMaxKS = 64;          // keys per stage at Hkv = 1
+constexpr int kAttnPartStride = kAttnD + 4;  // floats per split partial: O[128], m, l, 2 pad (16-byte rows)
 
 // Rows of zeros that stand in for slots naming no key (Hkv * 256 bytes at most).
 __device__ __align__(128) uint8_t g_attn_zero_row[4 * kAttnD * 2];
@@ -60,7 +61,7 @@ struct AttnParams {
     __nv_bfloat16* out;       // [T, Hq, D]
     float* lse;               // [T, Hq] natural-log LSE, may be null
     int nsplit;               // key splits per token
-    float* part;              // nsplit > 1: [T, nsplit, Hq, D + 2]
+    float* part;              // nsplit > 1: [T, nsplit, Hq, kAttnPartStride]
     long long window;         // > 0 (prefill): a row holds at most min(topk, window) keys
 };
 
@@ -370,7 +371,7 @@ __global__ void __launch_bounds__(kAttnThreads, NT == 1 ? 2 : 1) sparse_attn_ker
                         P.lse[(long long)t * P.Hq + h] =
                             l_run[nt][j] > 0.f ? (m_run[nt][j] + log2f(l_run[nt][j])) * 0.69314718055994531f : -INFINITY;
                 } else {
-                    float* prow = P.part + (((long long)t * P.nsplit + split) * P.Hq + h) * (kAttnD + 2);
+                    float* prow = P.part + (((long long)t * P.nsplit + split) * P.Hq + h) * kAttnPartStride;
 #pragma unroll
                     for (int dt = 0; dt < 8; ++dt) {
                         prow[dt * 16 + (lane >> 2)] = o[nt][dt][j];
@@ -386,33 +387,53 @@ __global__ void __launch_bounds__(kAttnThreads, NT == 1 ? 2 : 1) sparse_attn_ker
     }
 }
 
-// Merge split partials: one warp per (token, head).  With advance_ctx (decode), block 0 also
-// moves every sequence's context length one position on (nothing later in the step reads it).
+// Merge split partials: one warp per (token, head).  Lane s < nsplit holds split s's running
+// max and sum; every lane then accumulates its 4 output dims over all splits with independent
+// 16-byte loads.  With advance_ctx (decode), block 0 also moves every sequence's context length
+// one position on (nothing later in the step reads it).
 __global__ void __launch_bounds__(128) attn_combine_kernel(const float* part, int T, int nsplit, int Hq,
                                                            __nv_bfloat16* out, float* lse, int* advance_ctx,
                                                            long long Lmax) {
+    constexpr int kMaxSplits = 32;
     const int wid = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
     if (advance_ctx && blockIdx.x == 0)
         for (int b = threadIdx.x; b < T; b += blockDim.x)
             if (advance_ctx[b] >= 0 && advance_ctx[b] < Lmax) advance_ctx[b] += 1;
-    if (wid >= T * Hq) return;
+    if (wid >= T * Hq || nsplit > kMaxSplits) return;
     const int t = wid / Hq, h = wid % Hq;
-    float mx = -INFINITY;
-    for (int s = 0; s < nsplit; ++s) mx = fmaxf(mx, part[(((long long)t * nsplit + s) * Hq + h) * (kAttnD + 2) + kAttnD]);
-    const float bs = mx == -INFINITY ? 0.f : mx;
-    float acc[4] = {0.f, 0.f, 0.f, 0.f}, l = 0.f;
-    for (int s = 0; s < nsplit; ++s) {
-        const float* pr = part + (((long long)t * nsplit + s) * Hq + h) * (kAttnD + 2);
-        const float a = exp2f(pr[kAttnD] - bs);
-        l += pr[kAttnD + 1] * a;
+    const long long sstride = (long long)Hq * kAttnPartStride;
+    const float* base = part + ((long long)t * nsplit * Hq + h) * kAttnPartStride;
+    float m_s = -INFINITY, l_s = 0.f;
+    if (lane < nsplit) {
+        const float2 ml = *reinterpret_cast<const float2*>(base + lane * sstride + kAttnD);
+        m_s = ml.x;
+        l_s = ml.y;
+    }
+    float mx = m_s;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) acc[i] += pr[lane * 4 + i] * a;
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    const float bs = mx == -INFINITY ? 0.f : mx;
+    const float a_s = lane < nsplit ? exp2f(m_s - bs) : 0.f;
+    float l = l_s * a_s;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int s = 0; s < kMaxSplits; ++s) {
+        const float w = __shfl_sync(0xffffffffu, a_s, s);
+        if (s < nsplit) {
+            const float4 v = *reinterpret_cast<const float4*>(base + s * sstride + lane * 4);
+            acc.x += v.x * w;
+            acc.y += v.y * w;
+            acc.z += v.z * w;
+            acc.w += v.w * w;
+        }
     }
     const float inv = l > 0.f ? 1.f / l : 0.f;
-    __nv_bfloat16* orow = out + ((long long)t * Hq + h) * kAttnD;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) orow[lane * 4 + i] = __float2bfloat16_rn(acc[i] * inv);
+    __nv_bfloat162* orow = reinterpret_cast<__nv_bfloat162*>(out + ((long long)t * Hq + h) * kAttnD + lane * 4);
+    orow[0] = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
+    orow[1] = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
     if (lse && lane == 0) lse[(long long)t * Hq + h] = l > 0.f ? (mx + log2f(l)) * 0.69314718055994531f : -INFINITY;
 }
 

@@ -24,6 +24,7 @@ namespace {
 constexpr int kVersion = 10000;
 constexpr int kMaxTopk = 65536;
 constexpr int kMaxDecodeSplits = 16;
+static_assert(kMaxDecodeSplits <= 32, "attn_combine_kernel holds one split per lane");
 constexpr int kDecodeIdxStages = 8;
 constexpr int kPrefillIdxStages = 4;
 
@@ -353,7 +354,7 @@ DecodeWs decode_ws_layout(int64_t Lmax, int B, int Hq, int topk, bool need_idx) 
     w.idx = off;
     if (need_idx) off = align_up(off + (size_t)B * topk * 4, 256);
     w.part = off;
-    off = align_up(off + (size_t)B * kMaxDecodeSplits * Hq * (kAttnD + 2) * 4, 256);
+    off = align_up(off + (size_t)B * kMaxDecodeSplits * Hq * kAttnPartStride * 4, 256);
     w.total = off;
     return w;
 }

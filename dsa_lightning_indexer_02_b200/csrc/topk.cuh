@@ -309,13 +309,22 @@ __device__ __forceinline__ uint32_t stream_collect(TopkSmem& S, const float4* ro
 // keys above that bin are all kept, and the bin's members are ranked by (key desc, index asc).
 // Returns false, writing nothing, when more than kTkBins candidates share the last bin.
 constexpr int kTkSmallBin = 64;
+constexpr int kTkBatch = 4;  // shared-memory loads batched per thread in the refinement passes
 
 __device__ __forceinline__ bool refine_and_emit(TopkSmem& S, uint32_t lo, int k, int* out) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int nreg = S.nreg;
+    // The passes below hoist each region's pointers and count into registers and batch their
+    // shared-memory loads (kTkBatch per thread ahead of the use), so that they overlap instead of
+    // each waiting for the one before (stores and atomics in the loops would otherwise make the
+    // compiler reload the bounds and serialise the loads).
     uint32_t mx = 0;
-    for (int r = 0; r < nreg; ++r)
-        for (int e = tid; e < S.reg_cnt[r]; e += kTkThreads) mx = max(mx, S.reg_kp[r][e] - lo);
+    for (int r = 0; r < nreg; ++r) {
+        const uint32_t* kp = S.reg_kp[r];
+        const int cnt = S.reg_cnt[r];
+#pragma unroll 4
+        for (int e = tid; e < cnt; e += kTkThreads) mx = max(mx, kp[e] - lo);
+    }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
     __syncthreads();
@@ -334,12 +343,23 @@ __device__ __forceinline__ bool refine_and_emit(TopkSmem& S, uint32_t lo, int k,
         __syncthreads();
         clear_hist(S, nbins);
         __syncthreads();
-        for (int r = 0; r < nreg; ++r)
-            for (int e = tid; e < S.reg_cnt[r]; e += kTkThreads) {
-                const uint32_t d = S.reg_kp[r][e] - lo;
-                const bool match = fixed >= 32 ? true : ((d >> fixed) == (pv >> fixed));
-                if (match) atomicAdd(&S.hist[(d >> sh) & (nbins - 1)], 1u);
+        for (int r = 0; r < nreg; ++r) {
+            const uint32_t* kp = S.reg_kp[r];
+            const int cnt = S.reg_cnt[r];
+            for (int e0 = tid; e0 < cnt; e0 += kTkBatch * kTkThreads) {
+                uint32_t d[kTkBatch];
+#pragma unroll
+                for (int j = 0; j < kTkBatch; ++j) {
+                    const int e = e0 + j * kTkThreads;
+                    d[j] = e < cnt ? kp[e] - lo : 0u;
+                }
+#pragma unroll
+                for (int j = 0; j < kTkBatch; ++j) {
+                    const bool match = fixed >= 32 ? true : ((d[j] >> fixed) == (pv >> fixed));
+                    if (e0 + j * kTkThreads < cnt && match) atomicAdd(&S.hist[(d[j] >> sh) & (nbins - 1)], 1u);
+                }
             }
+        }
         __syncthreads();
         find_threshold_bin(S, nbins, need);
         need -= S.sel_gt;
@@ -362,15 +382,27 @@ __device__ __forceinline__ bool refine_and_emit(TopkSmem& S, uint32_t lo, int k,
     auto loc_idx = [&](uint32_t l) { return S.reg_ip[l >> 16][l & 0xFFFFu]; };
     if (tid == 0) S.sel_bin = 0;
     __syncthreads();
-    for (int r = 0; r < nreg; ++r)
-        for (int e = tid; e < S.reg_cnt[r]; e += kTkThreads) {
-            const uint32_t key = S.reg_kp[r][e];
-            if (in_bin(key - lo)) {
-                const uint32_t p = atomicAdd(&S.sel_bin, 1u);
-                bkey[p] = key;
-                bloc[p] = ((uint32_t)r << 16) | (uint32_t)e;
+    for (int r = 0; r < nreg; ++r) {
+        const uint32_t* kp = S.reg_kp[r];
+        const int cnt = S.reg_cnt[r];
+        for (int e0 = tid; e0 < cnt; e0 += kTkBatch * kTkThreads) {
+            uint32_t key[kTkBatch];
+#pragma unroll
+            for (int j = 0; j < kTkBatch; ++j) {
+                const int e = e0 + j * kTkThreads;
+                key[j] = e < cnt ? kp[e] : 0u;
+            }
+#pragma unroll
+            for (int j = 0; j < kTkBatch; ++j) {
+                const int e = e0 + j * kTkThreads;
+                if (e < cnt && in_bin(key[j] - lo)) {
+                    const uint32_t p = atomicAdd(&S.sel_bin, 1u);
+                    bkey[p] = key[j];
+                    bloc[p] = ((uint32_t)r << 16) | (uint32_t)e;
+                }
             }
         }
+    }
     __syncthreads();
     bool drop[(kTkBins / 2 + kTkThreads - 1) / kTkThreads];
 #pragma unroll
@@ -402,7 +434,11 @@ __device__ __forceinline__ bool refine_and_emit(TopkSmem& S, uint32_t lo, int k,
     // write the kept keys region by region, each region in its own (ascending) order
     for (int r = warp; r < nreg; r += kTkWarps) {
         uint32_t c = 0;
-        for (int e = lane; e < S.reg_cnt[r]; e += 32) c += kept(S.reg_kp[r][e], S.reg_ip[r][e]);
+        const uint32_t* kp = S.reg_kp[r];
+        const int* ip = S.reg_ip[r];
+        const int cnt = S.reg_cnt[r];
+#pragma unroll 4
+        for (int e = lane; e < cnt; e += 32) c += kept(kp[e], ip[e]);
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
         if (lane == 0) S.reg_gt[r] = (int)c;
@@ -411,14 +447,25 @@ __device__ __forceinline__ bool refine_and_emit(TopkSmem& S, uint32_t lo, int k,
     for (int r = warp; r < nreg; r += kTkWarps) {
         uint32_t base = 0;
         for (int q = 0; q < r; ++q) base += (uint32_t)S.reg_gt[q];
-        for (int e0 = 0; e0 < S.reg_cnt[r]; e0 += 32) {
-            const int e = e0 + lane;
-            const bool in = e < S.reg_cnt[r];
-            const int ix = in ? S.reg_ip[r][e] : 0;
-            const bool keep = in && kept(S.reg_kp[r][e], ix);
-            const uint32_t bk = __ballot_sync(0xffffffffu, keep);
-            if (keep) out[base + __popc(bk & ((1u << lane) - 1u))] = ix;
-            base += __popc(bk);
+        const uint32_t* kp = S.reg_kp[r];
+        const int* ip = S.reg_ip[r];
+        const int cnt = S.reg_cnt[r];
+        for (int e0 = 0; e0 < cnt; e0 += 32 * kTkBatch) {
+            int ix[kTkBatch];
+            bool keep[kTkBatch];
+#pragma unroll
+            for (int j = 0; j < kTkBatch; ++j) {
+                const int e = e0 + 32 * j + lane;
+                const bool in = e < cnt;
+                ix[j] = in ? ip[e] : 0;
+                keep[j] = in && kept(in ? kp[e] : 0u, ix[j]);
+            }
+#pragma unroll
+            for (int j = 0; j < kTkBatch; ++j) {
+                const uint32_t bk = __ballot_sync(0xffffffffu, keep[j]);
+                if (keep[j]) out[base + __popc(bk & ((1u << lane) - 1u))] = ix[j];
+                base += __popc(bk);
+            }
         }
     }
     return true;
@@ -586,13 +633,13 @@ __global__ void __launch_bounds__(kTkThreads, 6) topk_kernel(const TopkParams P)
 // 1/kTkCluster of the row; the sample keys go to CTA 0, which sets the threshold, gathers every
 // CTA's candidate regions through distributed shared memory, then refines and writes the row.
 // Dynamic shared memory: sizeof(TopkSmem) + kTkCap * 8 bytes (CTA 0's gather buffer).
-__global__ void __launch_bounds__(kTkThreads) topk_cluster_kernel(const TopkParams P) {
+__global__ void __launch_bounds__(kTkThreads, 1) topk_cluster_kernel(const TopkParams P) {
     extern __shared__ __align__(1024) uint8_t topk_smem[];
     __shared__ int src_cnt[kTkMaxRegions];
     TopkSmem& S = *reinterpret_cast<TopkSmem*>(topk_smem);
     cg::cluster_group cluster = cg::this_cluster();
     const int crank = (int)cluster.block_rank();
-    const int r = blockIdx.x / kTkCluster, tid = threadIdx.x, warp = tid >> 5;
+    const int r = blockIdx.x / kTkCluster, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int n = (int)row_length(P, r, tid == 0 && crank == 0);
     const int lo = row_first_key(P, n), ne = n - lo;  // competing keys: [lo, n)
     const int k = P.k;
@@ -642,8 +689,8 @@ __global__ void __launch_bounds__(kTkThreads) topk_cluster_kernel(const TopkPara
             fits = fits && total >= (uint32_t)k && total <= (uint32_t)kTkCap;
             if (fits) {
                 // gather every CTA's regions into a local buffer, region-major (region w of CTA 0,
-                // of CTA 1, ...), in one flattened pass so the remote loads overlap; region w of
-                // the row then stays one ascending run, as in the one-CTA kernel
+                // of CTA 1, ...); region w of the row then stays one ascending run, as in the
+                // one-CTA kernel
                 uint32_t* gkey = reinterpret_cast<uint32_t*>(topk_smem + sizeof(TopkSmem));
                 int* gidx = reinterpret_cast<int*>(gkey + kTkCap);
                 __shared__ int src_pre[kTkMaxRegions + 1];
@@ -656,17 +703,36 @@ __global__ void __launch_bounds__(kTkThreads) topk_cluster_kernel(const TopkPara
                     src_pre[kTkMaxRegions] = acc;
                 }
                 __syncthreads();
-#pragma unroll 4
-                for (int f = tid; f < (int)total; f += kTkThreads) {
-                    int q = 0;  // last q with src_pre[q] <= f (binary search)
+                // warp w copies source regions q = w, w + 4, ...: consecutive lanes read
+                // consecutive entries of one remote region (coalesced), four per lane in flight
+                for (int q = warp; q < kTkMaxRegions; q += kTkWarps) {
+                    const int c = q % kTkCluster, w = q / kTkCluster;
+                    const int cnt = src_pre[q + 1] - src_pre[q], dst0 = src_pre[q];
+                    const TopkSmem* Src = cluster.map_shared_rank(&S, c);
+                    const uint32_t* sk = Src->cand_key + w * kTkRegion;
+                    const int* si = Src->cand_idx + w * kTkRegion;
+                    for (int e0 = 0; e0 < cnt; e0 += 32 * kTkBatch) {
+                        uint32_t kk[kTkBatch];
+                        int ii[kTkBatch];
 #pragma unroll
-                    for (int step = kTkMaxRegions / 2; step > 0; step >>= 1)
-                        if (q + step < kTkMaxRegions && src_pre[q + step] <= f) q += step;
-                    const int e = f - src_pre[q];
-                    const TopkSmem* Src = cluster.map_shared_rank(&S, q % kTkCluster);
-                    gkey[f] = Src->cand_key[(q / kTkCluster) * kTkRegion + e];
-                    gidx[f] = Src->cand_idx[(q / kTkCluster) * kTkRegion + e];
+                        for (int j = 0; j < kTkBatch; ++j) {
+                            const int e = e0 + 32 * j + lane;
+                            if (e < cnt) {
+                                kk[j] = sk[e];
+                                ii[j] = si[e];
+                            }
+                        }
+#pragma unroll
+                        for (int j = 0; j < kTkBatch; ++j) {
+                            const int e = e0 + 32 * j + lane;
+                            if (e < cnt) {
+                                gkey[dst0 + e] = kk[j];
+                                gidx[dst0 + e] = ii[j];
+                            }
+                        }
+                    }
                 }
+                __syncthreads();
                 if (tid < kTkWarps) {
                     S.reg_kp[tid] = gkey + src_pre[tid * kTkCluster];
                     S.reg_ip[tid] = gidx + src_pre[tid * kTkCluster];

@@ -62,6 +62,7 @@ struct AttnParams {
     float* lse;               // [T, Hq] natural-log LSE, may be null
     int nsplit;               // key splits per token
     float* part;              // nsplit > 1: [T, nsplit, Hq, kAttnPartStride]
+    int* advance_ctx;         // decode with nsplit == 1, may be null: ctx_len[t] += 1 once token t is done
     long long window;         // > 0 (prefill): a row holds at most min(topk, window) keys
 };
 
@@ -385,6 +386,10 @@ __global__ void __launch_bounds__(kAttnThreads, NT == 1 ? 2 : 1) sparse_attn_ker
             }
         }
     }
+    // decode with one CTA per token: advance its context length here (every thread read
+    // ctx_len[t] before the first barrier of the kernel); with splits the merge kernel does it
+    if (P.nsplit == 1 && P.advance_ctx && threadIdx.x == 0 && P.advance_ctx[t] >= 0 && P.advance_ctx[t] < P.n_keys)
+        P.advance_ctx[t] += 1;
 }
 
 // Merge split partials: one warp per (token, head).  Lane s < nsplit holds split s's running

@@ -158,7 +158,7 @@ dsa_status launch_indexer_t(const CUtensorMap& mq, const CUtensorMap& mk, const 
 // Shared by dsa_index (P = 1) and the decode step (P = B, one query each).
 dsa_status run_indexer(const void* qI, const void* kI, const __nv_bfloat16* w, int P_, int Lq, int64_t q_pos0,
                        const int* ctx_len, int64_t Lk, int HI, float* scores, int64_t ld, cudaStream_t s,
-                       int64_t window = 0) {
+                       int64_t window = 0, const IndexerParams* append = nullptr) {
     const bool decode = ctx_len != nullptr;
     const int BN = decode ? HI : 256;
     const int TB = BN / HI;
@@ -173,6 +173,16 @@ dsa_status run_indexer(const void* qI, const void* kI, const __nv_bfloat16* w, i
     P.ld = ld;
     P.num_qb = (Lq + TB - 1) / TB;
     P.window = decode ? 0 : window;
+    if (append) {
+        P.new_k = append->new_k;
+        P.new_v = append->new_v;
+        P.new_kI = append->new_kI;
+        P.cache_k = append->cache_k;
+        P.cache_v = append->cache_v;
+        P.cache_kI = append->cache_kI;
+        P.kv16 = append->kv16;
+        P.kI16 = append->kI16;
+    }
     const int sms = num_sms();
     if (sms <= 0) return DSA_ERR_CUDA;
     const int64_t ktiles = (Lk + kIdxBM - 1) / kIdxBM;
@@ -284,38 +294,9 @@ dsa_status run_attn(const AttnParams& P, cudaStream_t s) {
 }
 
 // ------------------------------------------------------------------ decode helpers
-__global__ void decode_append_kernel(const __nv_bfloat16* k_new, const __nv_bfloat16* v_new,
-                                     const __nv_bfloat16* kI_new, __nv_bfloat16* k_cache, __nv_bfloat16* v_cache,
-                                     __nv_bfloat16* kI_cache, const int* ctx_len, long long Lmax, int kv_elems,
-                                     int dI) {
-    const int b = blockIdx.x;
-    const long long pos = ctx_len[b];
-    if (pos < 0 || pos >= Lmax) {
-        if (threadIdx.x == 0) record_error(DSA_DEV_ERR_BOUNDS, 0x501);
-        return;
-    }
-    const int kv16 = kv_elems / 8, kI16 = dI / 8;  // 16-byte vectors
-    const uint4* ks = reinterpret_cast<const uint4*>(k_new + (long long)b * kv_elems);
-    const uint4* vs = reinterpret_cast<const uint4*>(v_new + (long long)b * kv_elems);
-    uint4* kd = reinterpret_cast<uint4*>(k_cache + ((long long)b * Lmax + pos) * kv_elems);
-    uint4* vd = reinterpret_cast<uint4*>(v_cache + ((long long)b * Lmax + pos) * kv_elems);
-    for (int i = threadIdx.x; i < kv16; i += blockDim.x) {
-        kd[i] = ks[i];
-        vd[i] = vs[i];
-    }
-    const uint4* is = reinterpret_cast<const uint4*>(kI_new + (long long)b * dI);
-    uint4* id = reinterpret_cast<uint4*>(kI_cache + ((long long)b * Lmax + pos) * dI);
-    for (int i = threadIdx.x; i < kI16; i += blockDim.x) id[i] = is[i];
-}
-
-__global__ void decode_advance_kernel(int* ctx_len, int B, long long Lmax) {
-    const int b = blockIdx.x * blockDim.x + threadIdx.x;
-    if (b < B && ctx_len[b] >= 0 && ctx_len[b] < Lmax) ctx_len[b] += 1;
-}
-
 // Sequences whose ctx_len is out of range must not be read past the caches by the other kernels;
 // the indexer, top-k and attention kernels clamp their key counts to the cache capacity, and the
-// append kernel reports the bad input.
+// indexer (which appends the new token) reports the bad input.
 
 __global__ void selftest_timeout_kernel(unsigned long long limit_ns) {
     __shared__ uint64_t bar;
@@ -587,15 +568,18 @@ dsa_status dsa_decode(const void* q, const void* qI, const void* w, const void* 
     int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(wsb + L.idx);
     float* part = reinterpret_cast<float*>(wsb + L.part);
     const int64_t ld = (int64_t)align_up((size_t)Lmax, 4);
-    {
-        LaunchScope ls(K_APPEND, s);
-        decode_append_kernel<<<B, 128, 0, s>>>(
-            static_cast<const __nv_bfloat16*>(k_new), static_cast<const __nv_bfloat16*>(v_new),
-            static_cast<const __nv_bfloat16*>(kI_new), static_cast<__nv_bfloat16*>(k_cache),
-            static_cast<__nv_bfloat16*>(v_cache), static_cast<__nv_bfloat16*>(kI_cache), ctx_len, Lmax, Hkv * D, dI);
-        if ((st = launch_status()) != DSA_OK) return st;
-    }
-    st = run_indexer(qI, kI_cache, static_cast<const __nv_bfloat16*>(w), B, 1, 0, ctx_len, Lmax, HI, scores, ld, s);
+    // the indexer appends the new tokens' K, V and kI rows to the caches (ahead of its own loads)
+    IndexerParams app{};
+    app.new_k = static_cast<const uint4*>(k_new);
+    app.new_v = static_cast<const uint4*>(v_new);
+    app.new_kI = static_cast<const uint4*>(kI_new);
+    app.cache_k = static_cast<uint4*>(k_cache);
+    app.cache_v = static_cast<uint4*>(v_cache);
+    app.cache_kI = static_cast<uint4*>(kI_cache);
+    app.kv16 = Hkv * D / 8;
+    app.kI16 = dI / 8;
+    st = run_indexer(qI, kI_cache, static_cast<const __nv_bfloat16*>(w), B, 1, 0, ctx_len, Lmax, HI, scores, ld, s,
+                     0, &app);
     if (st != DSA_OK) return st;
     st = run_topk(scores, ld, B, 0, ctx_len, Lmax, topk, idx, s);
     if (st != DSA_OK) return st;
@@ -615,6 +599,7 @@ dsa_status dsa_decode(const void* q, const void* qI, const void* w, const void* 
     P.out = static_cast<__nv_bfloat16*>(out);
     P.nsplit = decode_attn_splits(B);
     P.part = part;
+    P.advance_ctx = (update_ctx && P.nsplit == 1) ? ctx_len : nullptr;
     st = run_attn(P, s);
     if (st != DSA_OK) return st;
     if (P.nsplit > 1) {
@@ -622,10 +607,6 @@ dsa_status dsa_decode(const void* q, const void* qI, const void* w, const void* 
         const int warps = B * Hq;
         attn_combine_kernel<<<(warps + 3) / 4, 128, 0, s>>>(part, B, P.nsplit, Hq, P.out, nullptr,
                                                             update_ctx ? ctx_len : nullptr, Lmax);
-        if ((st = launch_status()) != DSA_OK) return st;
-    } else if (update_ctx) {
-        LaunchScope ls(K_ADVANCE, s);
-        decode_advance_kernel<<<(B + 127) / 128, 128, 0, s>>>(ctx_len, B, Lmax);
         if ((st = launch_status()) != DSA_OK) return st;
     }
     return DSA_OK;

@@ -45,6 +45,15 @@ struct IndexerParams {
     uint32_t q_box_bytes;       // bytes one Q TMA box brings
     uint32_t k_box_bytes;       // bytes one kI TMA box brings
     long long window;           // > 0 (prefill): keys s <= t - window are not needed (not scored)
+    // decode: the new token of sequence p goes to row ctx_len[p] of the caches before any load of
+    // that key tile (the CTA that owns the tile writes it); null when nothing is appended
+    const uint4* new_k;         // [P, kv16] 16-byte units
+    const uint4* new_v;
+    const uint4* new_kI;        // [P, kI16]
+    uint4* cache_k;             // [P, Lk, kv16]
+    uint4* cache_v;
+    uint4* cache_kI;            // [P, Lk, kI16]
+    int kv16, kI16;
 };
 
 struct IndexerUnit {
@@ -216,6 +225,30 @@ __global__ void __launch_bounds__(IndexerCfg<HI, BN, STAGES>::THREADS, 1)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
+    if (P.new_kI) {
+        // append each sequence's new token in the CTA that owns the key tile holding it, ahead of
+        // that tile's TMA load (generic-proxy stores, then a proxy fence and the barrier below)
+        for (int rd = 0;; ++rd) {
+            const int u = indexer_unit_of(rd, blockIdx.x, gridDim.x);
+            if (u >= P.num_units) break;
+            const IndexerUnit U = indexer_unit<C::TB>(P, u);
+            const long long pos = P.ctx_len[U.p];
+            if (pos < 0 || pos >= P.Lk) {  // reported once per sequence; the sequence is not appended
+                if (U.kt0 == 0 && threadIdx.x == 0) record_error(DSA_DEV_ERR_BOUNDS, 0x501);
+                continue;
+            }
+            const int kt = (int)(pos / kIdxBM);
+            if (kt < U.kt0 || kt >= U.kt1) continue;
+            const long long row = (long long)U.p * P.Lk + pos;
+            for (int i = threadIdx.x; i < P.kv16; i += blockDim.x) {
+                P.cache_k[row * P.kv16 + i] = P.new_k[(long long)U.p * P.kv16 + i];
+                P.cache_v[row * P.kv16 + i] = P.new_v[(long long)U.p * P.kv16 + i];
+            }
+            for (int i = threadIdx.x; i < P.kI16; i += blockDim.x)
+                P.cache_kI[row * P.kI16 + i] = P.new_kI[(long long)U.p * P.kI16 + i];
+        }
+        asm volatile("fence.proxy.async.global;" ::: "memory");
+    }
     if (threadIdx.x == 0) {
         for (int i = 0; i < STAGES; ++i) {
             mbar_init(&a_full[i], 1);

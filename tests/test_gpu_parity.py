@@ -261,6 +261,44 @@ def test_decode_steps_against_oracle(cuda_ok):
             assert_output_ok(got_out[b:b + 1], own, f"decode b={b} step={j}")
 
 
+def test_decode_many_sequences_one_cta_per_token(cuda_ok):
+    """Enough sequences that the attention runs one CTA per token (no key splits): the new rows
+    land in the caches, every context length advances by one, and sampled sequences match the
+    oracle; one sequence has a context longer than k so its top-k is a real selection."""
+    B, Lmax, steps = 300, 2200, 2
+    rng = np.random.default_rng(15)
+    ctx = rng.integers(1, 400, size=B)
+    ctx[7] = 2100
+    cfg, data, kc, vc, kIc = make_decode_case(B, Lmax, ctx, steps)
+    kc_t, vc_t, kIc_t = dev(kc), dev(vc), dev(kIc)
+    ctx_t = torch.from_numpy(ctx.astype(np.int32)).cuda()
+    out = torch.empty((B, cfg.Hq, cfg.D), dtype=torch.bfloat16, device="cuda")
+    idx = torch.empty((B, cfg.k), dtype=torch.int32, device="cuda")
+    for j in range(steps):
+        pos = ctx + j
+        sel = lambda name: np.stack([data[b][name][pos[b]] for b in range(B)])  # noqa: E731
+        dsa.dsa_decode(dev(sel("q")), dev(sel("qI")), dev(sel("w")), dev(sel("k")), dev(sel("v")), dev(sel("kI")),
+                       kc_t, vc_t, kIc_t, ctx_t, cfg.k, cfg.scale, out, idx, update_ctx=True)
+        assert dsa.sync_status() == dsa.DSA_OK
+        assert np.array_equal(ctx_t.cpu().numpy(), pos + 1)
+        for b in (0, 7, 100, B - 1):
+            row = lambda c: c[b, int(pos[b])].view(torch.int16).cpu().numpy().view(np.uint16)  # noqa: E731
+            assert np.array_equal(row(kc_t), data[b]["k"][pos[b]])
+            assert np.array_equal(row(vc_t), data[b]["v"][pos[b]])
+            assert np.array_equal(row(kIc_t), data[b]["kI"][pos[b]])
+        got_idx, got_out = idx.cpu().numpy(), bf16_tensor_to_f64(out)
+        for b in (0, 7, 100, B - 1):
+            t = int(pos[b])
+            d = data[b]
+            r = np.array([t])
+            ref = oracle.dsa_rows(d["q"][r], d["qI"][r], d["w"][r], d["k"], d["v"], d["kI"], r, cfg.k, cfg.scale,
+                                  keep_scores=True)
+            mm = index_set_mismatch(got_idx[b:b + 1], ref["idx"], ref["scores"], ref["tau"], ref["absmax"], r + 1)
+            assert mm["structural"] == 0 and mm["out_of_band"] == 0, (b, j, mm)
+            own, _ = oracle.sparse_attn_rows(d["q"][r], d["k"], d["v"], got_idx[b:b + 1], cfg.scale)
+            assert_output_ok(got_out[b:b + 1], own, f"decode b={b} step={j}")
+
+
 def test_decode_matches_prefill_row(cuda_ok):
     """A decode step at position t gives the prefill result of row t (same indices, close output)."""
     cfg = synth.CONFIGS["32k"]

@@ -41,9 +41,10 @@ def _load():
         lib.oracle_sparse_attn_rows.argtypes = [p, p, p, p, i64, i32, i32, i32, i32, f64, p, p]
         lib.oracle_dsa_rows.argtypes = [p, p, p, p, p, p, p, i64, i32, i32, i32, i32, i32, i32, i64, f64,
                                         p, p, p, p, i64, p, p]
+        lib.oracle_kl_rows.argtypes = [p, p, p, p, p, p, i64, i32, i32, i32, i32, i32, f64, p]
         lib.oracle_num_threads.restype = i32
         for f in ("oracle_index_rows", "oracle_topk_rows", "oracle_sparse_attn_rows",
-                  "oracle_dsa_rows"):
+                  "oracle_dsa_rows", "oracle_kl_rows"):
             getattr(lib, f).restype = None
         _lib = lib
     return _lib
@@ -142,3 +143,24 @@ def dsa_rows(q_rows, qI_rows, w_rows, k, v, kI, t_rows, topk: int, scale: float,
     if keep_scores:
         res["scores"] = scores
     return res
+
+
+def kl_rows(q_rows, k, qI_rows, w_rows, kI, t_rows, scale: float) -> np.ndarray:
+    """Indexer warm-up target KL(P_t || Q_t) (float64 [rows]) for query positions t_rows: P_t the
+    dense causal attention distribution averaged over the Hq heads, Q_t the softmax of the
+    indexer scores over keys 0..t.  q_rows/qI_rows/w_rows hold those positions' rows; k and kI
+    the whole prefix."""
+    t_rows = _c(np.atleast_1d(t_rows), np.int64)
+    nr = t_rows.size
+    q_rows, qI_rows, w_rows = _c(q_rows, np.uint16), _c(qI_rows, np.uint16), _c(w_rows, np.uint16)
+    k, kI = _c(k, np.uint16), _c(kI, np.uint16)
+    _, Hq, D = q_rows.shape
+    Hkv = k.shape[1]
+    HI, dI = qI_rows.shape[1], qI_rows.shape[2]
+    assert q_rows.shape[0] == nr and qI_rows.shape[0] == nr and w_rows.shape == (nr, HI)
+    assert Hq % Hkv == 0 and k.shape[2] == D and kI.shape[1] == dI
+    assert k.shape[0] >= int(t_rows.max()) + 1 and kI.shape[0] >= int(t_rows.max()) + 1
+    kl = np.empty(nr)
+    _load().oracle_kl_rows(_ptr(q_rows), _ptr(k), _ptr(qI_rows), _ptr(w_rows), _ptr(kI), _ptr(t_rows), nr, Hq, Hkv,
+                           D, HI, dI, float(scale), _ptr(kl))
+    return kl

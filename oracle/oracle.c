@@ -28,6 +28,13 @@
  *     (wmrh.cn page, section 2, step 3: standard scaled dot-product attention on the
  *     selected candidates; gsyq.cn page, section 一: GQA adaptation of DSA).
  *
+ *  4. Indexer warm-up target (forward only; the pages' training stage 1 fits the scout to the
+ *     full attention distribution by minimising a KL divergence: gsyq.cn page, section 一, the
+ *     "dense warm-up" paragraph; the pages give no formula, this is the plainest reading):
+ *       P_t(s) = (1/Hq) sum_h softmax_s(scale * q[t,h] . k[s,g(h)])   over s = 0..t (dense)
+ *       Q_t(s) = softmax_s(score(t, s))                                over s = 0..t
+ *       KL_t   = sum_s P_t(s) * (log P_t(s) - log Q_t(s))   (a term with P_t(s) = 0 adds 0)
+ *
  * Inputs are bf16 bit patterns (uint16); each is widened exactly to double.  Every product
  * of two bf16 values is exact in double, so the scores are the true scores up to the
  * rounding of the fp64 sums.  Rows are independent: OpenMP splits them over host cores.
@@ -135,6 +142,45 @@ static void attend_row(const uint16_t *q_row, const uint16_t *kc, const uint16_t
     free(z);
 }
 
+/* Step 4 for one query row with n = t + 1 keys. */
+static double kl_row(const uint16_t *q_row, const uint16_t *kc, const uint16_t *qI_row, const uint16_t *w_row,
+                     const uint16_t *kI, int64_t n, int Hq, int Hkv, int D, int HI, int dI, double scale) {
+    int G = Hq / Hkv;
+    double *z = (double *)malloc((size_t)n * sizeof(double));
+    double *P = (double *)calloc((size_t)n, sizeof(double));
+    double *I = (double *)malloc((size_t)n * sizeof(double));
+    /* P: the dense attention distribution of every head, averaged over heads */
+    for (int h = 0; h < Hq; ++h) {
+        int g = h / G;
+        const uint16_t *qh = q_row + (int64_t)h * D;
+        double zmax = -INFINITY;
+        for (int64_t s = 0; s < n; ++s) {
+            const uint16_t *ks = kc + (s * Hkv + g) * D;
+            double dot = 0.0;
+            for (int d = 0; d < D; ++d) dot += bf16_to_double(qh[d]) * bf16_to_double(ks[d]);
+            z[s] = scale * dot;
+            if (z[s] > zmax) zmax = z[s];
+        }
+        double denom = 0.0;
+        for (int64_t s = 0; s < n; ++s) denom += exp(z[s] - zmax);
+        for (int64_t s = 0; s < n; ++s) P[s] += exp(z[s] - zmax) / denom / (double)Hq;
+    }
+    /* log Q: log-softmax of the indexer scores */
+    index_row(qI_row, w_row, kI, n, HI, dI, I);
+    double imax = -INFINITY;
+    for (int64_t s = 0; s < n; ++s) imax = I[s] > imax ? I[s] : imax;
+    double isum = 0.0;
+    for (int64_t s = 0; s < n; ++s) isum += exp(I[s] - imax);
+    double lse_i = imax + log(isum);
+    double kl = 0.0;
+    for (int64_t s = 0; s < n; ++s)
+        if (P[s] > 0.0) kl += P[s] * (log(P[s]) - (I[s] - lse_i));
+    free(z);
+    free(P);
+    free(I);
+    return kl;
+}
+
 /* ------------------------------------------------------------------------------------- */
 /* Exported entry points.  Row r of every per-row array belongs to query position t_rows[r]. */
 
@@ -194,6 +240,17 @@ void oracle_dsa_rows(const uint16_t *q, const uint16_t *qI, const uint16_t *w, c
                    lse ? lse + r * Hq : NULL);
         if (!scores) free(row);
     }
+}
+
+/* Step 4.  q: [nr, Hq, D], qI: [nr, HI, dI], w: [nr, HI]; k: [>= max t + 1, Hkv, D], kI: [>= max t + 1, dI].
+ * kl[r] = KL(P_t || Q_t) for t = t_rows[r]. */
+void oracle_kl_rows(const uint16_t *q, const uint16_t *kc, const uint16_t *qI, const uint16_t *w, const uint16_t *kI,
+                    const int64_t *t_rows, int64_t nr, int Hq, int Hkv, int D, int HI, int dI, double scale,
+                    double *kl) {
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t r = 0; r < nr; ++r)
+        kl[r] = kl_row(q + r * Hq * D, kc, qI + r * HI * dI, w + r * HI, kI, t_rows[r] + 1, Hq, Hkv, D, HI, dI,
+                       scale);
 }
 
 int oracle_num_threads(void) {

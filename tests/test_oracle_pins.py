@@ -271,3 +271,73 @@ def test_sliding_window_topk_brute_force():
     res = oracle.dsa_rows(rand_bf16(rng, (L, 2, 16)), qI, w, rand_bf16(rng, (L, 1, 16)), rand_bf16(rng, (L, 1, 16)),
                           kI, np.arange(L), k, 0.25, window=1)
     assert np.array_equal(res["idx"][:, 0], np.arange(L)) and np.all(res["idx"][:, 1:] == -1)
+
+
+# ----------------------------------------------------------------------------- warm-up KL target
+
+
+def test_kl_two_keys_closed_form():
+    """Two keys, one head: logits (0, ln 3) give P = (1/4, 3/4); w = 0 gives uniform Q, so
+    KL(P || Q) = ln(27/16) / 4 exactly (the reverse direction would be ln(4/3) / 2)."""
+    D, dI = 128, 64
+    q = np.zeros((1, 1, D)); q[0, 0, 0] = 1.0
+    k = np.zeros((2, 1, D)); k[1, 0, 0] = 1.0
+    qI = np.zeros((1, 1, dI)); qI[0, 0, 0] = 1.0
+    kI = np.ones((2, dI))
+    w = np.zeros((1, 1))
+    got = oracle.kl_rows(bf16_bits(q), bf16_bits(k), bf16_bits(qI), bf16_bits(w), bf16_bits(kI), [1], math.log(3.0))
+    assert got[0] == pytest.approx(math.log(27.0 / 16.0) / 4.0, rel=1e-13)
+
+
+def nonneg_bf16(rng, shape):
+    x = torch.as_tensor(np.abs(rng.standard_normal(shape)) * 0.3, dtype=torch.float32).to(torch.bfloat16)
+    return x.view(torch.int16).numpy().view(np.uint16)
+
+
+def test_kl_vanishes_when_attention_equals_the_indexer():
+    """One head, q = [qI, 0], k = [kI, 0], scale 1, one indexer head of weight 1 and non-negative
+    qI, kI (so the ReLU is the identity): the attention logits equal the indexer scores, P = Q
+    and KL = 0 on every row, including t = 0."""
+    rng = np.random.default_rng(21)
+    L, D, dI = 40, 128, 64
+    qI = nonneg_bf16(rng, (L, 1, dI))
+    kI = nonneg_bf16(rng, (L, dI))
+    q = np.zeros((L, 1, D), dtype=np.uint16); q[:, :, :dI] = qI
+    k = np.zeros((L, 1, D), dtype=np.uint16); k[:, 0, :dI] = kI
+    w = bf16_bits(np.ones((L, 1)))
+    rows = np.arange(L)
+    got = oracle.kl_rows(q, k, qI, w, kI, rows, 1.0)
+    assert np.all(np.abs(got) < 1e-12), got
+
+
+def test_kl_head_average_and_gibbs():
+    """Two query heads with the same query rows give the same P as one head (P is the head
+    average, not the sum); KL >= 0 on random rows, = 0 at t = 0 (a single key)."""
+    rng = np.random.default_rng(22)
+    L, D, HI, dI = 33, 128, 4, 64
+    q1 = rand_bf16(rng, (L, 1, D))
+    q2 = np.concatenate([q1, q1], axis=1)
+    k = rand_bf16(rng, (L, 1, D))
+    qI, kI, w = rand_bf16(rng, (L, HI, dI)), rand_bf16(rng, (L, dI)), rand_bf16(rng, (L, HI))
+    rows = np.arange(L)
+    one = oracle.kl_rows(q1, k, qI, w, kI, rows, 0.0883883)
+    two = oracle.kl_rows(q2, k, qI, w, kI, rows, 0.0883883)
+    np.testing.assert_allclose(two, one, rtol=1e-12, atol=1e-14)
+    assert one[0] == pytest.approx(0.0, abs=1e-15)
+    assert np.all(one[1:] > 0.0)
+
+
+def test_kl_gqa_head_map():
+    """GQA: with Hq = 4 over Hkv = 2, head h reads KV head h // 2.  Swapping the two KV heads and
+    the two query-head pairs together leaves KL unchanged; swapping only the KV heads changes it."""
+    rng = np.random.default_rng(23)
+    L, D, HI, dI = 20, 128, 2, 64
+    q = rand_bf16(rng, (L, 4, D))
+    k = rand_bf16(rng, (L, 2, D))
+    qI, kI, w = rand_bf16(rng, (L, HI, dI)), rand_bf16(rng, (L, dI)), rand_bf16(rng, (L, HI))
+    rows = np.arange(L)
+    base = oracle.kl_rows(q, k, qI, w, kI, rows, 0.0883883)
+    both = oracle.kl_rows(q[:, [2, 3, 0, 1]], k[:, [1, 0]], qI, w, kI, rows, 0.0883883)
+    kv_only = oracle.kl_rows(q, k[:, [1, 0]], qI, w, kI, rows, 0.0883883)
+    np.testing.assert_allclose(both, base, rtol=1e-12, atol=1e-14)
+    assert np.max(np.abs(kv_only - base)) > 1e-6

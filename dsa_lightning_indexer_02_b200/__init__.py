@@ -31,8 +31,8 @@ _lib = ctypes.CDLL(LIB_PATH)
 
 DSA_OK, DSA_ERR_INVALID_ARG, DSA_ERR_UNSUPPORTED, DSA_ERR_WORKSPACE, DSA_ERR_CUDA, DSA_ERR_TIMEOUT, \
     DSA_ERR_DEVICE_INPUT = range(7)
-DSA_OP_INDEX, DSA_OP_TOPK, DSA_OP_SPARSE_ATTN, DSA_OP_PREFILL, DSA_OP_DECODE = range(5)
-PROFILE_KINDS = ("indexer", "topk", "sparse_attn", "combine", "decode_append", "advance", "selftest")
+DSA_OP_INDEX, DSA_OP_TOPK, DSA_OP_SPARSE_ATTN, DSA_OP_PREFILL, DSA_OP_DECODE, DSA_OP_INDEXER_KL = range(6)
+PROFILE_KINDS = ("indexer", "topk", "sparse_attn", "combine", "decode_append", "advance", "selftest", "kl")
 
 _p, _i, _i64, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
 _SIGS = {
@@ -52,6 +52,7 @@ _SIGS = {
     "dsa_decode_noalloc": (_i, [_p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _i, _i64, _i, _i, _i, _i, _i, _i, _f, _i,
                                 _p, _p, _p]),
     "dsa_decode_noalloc_scratch_bytes": (_sz, []),
+    "dsa_indexer_kl": (_i, [_p, _p, _p, _p, _p, _i64, _i, _i, _i, _i, _i, _f, _p, _p, _sz, _p]),
     "dsa_workspace_size": (_sz, [_i, _i64, _i, _i, _i, _i]),
     "dsa_sync_status": (_i, [_p]),
     "dsa_profile_begin": (None, []),
@@ -204,6 +205,23 @@ def dsa_prefill_rows(q_rows, k, v, qI_rows, kI, w_rows, row0: int, topk: int, sc
                                k.shape[1], D, HI, dI, topk, window, float(scale), _ptr(out_rows), _ptr(idx_rows),
                                _ptr(ws), ws.numel() * ws.element_size(), _stream(stream))
     _check(st, "dsa_prefill_rows")
+
+
+def dsa_indexer_kl(q, k, qI, kI, w, scale: float, kl, ws=None, stream=None) -> None:
+    """Indexer warm-up target KL(P_t || Q_t) for every query row of one causal sequence into kl
+    (float32 [L]); see dsa_indexer_kl in include/dsa.h."""
+    import torch
+    _need(q, torch.bfloat16, "q", 3), _need(k, torch.bfloat16, "k", 3), _need(qI, torch.bfloat16, "qI", 3)
+    _need(kI, torch.bfloat16, "kI", 2), _need(w, torch.bfloat16, "w", 2), _need(kl, torch.float32, "kl", 1)
+    L, Hq, D = q.shape
+    HI, dI = qI.shape[1], qI.shape[2]
+    if k.shape[0] < L or kI.shape[0] < L or kl.shape[0] < L:
+        raise ValueError("k, kI and kl must cover the L query rows")
+    if ws is None:
+        ws = torch.empty(workspace_size(DSA_OP_INDEXER_KL, L, 1, Hq, HI, 1), dtype=torch.uint8, device=q.device)
+    st = _lib.dsa_indexer_kl(_ptr(q), _ptr(k), _ptr(qI), _ptr(kI), _ptr(w), L, Hq, k.shape[1], D, HI, dI,
+                             float(scale), _ptr(kl), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream))
+    _check(st, "dsa_indexer_kl")
 
 
 def dsa_decode(q, qI, w, k_new, v_new, kI_new, k_cache, v_cache, kI_cache, ctx_len, topk: int, scale: float, out,

@@ -12,6 +12,7 @@
 #include <vector>
 
 #include "attn.cuh"
+#include "kl.cuh"
 #include "dsa.h"
 #include "indexer.cuh"
 #include "ptx.cuh"
@@ -72,7 +73,7 @@ struct LaunchScope {
     }
 };
 
-enum { K_INDEX = 0, K_TOPK = 1, K_ATTN = 2, K_COMBINE = 3, K_APPEND = 4, K_ADVANCE = 5, K_SELFTEST = 6 };
+enum { K_INDEX = 0, K_TOPK = 1, K_ATTN = 2, K_COMBINE = 3, K_APPEND = 4, K_ADVANCE = 5, K_SELFTEST = 6, K_KL = 7 };
 
 dsa_status launch_status() {
     cudaError_t e = cudaGetLastError();
@@ -450,6 +451,14 @@ dsa_status dsa_sparse_attn(const void* q, const void* k, const void* v, const in
 }
 
 size_t dsa_workspace_size(int op, int64_t L, int B, int Hq, int HI, int topk) {
+    if (op == DSA_OP_INDEXER_KL) {  // score rows only (topk unused)
+        if (L <= 0 || HI <= 0) return 0;
+        const int64_t ld = prefill_ld(L);
+        int64_t rows = (int64_t(4) << 30) / (ld * 4);
+        rows = std::max<int64_t>(256, rows / 256 * 256);
+        rows = std::min<int64_t>(rows, L);
+        return align_up((size_t)rows * ld * 4, 256);
+    }
     if (L <= 0 || topk <= 0 || HI <= 0) return 0;
     switch (op) {
     case DSA_OP_INDEX:
@@ -467,6 +476,57 @@ size_t dsa_workspace_size(int op, int64_t L, int B, int Hq, int HI, int topk) {
         return decode_ws_layout(L, B, Hq, topk, true).total;
     default: return 0;
     }
+}
+
+dsa_status dsa_indexer_kl(const void* q, const void* k, const void* qI, const void* kI, const void* w, int64_t L,
+                          int Hq, int Hkv, int D, int HI, int dI, float scale, float* kl, void* ws, size_t ws_bytes,
+                          dsa_stream_t stream) {
+    if (!q || !k || !qI || !kI || !w || !kl) return DSA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(qI) || !aligned16(kI) || !aligned16(w) ||
+        (reinterpret_cast<uintptr_t>(kl) & 3u))
+        return DSA_ERR_INVALID_ARG;
+    if (L <= 0 || HI <= 0 || dI <= 0 || !(scale == scale)) return DSA_ERR_INVALID_ARG;
+    dsa_status st = check_attn_shape(Hq, Hkv, D);
+    if (st != DSA_OK) return st;
+    if (Hq / Hkv > 8 || dI != kIdxBK || !hi_supported_prefill(HI) || L * HI > (int64_t)INT32_MAX)
+        return DSA_ERR_UNSUPPORTED;
+    if (!ws || !aligned16(ws)) return DSA_ERR_WORKSPACE;
+    const int64_t ld = prefill_ld(L);
+    const int TB = 256 / HI;
+    int64_t C = (int64_t)((ws_bytes > 512 ? ws_bytes - 512 : 0) / ((size_t)ld * 4));
+    C = std::min<int64_t>(C, L);
+    if (C >= TB) C = C / TB * TB;
+    if (C < std::min<int64_t>(L, TB)) return DSA_ERR_WORKSPACE;
+    float* scores = static_cast<float*>(ws);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    static bool attr_set = false;
+    if (!attr_set) {
+        if (cudaFuncSetAttribute(indexer_kl_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kl_smem_bytes(4)) !=
+            cudaSuccess)
+            return DSA_ERR_CUDA;
+        attr_set = true;
+    }
+    for (int64_t t0 = 0; t0 < L; t0 += C) {
+        const int n = (int)std::min<int64_t>(C, L - t0);
+        st = run_indexer(static_cast<const __nv_bfloat16*>(qI) + t0 * HI * dI, kI,
+                         static_cast<const __nv_bfloat16*>(w) + t0 * HI, 1, n, t0, nullptr, t0 + n, HI, scores, ld, s);
+        if (st != DSA_OK) return st;
+        KlParams P{};
+        P.q = static_cast<const __nv_bfloat16*>(q) + t0 * Hq * D;
+        P.k = static_cast<const __nv_bfloat16*>(k);
+        P.scores = scores;
+        P.ld = ld;
+        P.T = n;
+        P.q_pos0 = t0;
+        P.Hq = Hq;
+        P.Hkv = Hkv;
+        P.scale_log2 = scale * 1.4426950408889634f;
+        P.kl = kl + t0;
+        LaunchScope ls(K_KL, s);
+        indexer_kl_kernel<<<(n + kKlTokens - 1) / kKlTokens, kKlTokens * 32, kl_smem_bytes(Hkv), s>>>(P);
+        if ((st = launch_status()) != DSA_OK) return st;
+    }
+    return DSA_OK;
 }
 
 dsa_status dsa_prefill_rows(const void* q, const void* k, const void* v, const void* qI, const void* kI,

@@ -50,7 +50,8 @@ typedef enum {
 } dsa_status;
 
 /* Workspace kinds for dsa_workspace_size(). */
-enum { DSA_OP_INDEX = 0, DSA_OP_TOPK = 1, DSA_OP_SPARSE_ATTN = 2, DSA_OP_PREFILL = 3, DSA_OP_DECODE = 4 };
+enum { DSA_OP_INDEX = 0, DSA_OP_TOPK = 1, DSA_OP_SPARSE_ATTN = 2, DSA_OP_PREFILL = 3, DSA_OP_DECODE = 4,
+       DSA_OP_INDEXER_KL = 5 };
 
 /* Human-readable name of a status code (static string, never NULL). */
 const char *dsa_status_string(int status);
@@ -141,6 +142,25 @@ dsa_status dsa_prefill_rows(const void *q, const void *k, const void *v, const v
                             size_t ws_bytes, dsa_stream_t stream);
 
 /*
+ * Indexer warm-up target, forward only (the pages' training stage 1 fits the scout to the full
+ * attention distribution by minimising a KL divergence: page gsyq.cn, section 一; the pages
+ * give no formula, this is the library's reading).  For every query position t < L:
+ *   P_t(s) = (1/Hq) sum_h softmax_s(scale * q[t,h] . k[s, h / (Hq/Hkv)])   s = 0..t  (dense)
+ *   Q_t(s) = softmax_s(score(t, s))          with score as in dsa_index
+ *   kl[t]  = sum_s P_t(s) * (log P_t(s) - log Q_t(s))                      (natural log)
+ *   q bf16 [L, Hq, D]; k bf16 [L, Hkv, D]; qI bf16 [L, HI, dI]; kI bf16 [L, dI]; w bf16 [L, HI]
+ *   kl      float [L] (device, 4-byte aligned), written
+ *   ws      score rows for a chunk of queries: at least
+ *           dsa_workspace_size(DSA_OP_INDEXER_KL, L, 1, Hq, HI, 1) bytes recommended; any size
+ *           holding min(L, 256/HI) rows works (smaller sizes mean more, shorter chunks).
+ * Supported: D = 128, dI = 64, Hkv in {1, 2, 4}, Hq/Hkv <= 8, HI a power of two <= 64.  Dense
+ * cost: 4 x Hq x D flop per causal (t, s) pair plus the indexer.  Status codes as dsa_prefill.
+ */
+dsa_status dsa_indexer_kl(const void *q, const void *k, const void *qI, const void *kI, const void *w, int64_t L,
+                          int Hq, int Hkv, int D, int HI, int dI, float scale, float *kl, void *ws, size_t ws_bytes,
+                          dsa_stream_t stream);
+
+/*
  * dsa_prefill with a sliding window of `window` keys per query (SW-DSA, see dsa_topk_window): the
  * indexer skips key tiles that lie wholly before every window of a query block, top-k selects
  * within the window, attention runs over the selected keys.  window = 0: identical to dsa_prefill.
@@ -202,7 +222,8 @@ size_t dsa_decode_noalloc_scratch_bytes(void);
  * Bytes of workspace an entry point needs.  op: DSA_OP_*.  L: sequence length (prefill) or cache
  * capacity Lmax (decode); B: sequences (decode); Hq: query heads; HI: indexer heads; topk.
  * DSA_OP_PREFILL returns the recommended size (score rows of up to 4 GiB per chunk plus index
- * rows); DSA_OP_INDEX/TOPK/SPARSE_ATTN return 0.  Returns 0 for invalid arguments.
+ * rows); DSA_OP_INDEXER_KL the score rows alone (topk ignored); DSA_OP_INDEX/TOPK/SPARSE_ATTN
+ * return 0.  Returns 0 for invalid arguments.
  */
 size_t dsa_workspace_size(int op, int64_t L, int B, int Hq, int HI, int topk);
 
@@ -217,9 +238,10 @@ dsa_status dsa_sync_status(dsa_stream_t stream);
  * kernel the library launches (on the launching stream); dsa_profile_end() synchronises those
  * events, stops recording and returns, per kernel kind, the number of launches and the total
  * milliseconds.  Kinds: 0 indexer, 1 top-k, 2 sparse attention, 3 split combine, 4 decode
- * append, 5 context advance, 6 self-test.  Arrays have DSA_PROFILE_KINDS entries.
+ * append and 5 context advance (both now done inside other kernels: always 0), 6 self-test,
+ * 7 indexer warm-up KL.  Arrays have DSA_PROFILE_KINDS entries.
  */
-#define DSA_PROFILE_KINDS 7
+#define DSA_PROFILE_KINDS 8
 void dsa_profile_begin(void);
 dsa_status dsa_profile_end(int64_t *launches, double *total_ms);
 

@@ -31,6 +31,8 @@ def test_workspace_sizes():
     assert dsa.workspace_size(dsa.DSA_OP_PREFILL, 1000, 1, 8, 4, 256) == 1000 * 1000 * 4 + 1024000
     assert dsa.workspace_size(dsa.DSA_OP_DECODE, 131328, 16, 32, 32, 2048) >= 16 * 131328 * 4
     assert dsa.workspace_size(dsa.DSA_OP_INDEX, 100) == 0
+    # indexer KL at 32K: all 32768 score rows fit in 4 GiB
+    assert dsa.workspace_size(dsa.DSA_OP_INDEXER_KL, 32768, 1, 32, 32, 1) == 32768 * 32768 * 4
     assert dsa.workspace_size(dsa.DSA_OP_PREFILL, 0) == 0
     assert dsa.workspace_size(99, 100) == 0
 
@@ -79,6 +81,14 @@ def test_host_validation_without_gpu():
         dsa.DSA_ERR_WORKSPACE
     assert lib.dsa_decode(*dargs, 0, 4096, 32, 4, 128, 32, 64, 2048, f, 0, A, None, A, 1 << 30, None) == \
         dsa.DSA_ERR_INVALID_ARG
+    # indexer KL: pointers, shapes, workspace
+    kargs = [A] * 5 + [1024]
+    assert lib.dsa_indexer_kl(None, *[A] * 4, 1024, 32, 4, 128, 32, 64, f, A, A, 1 << 30, None) == \
+        dsa.DSA_ERR_INVALID_ARG
+    assert lib.dsa_indexer_kl(*kargs, 32, 4, 64, 32, 64, f, A, A, 1 << 30, None) == dsa.DSA_ERR_UNSUPPORTED
+    assert lib.dsa_indexer_kl(*kargs, 64, 4, 128, 32, 64, f, A, A, 1 << 30, None) == dsa.DSA_ERR_UNSUPPORTED
+    assert lib.dsa_indexer_kl(*kargs, 32, 4, 128, 32, 64, f, A, None, 0, None) == dsa.DSA_ERR_WORKSPACE
+    assert lib.dsa_indexer_kl(*kargs, 32, 4, 128, 32, 64, f, A, A, 64, None) == dsa.DSA_ERR_WORKSPACE
     # self test bounds
     assert lib.dsa_selftest_timeout(0, None) == dsa.DSA_ERR_INVALID_ARG
     assert lib.dsa_selftest_timeout(3_000_000_000, None) == dsa.DSA_ERR_INVALID_ARG

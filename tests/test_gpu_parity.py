@@ -459,3 +459,58 @@ def test_prefill_rows_ranges_reproduce_prefill(cuda_ok, c32k):
     assert dsa.sync_status() == dsa.DSA_OK
     assert torch.equal(idx, idx_full)
     assert torch.equal(out.view(torch.int16), out_full.view(torch.int16))
+
+
+# ----------------------------------------------------------------------------- warm-up KL target
+# Tolerance: logits are fp32 sums of 128 exact bf16 products, P and log P come from fp32
+# exp2/log2 (a few ulp) and per-lane fp32 sums over <= 32K keys, and the indexer scores carry
+# their own fp32 error, which enters KL linearly (sum_s P_t(s) * dscore).  Together well below
+# 1e-4 relative on these inputs; the test allows 2e-4 + 2e-4 |KL|.
+KL_ATOL, KL_RTOL = 2e-4, 2e-4
+
+
+def run_kl(x, L, scale, ws_bytes=None):
+    kl = torch.empty(L, dtype=torch.float32, device="cuda")
+    ws = None if ws_bytes is None else torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
+    dsa.dsa_indexer_kl(dev(x["q"][:L]), dev(x["k"][:L]), dev(x["qI"][:L]), dev(x["kI"][:L]), dev(x["w"][:L]), scale,
+                       kl, ws)
+    assert dsa.sync_status() == dsa.DSA_OK
+    return kl.cpu().numpy().astype(np.float64)
+
+
+def test_indexer_kl_tiny_every_row(cuda_ok, tiny):
+    cfg, x, _ = tiny
+    got = run_kl(x, cfg.L, cfg.scale)
+    rows = np.arange(cfg.L)
+    want = oracle.kl_rows(x["q"], x["k"], x["qI"], x["w"], x["kI"], rows, cfg.scale)
+    np.testing.assert_allclose(got, want, rtol=KL_RTOL, atol=KL_ATOL)
+    assert got[0] == pytest.approx(0.0, abs=1e-6)
+
+
+def test_indexer_kl_32k_sampled_rows_and_chunking(cuda_ok, c32k):
+    cfg, x = c32k[0], c32k[1]
+    L = 6000
+    got = run_kl(x, L, cfg.scale)
+    rows = np.array([0, 1, 15, 16, 17, 255, 256, 2047, 2048, 4099, L - 2, L - 1])
+    want = oracle.kl_rows(x["q"][rows], x["k"], x["qI"][rows], x["w"][rows], x["kI"], rows, cfg.scale)
+    np.testing.assert_allclose(got[rows], want, rtol=KL_RTOL, atol=KL_ATOL)
+    assert np.all(np.isfinite(got)) and np.all(got > -KL_ATOL)
+    # a workspace of 1000 score rows: six chunks, the same values bit for bit
+    small = run_kl(x, L, cfg.scale, ws_bytes=1000 * ((L + 3) // 4 * 4) * 4 + 512)
+    assert np.array_equal(small, got)
+
+
+def test_indexer_kl_gqa_shapes(cuda_ok):
+    rng = np.random.default_rng(16)
+    L, HI, dI = 500, 8, 64
+    for Hq, Hkv in ((16, 2), (8, 4), (8, 1)):
+        q, k = rng.standard_normal((L, Hq, 128)), rng.standard_normal((L, Hkv, 128))
+        qI, kI, w = rng.standard_normal((L, HI, dI)), rng.standard_normal((L, dI)), rng.standard_normal((L, HI))
+        tq, tk, tqI, tkI, tw = (torch.from_numpy(a.astype(np.float32)).to(torch.bfloat16) for a in (q, k, qI, kI, w))
+        bits = [t.view(torch.int16).numpy().view(np.uint16) for t in (tq, tk, tqI, tkI, tw)]
+        kl = torch.empty(L, dtype=torch.float32, device="cuda")
+        dsa.dsa_indexer_kl(tq.cuda(), tk.cuda(), tqI.cuda(), tkI.cuda(), tw.cuda(), 0.0883883, kl)
+        assert dsa.sync_status() == dsa.DSA_OK
+        want = oracle.kl_rows(bits[0], bits[1], bits[2], bits[4], bits[3], np.arange(L), 0.0883883)
+        np.testing.assert_allclose(kl.cpu().numpy().astype(np.float64), want, rtol=KL_RTOL, atol=KL_ATOL,
+                                   err_msg=f"Hq={Hq} Hkv={Hkv}")

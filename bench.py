@@ -175,6 +175,7 @@ def main():
     ap.add_argument("--decode-steps", type=int, default=256)
     ap.add_argument("--decode-ctx", type=int, default=0, help="override the cached context (small profiling cases)")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-kl", action="store_true", help="skip the indexer warm-up KL measurement")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
@@ -368,6 +369,11 @@ def main():
             dcfg = dataclasses.replace(dcfg, L=args.decode_ctx, iid_from=args.decode_ctx)
         decode = run_decode(torch, dsa, dcfg, args.decode_steps, rank, world, barrier, max_over_ranks, peaks)
 
+    # ---- indexer warm-up KL target on the 32K workload (dense, tensor-core bound)
+    kl = None
+    if not args.no_kl:
+        kl = run_kl(torch, dsa, synth.CONFIGS["32k"], barrier, max_over_ranks, peaks)
+
     cpu = None
     if rank == 0 and not args.no_cpu and world == 1:
         cpu = cpu_baseline(cfg, x, budget_s=args.cpu_seconds)
@@ -381,7 +387,8 @@ def main():
                        "parallelism": f"dp{world} (independent sequences)",
                        "l2": "inputs (1.8 GB) larger than L2; no flush"},
             "roofline": roofline, "kernels": kern, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
-            "clocks": clk, "decode": decode, "adjacent_union_16": union16, "path_counters": counters}
+            "clocks": clk, "decode": decode, "indexer_kl": kl, "adjacent_union_16": union16,
+            "path_counters": counters}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -409,6 +416,47 @@ def lib_hash() -> str:
         with open(os.path.join(csrc, fn), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:12]
+
+
+def run_kl(torch, dsa, cfg, barrier, max_over_ranks, peaks, reps: int = 3):
+    """dsa_indexer_kl over one whole sequence of the workload: KL(P_t || Q_t) for every query row
+    (indexer scores per chunk, then the dense two-pass kernel); tokens/s and the dense kernel's
+    fraction of the bf16 tensor peak (4 x Hq x D flop per causal pair)."""
+    L = cfg.L
+    x = {n: synth.to_torch(synth.tensor(cfg, n, 0, L)).cuda() for n in ("q", "k", "qI", "kI", "w")}
+    kl = torch.empty(L, dtype=torch.float32, device="cuda")
+    ws = torch.empty(dsa.workspace_size(dsa.DSA_OP_INDEXER_KL, L, 1, cfg.Hq, cfg.HI, 1), dtype=torch.uint8,
+                     device="cuda")
+
+    def run():
+        dsa.dsa_indexer_kl(x["q"], x["k"], x["qI"], x["kI"], x["w"], cfg.scale, kl, ws)
+
+    run()
+    torch.cuda.synchronize()
+    if dsa.sync_status() != dsa.DSA_OK:
+        raise SystemExit("indexer KL warm-up failed")
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    dsa.profile_begin()
+    ev0.record()
+    for _ in range(reps):
+        run()
+    ev1.record()
+    torch.cuda.synchronize()
+    prof = dsa.profile_end()
+    ms = max_over_ranks(ev0.elapsed_time(ev1)) / reps
+    pairs = L * (L + 1) / 2
+    flop = 4.0 * cfg.Hq * cfg.D * pairs
+    k_ms = prof["kl"]["ms"] / reps
+    achieved = flop / (k_ms / 1e3) / 1e12
+    tpeak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    return {"workload": "prefill_32k", "value": L / (ms / 1e3), "unit": "tokens/s", "ms_per_sequence": ms,
+            "kernel_ms": k_ms, "indexer_ms": prof["indexer"]["ms"] / reps,
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": tpeak,
+                         "unit": "TFLOP/s", "frac": achieved / tpeak,
+                         "algorithmic": "4 x Hq x D flop per causal (t, s) pair (two passes of Q.K)"},
+            "mean_kl": float(kl.mean()), "mma": "warp-level m16n8k16 (mma.sync)"}
 
 
 def run_decode(torch, dsa, cfg, steps, rank, world, barrier, max_over_ranks, peaks):

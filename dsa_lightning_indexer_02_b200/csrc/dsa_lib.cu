@@ -343,6 +343,17 @@ DecodeWs decode_ws_layout(int64_t Lmax, int B, int Hq, int topk, bool need_idx) 
 
 int64_t prefill_ld(int64_t L) { return (int64_t)align_up((size_t)L, 4); }
 
+// Query rows per chunk for a workspace of ws_bytes holding C score rows of ld floats (and, with
+// idx_per_row > 0, an index region of C rows after them at a 256-byte boundary): the most that
+// fit, whole query blocks of TB rows unless the chunk covers every remaining row.  0 = too small.
+int64_t chunk_rows(size_t ws_bytes, int64_t ld, int64_t idx_per_row, int64_t rows, int TB) {
+    const size_t per_row = (size_t)ld * 4 + (size_t)idx_per_row * 4;
+    int64_t C = std::min<int64_t>(rows, (int64_t)(ws_bytes / per_row));
+    while (C > 0 && align_up((size_t)C * ld * 4, 256) + (size_t)C * idx_per_row * 4 > ws_bytes) --C;
+    if (C < rows && C >= TB) C = C / TB * TB;
+    return C;
+}
+
 }  // namespace
 
 // ------------------------------------------------------------------ allocation-free decode
@@ -493,9 +504,7 @@ dsa_status dsa_indexer_kl(const void* q, const void* k, const void* qI, const vo
     if (!ws || !aligned16(ws)) return DSA_ERR_WORKSPACE;
     const int64_t ld = prefill_ld(L);
     const int TB = 256 / HI;
-    int64_t C = (int64_t)((ws_bytes > 512 ? ws_bytes - 512 : 0) / ((size_t)ld * 4));
-    C = std::min<int64_t>(C, L);
-    if (C >= TB) C = C / TB * TB;
+    const int64_t C = chunk_rows(ws_bytes, ld, 0, L, TB);
     if (C < std::min<int64_t>(L, TB)) return DSA_ERR_WORKSPACE;
     float* scores = static_cast<float*>(ws);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -547,10 +556,7 @@ dsa_status dsa_prefill_rows(const void* q, const void* k, const void* v, const v
     if (!ws || !aligned16(ws)) return DSA_ERR_WORKSPACE;
     const int64_t ld = prefill_ld(Lk);
     const int TB = 256 / HI;
-    const size_t per_row = (size_t)ld * 4 + (idx_out ? 0 : (size_t)topk * 4);
-    int64_t C = (int64_t)((ws_bytes > 512 ? ws_bytes - 512 : 0) / per_row);  // 512: alignment slack
-    C = std::min<int64_t>(C, rows);
-    if (C >= TB) C = C / TB * TB;
+    const int64_t C = chunk_rows(ws_bytes, ld, idx_out ? 0 : topk, rows, TB);
     if (C < std::min<int64_t>(rows, TB)) return DSA_ERR_WORKSPACE;
     float* scores = static_cast<float*>(ws);
     int32_t* idx_ws = idx_out ? nullptr

@@ -176,6 +176,10 @@ def main():
     ap.add_argument("--decode-ctx", type=int, default=0, help="override the cached context (small profiling cases)")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-kl", action="store_true", help="skip the indexer warm-up KL measurement")
+    ap.add_argument("--kl-only", action="store_true",
+                    help="measure only the indexer warm-up KL and print its object (profiling cases)")
+    ap.add_argument("--kl-rows", type=int, default=0,
+                    help="query rows of the 32K workload for the KL measurement (default: all 32768)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
@@ -209,6 +213,11 @@ def main():
         return reduce_max(v, dist if world > 1 else None, device="cuda")
 
     peaks, peak_src = load_peaks()
+    if args.kl_only:
+        kl = run_kl(torch, dsa, synth.CONFIGS["32k"], barrier, max_over_ranks, peaks, rows=args.kl_rows)
+        if rank == 0:
+            print(json.dumps({"indexer_kl": kl}), flush=True)
+        return 0
     cfg = synth.CONFIGS[args.workload]
     x = synth.inputs(cfg, 0, cfg.L, seq=rank)
     names = ("q", "k", "v", "qI", "kI", "w")
@@ -372,7 +381,7 @@ def main():
     # ---- indexer warm-up KL target on the 32K workload (dense, tensor-core bound)
     kl = None
     if not args.no_kl:
-        kl = run_kl(torch, dsa, synth.CONFIGS["32k"], barrier, max_over_ranks, peaks)
+        kl = run_kl(torch, dsa, synth.CONFIGS["32k"], barrier, max_over_ranks, peaks, rows=args.kl_rows)
 
     cpu = None
     if rank == 0 and not args.no_cpu and world == 1:
@@ -418,11 +427,12 @@ def lib_hash() -> str:
     return h.hexdigest()[:12]
 
 
-def run_kl(torch, dsa, cfg, barrier, max_over_ranks, peaks, reps: int = 3):
-    """dsa_indexer_kl over one whole sequence of the workload: KL(P_t || Q_t) for every query row
-    (indexer scores per chunk, then the dense two-pass kernel); tokens/s and the dense kernel's
-    fraction of the bf16 tensor peak (4 x Hq x D flop per causal pair)."""
-    L = cfg.L
+def run_kl(torch, dsa, cfg, barrier, max_over_ranks, peaks, reps: int = 3, rows: int = 0):
+    """dsa_indexer_kl over one sequence of the workload (its first `rows` tokens, default all):
+    KL(P_t || Q_t) for every query row (indexer scores per chunk, then the dense two-pass
+    kernel); tokens/s and the dense kernel's fraction of the bf16 tensor peak (4 x Hq x D flop
+    per causal pair).  One untimed call, then `reps` timed calls."""
+    L = min(rows, cfg.L) if rows > 0 else cfg.L
     x = {n: synth.to_torch(synth.tensor(cfg, n, 0, L)).cuda() for n in ("q", "k", "qI", "kI", "w")}
     kl = torch.empty(L, dtype=torch.float32, device="cuda")
     ws = torch.empty(dsa.workspace_size(dsa.DSA_OP_INDEXER_KL, L, 1, cfg.Hq, cfg.HI, 1), dtype=torch.uint8,
@@ -451,7 +461,8 @@ def run_kl(torch, dsa, cfg, barrier, max_over_ranks, peaks, reps: int = 3):
     k_ms = prof["kl"]["ms"] / reps
     achieved = flop / (k_ms / 1e3) / 1e12
     tpeak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
-    return {"workload": "prefill_32k", "value": L / (ms / 1e3), "unit": "tokens/s", "ms_per_sequence": ms,
+    return {"workload": "prefill_32k" if L == cfg.L else f"prefill_32k_first_{L}", "value": L / (ms / 1e3),
+            "unit": "tokens/s", "ms_per_sequence": ms,
             "kernel_ms": k_ms, "indexer_ms": prof["indexer"]["ms"] / reps,
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": tpeak,
                          "unit": "TFLOP/s", "frac": achieved / tpeak,

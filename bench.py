@@ -139,6 +139,13 @@ def cpu_baseline(cfg, x, budget_s: float = 15.0, seed: int = 7) -> dict:
 
 
 # ----------------------------------------------------------------------------- reference arm
+def bench_config(cfg, workload: str, world: int) -> dict:
+    """The `config` object of the JSON line, identical for both arms."""
+    return {"workload": f"prefill_{workload}", "L": cfg.L, "k": cfg.k, "Hq": cfg.Hq, "Hkv": cfg.Hkv, "D": cfg.D,
+            "HI": cfg.HI, "dI": cfg.dI, "batch": 1, "parallelism": f"dp{world} (independent sequences)",
+            "l2": "inputs (1.8 GB) larger than L2; no flush"}
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -157,7 +164,7 @@ def run_reference(args):
     line = {"metric": METRIC, "value": value, "unit": UNIT, "impl": "reference", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * cfg.L / value,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": {"workload": f"prefill_{args.workload}", "L": cfg.L, "k": cfg.k},
+            "data": "synthetic", "config": bench_config(cfg, args.workload, max(1, args.gpus)),
             "cpu_baseline": cb, "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
                                         "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -391,10 +398,7 @@ def main():
             "warmup": max(3, args.warmup), "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded; 512 frame + 64 text token layout, block-structured keys)",
-            "config": {"workload": f"prefill_{args.workload}", "L": cfg.L, "k": cfg.k, "Hq": cfg.Hq,
-                       "Hkv": cfg.Hkv, "D": cfg.D, "HI": cfg.HI, "dI": cfg.dI, "batch": 1,
-                       "parallelism": f"dp{world} (independent sequences)",
-                       "l2": "inputs (1.8 GB) larger than L2; no flush"},
+            "config": bench_config(cfg, args.workload, world),
             "roofline": roofline, "kernels": kern, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
             "clocks": clk, "decode": decode, "indexer_kl": kl, "adjacent_union_16": union16,
             "path_counters": counters}

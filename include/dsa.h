@@ -78,8 +78,9 @@ dsa_status dsa_index(const void *qI, const void *kI, const void *w, int Lq, int6
  *   idx     int32 [Lq, k]: the min(k, n_i) keys with the largest scores (equal scores: lower key
  *           index first), then -1 padding.  Exact and deterministic: a row's output depends
  *           only on that row's scores (not on Lq, chunking or the kernel variant).  Order within
- *           a row: the selected keys grouped by region ((index / 32) mod 4, regions 0..3 in turn),
- *           ascending within a region; callers may treat a row as a set.
+ *           a row: when the row has no more than k competing keys, all of them in ascending
+ *           order; otherwise the selected keys grouped by region ((index / 32) mod 4, regions 0..3
+ *           in turn), ascending within a region.  Callers may treat a row as a set.
  *   ws, ws_bytes  unused (may be NULL/0); kept so callers can pass a workspace uniformly.
  * Cites: page gsyq.cn section 一 (top 2048 per token), section 八 (deterministic top-k).
  */

@@ -514,3 +514,54 @@ def test_indexer_kl_gqa_shapes(cuda_ok):
         want = oracle.kl_rows(bits[0], bits[1], bits[2], bits[4], bits[3], np.arange(L), 0.0883883)
         np.testing.assert_allclose(kl.cpu().numpy().astype(np.float64), want, rtol=KL_RTOL, atol=KL_ATOL,
                                    err_msg=f"Hq={Hq} Hkv={Hkv}")
+
+
+def canonical_order(selected, n_comp, lo, k):
+    """The documented output order of a top-k row: ascending when every competing key is kept,
+    else grouped by region ((index / 32) mod 4) and ascending within a region; -1 padding."""
+    sel = [int(i) for i in selected if i >= 0]
+    if n_comp <= k:
+        row = list(range(lo, lo + n_comp))
+    else:
+        row = sorted(sel, key=lambda i: ((i // 32) % 4, i))
+    return row + [-1] * (k - len(row))
+
+
+def test_topk_randomized_exact_order(cuda_ok):
+    """Random row lengths, k, windows and score distributions (Gaussian, heavy integer ties,
+    signed zeros): the GPU rows equal the oracle's sets in the documented order, entry by entry."""
+    rng = np.random.default_rng(17)
+    for case in range(18):
+        rows = int(rng.integers(1, 24))
+        q_pos0 = int(rng.integers(0, 20000))
+        k = int(rng.choice([1, 7, 64, 300, 2048, 4096]))
+        window = int(rng.choice([0, 0, 100, 5000]))
+        n_max = q_pos0 + rows
+        ld = (n_max + 3) // 4 * 4
+        kind = case % 3
+        if kind == 0:
+            s = (rng.standard_normal((rows, ld)) * 10).astype(np.float32)
+        elif kind == 1:
+            s = rng.integers(-2, 3, size=(rows, ld)).astype(np.float32)
+        else:
+            s = np.where(rng.random((rows, ld)) < 0.5, np.float32(0.0), np.float32(-0.0))
+            s[:, ::13] = 2.0
+        idx = torch.empty((rows, k), dtype=torch.int32, device="cuda")
+        dsa.dsa_topk(torch.from_numpy(s).cuda(), q_pos0, k, idx, window=window)
+        assert dsa.sync_status() == dsa.DSA_OK
+        n = q_pos0 + np.arange(rows) + 1
+        want, _ = oracle.topk_rows(s.astype(np.float64), n, k, window=window)
+        got = idx.cpu().numpy()
+        for r in range(rows):
+            lo = max(0, int(n[r]) - window) if window > 0 else 0
+            expect = canonical_order(want[r], int(n[r]) - lo, lo, k)
+            assert got[r].tolist() == expect, (case, r, rows, q_pos0, k, window, kind)
+
+
+def test_indexer_kl_short_and_ragged_sequences(cuda_ok, tiny):
+    """L = 1 (KL 0), L < 8 and L not a multiple of the 8-token blocks."""
+    cfg, x, _ = tiny
+    for L in (1, 5, 13, 100):
+        got = run_kl(x, L, cfg.scale)
+        want = oracle.kl_rows(x["q"][:L], x["k"], x["qI"][:L], x["w"][:L], x["kI"], np.arange(L), cfg.scale)
+        np.testing.assert_allclose(got, want, rtol=KL_RTOL, atol=KL_ATOL, err_msg=f"L={L}")

@@ -565,3 +565,62 @@ def test_indexer_kl_short_and_ragged_sequences(cuda_ok, tiny):
         got = run_kl(x, L, cfg.scale)
         want = oracle.kl_rows(x["q"][:L], x["k"], x["qI"][:L], x["w"][:L], x["kI"], np.arange(L), cfg.scale)
         np.testing.assert_allclose(got, want, rtol=KL_RTOL, atol=KL_ATOL, err_msg=f"L={L}")
+
+
+@pytest.mark.parametrize("HI", [1, 2, 8, 16, 64])
+def test_index_every_head_count(cuda_ok, HI):
+    """Every supported indexer head count (its own kernel instantiation: HI = 64 spans two
+    accumulator chunks per token, HI < 4 has no ReLU pipe split): a ragged slice of a causal
+    sequence against the oracle, within the fp32 bound, nothing written past the diagonal."""
+    rng = np.random.default_rng(18 + HI)
+    q_pos0, Lq, dI = 700, 333, 64
+    Lk = q_pos0 + Lq
+    tqI, tkI, tw = (torch.from_numpy(a.astype(np.float32)).to(torch.bfloat16)
+                    for a in (rng.standard_normal((Lq, HI, dI)), rng.standard_normal((Lk, dI)),
+                              rng.standard_normal((Lq, HI))))
+    qI, kI, w = (t.view(torch.int16).numpy().view(np.uint16) for t in (tqI, tkI, tw))
+    ld = (Lk + 3) // 4 * 4
+    scores = torch.full((Lq, ld), float("nan"), device="cuda")
+    dsa.dsa_index(tqI.cuda(), tkI.cuda(), tw.cuda(), q_pos0, scores)
+    assert dsa.sync_status() == dsa.DSA_OK
+    rows = np.arange(q_pos0, q_pos0 + Lq)
+    ref = oracle.index_rows(qI, w, kI, rows)
+    got = scores.cpu().double().numpy()[:, :Lk]
+    bound = 1e-5 * score_bound(qI, w, kI, rows) + 1e-30
+    for r in range(Lq):
+        n = rows[r] + 1
+        assert np.all(np.abs(got[r, :n] - ref[r, :n]) <= bound[r, :n]), (HI, r)
+        assert np.all(np.isnan(got[r, n:]))
+
+
+def test_decode_sixteen_heads_per_kv_group(cuda_ok):
+    """Decode with Hq = 32 over Hkv = 2 (16 heads per group: two 8-head MMA tiles, with key
+    splits and the merge) and HI = 16, against the oracle on every sequence."""
+    rng = np.random.default_rng(19)
+    B, Lmax, Hq, Hkv, D, HI, dI, topk, scale = 3, 3000, 32, 2, 128, 16, 64, 512, 0.0883883
+    ctx = np.array([10, 700, 2900])
+    f = lambda *sh: torch.from_numpy(rng.standard_normal(sh).astype(np.float32)).to(torch.bfloat16)  # noqa: E731
+    kc, vc, kIc = f(B, Lmax, Hkv, D), f(B, Lmax, Hkv, D), f(B, Lmax, dI)
+    q, qI, w = f(B, Hq, D), f(B, HI, dI), f(B, HI)
+    kn, vn, kIn = f(B, Hkv, D), f(B, Hkv, D), f(B, dI)
+    bits = lambda t: t.view(torch.int16).numpy().view(np.uint16)  # noqa: E731
+    ctx_t = torch.from_numpy(ctx.astype(np.int32)).cuda()
+    kc_d, vc_d, kIc_d = kc.cuda(), vc.cuda(), kIc.cuda()
+    out = torch.empty((B, Hq, D), dtype=torch.bfloat16, device="cuda")
+    idx = torch.empty((B, topk), dtype=torch.int32, device="cuda")
+    dsa.dsa_decode(q.cuda(), qI.cuda(), w.cuda(), kn.cuda(), vn.cuda(), kIn.cuda(), kc_d, vc_d, kIc_d, ctx_t, topk,
+                   scale, out, idx, update_ctx=True)
+    assert dsa.sync_status() == dsa.DSA_OK
+    assert np.array_equal(ctx_t.cpu().numpy(), ctx + 1)
+    got_idx, got_out = idx.cpu().numpy(), bf16_tensor_to_f64(out)
+    for b in range(B):
+        t = int(ctx[b])
+        k_all, v_all, kI_all = bits(kc[b]).copy(), bits(vc[b]).copy(), bits(kIc[b]).copy()
+        k_all[t], v_all[t], kI_all[t] = bits(kn[b]), bits(vn[b]), bits(kIn[b])
+        r = np.array([t])
+        ref = oracle.dsa_rows(bits(q[b:b + 1]), bits(qI[b:b + 1]), bits(w[b:b + 1]), k_all, v_all, kI_all, r, topk,
+                              scale, keep_scores=True)
+        mm = index_set_mismatch(got_idx[b:b + 1], ref["idx"], ref["scores"], ref["tau"], ref["absmax"], r + 1)
+        assert mm["structural"] == 0 and mm["out_of_band"] == 0, (b, mm)
+        own, _ = oracle.sparse_attn_rows(bits(q[b:b + 1]), k_all, v_all, got_idx[b:b + 1], scale)
+        assert_output_ok(got_out[b:b + 1], own, f"decode G=16 b={b}")

@@ -9,21 +9,22 @@
 // Scores are compared through an order-preserving map float -> uint32 ("key"; -0 folded onto
 // +0).  One CTA of 4 warps per row (a cluster of CTAs per row when rows are few and long):
 //   sample   ~n/32 scores at evenly spaced float4s give T0, an estimate of the key at rank
-//            1.5k (two 10-bit histogram rounds over the sample keys);
+//            1.5k (two histogram rounds over the sample keys, bins spanning the samples'
+//            own key range);
 //   stream   the row is read once; each warp takes every 4th 128-byte piece (so frames of
 //            correlated scores spread evenly over the warps) and compacts the scores >= T0 into
-//            its own shared-memory region with warp-level scans -- no block barrier per load;
+//            its own shared-memory region, positions from warp ballots -- no block barrier per load;
 //   refine   if every region fits and the total is >= k, the candidates contain the exact
 //            top-k: radix rounds over the key offsets from T0 (first round scaled to the
-//            candidates' key range) narrow the bin that holds the k-th key until it is small;
-//   emit     keys above that bin are written region by region; the bin's few members are ranked
-//            by (key desc, index asc) and the best ones complete the row.
+//            candidates' key range) narrow the bin that holds the k-th key until it is small, and
+//            that bin's members are ranked once by (key desc, index asc);
+//   emit     the kept keys are written region by region, each region in ascending key order.
 // If the candidates miss the window [k, capacity], the estimate is redone once, aimed using the
-// observed count, and the row streamed again.  Rows that still miss (or where more than 1024
-// keys tie at tau) take an exact radix select over the row itself (10-bit rounds, then one
-// ordered pass): slower, and rare.
-// Output order: keys above the boundary bin region by region (each region ascending), then the
-// boundary bin's kept members by (key desc, index asc).
+// observed count, and the row streamed again.  Rows that still miss (or where more than 512
+// keys tie in the boundary bin) take an exact radix select over the row itself (10-bit rounds,
+// then one ordered pass): slower, and rare.
+// Output order, the same on every path: when every competing key is kept, ascending; otherwise
+// grouped by region ((index / 32) mod 4, the pieces of one warp) and ascending within a region.
 // Sliding window (SW-DSA, page "DSA注意力机制：多模态学习中的强化推理新范式", showapi.com,
 // section 1.4: the selection is restricted to a local window): with window W > 0 only keys
 // s > t - W compete; everything else is unchanged.
@@ -307,7 +308,7 @@ __device__ __forceinline__ uint32_t stream_collect(TopkSmem& S, const float4* ro
 // >= k and includes every key of the row >= lo).  Radix rounds over the key offsets narrow down
 // the bin holding the k-th key until it holds at most kTkSmallBin candidates (or one key value);
 // keys above that bin are all kept, and the bin's members are ranked by (key desc, index asc).
-// Returns false, writing nothing, when more than kTkBins candidates share the last bin.
+// Returns false, writing nothing, when more than kTkBins / 2 candidates share the last bin.
 constexpr int kTkSmallBin = 64;
 constexpr int kTkBatch = 4;  // shared-memory loads batched per thread in the refinement passes
 

@@ -81,14 +81,41 @@ dsa_status launch_status() {
 }
 
 // ------------------------------------------------------------------ device properties
+// The SM count and the kernels' shared-memory limits belong to a device: both are cached per
+// device id, so that a process which moves between devices (cudaSetDevice) between calls still
+// configures each device before its first launch there.
+constexpr int kMaxDevices = 256;
+
+int current_device() {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return -1;
+    return dev;
+}
+
 int num_sms() {
-    static int n = 0;
-    if (n == 0) {
-        int dev = 0;
-        if (cudaGetDevice(&dev) != cudaSuccess) return 0;
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    static std::atomic<int> n[kMaxDevices];
+    const int dev = current_device();
+    if (dev < 0) return 0;
+    int v = n[dev].load(std::memory_order_relaxed);
+    if (v <= 0) {
+        if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) return 0;
+        n[dev].store(v, std::memory_order_relaxed);
     }
-    return n;
+    return v;
+}
+
+// One flag per device: the kernel's dynamic shared-memory limit has been raised there.
+using DeviceFlags = std::atomic<bool>[kMaxDevices];
+
+// Raise `kern`'s dynamic shared-memory limit to `bytes` on the current device, once per device.
+template <typename Kern>
+bool set_smem_limit(Kern* kern, int bytes, DeviceFlags& done) {
+    const int dev = current_device();
+    if (dev < 0) return false;
+    if (done[dev].load(std::memory_order_acquire)) return true;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess) return false;
+    done[dev].store(true, std::memory_order_release);
+    return true;
 }
 
 // ------------------------------------------------------------------ TMA descriptors
@@ -145,12 +172,8 @@ dsa_status launch_indexer_t(const CUtensorMap& mq, const CUtensorMap& mk, const 
                             cudaStream_t s) {
     using C = IndexerCfg<HI, BN, STAGES>;
     auto kern = indexer_kernel<HI, BN, STAGES>;
-    static bool attr_set = false;
-    if (!attr_set) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
-            return DSA_ERR_CUDA;
-        attr_set = true;
-    }
+    static DeviceFlags attr_set;
+    if (!set_smem_limit(kern, C::SMEM, attr_set)) return DSA_ERR_CUDA;
     LaunchScope ls(K_INDEX, s);
     kern<<<grid, C::THREADS, C::SMEM, s>>>(mq, mk, P);
     return launch_status();
@@ -237,13 +260,8 @@ dsa_status run_topk(const float* scores, int64_t ld, int rows, int64_t q_pos0, c
     // Few long rows: a cluster of CTAs per row; otherwise one CTA per row.
     if ((long long)rows * kTkCluster <= 2LL * sms && n_max > 4LL * kTkCap) {
         const int csmem = smem + kTkCap * 8;
-        static bool cattr = false;
-        if (!cattr) {
-            if (cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, csmem) !=
-                cudaSuccess)
-                return DSA_ERR_CUDA;
-            cattr = true;
-        }
+        static DeviceFlags cattr;
+        if (!set_smem_limit(topk_cluster_kernel, csmem, cattr)) return DSA_ERR_CUDA;
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(rows * kTkCluster);
         cfg.blockDim = dim3(kTkThreads);
@@ -260,12 +278,8 @@ dsa_status run_topk(const float* scores, int64_t ld, int rows, int64_t q_pos0, c
         if (cudaLaunchKernelEx(&cfg, topk_cluster_kernel, P) != cudaSuccess) return DSA_ERR_CUDA;
         return launch_status();
     }
-    static bool attr_set = false;
-    if (!attr_set) {
-        if (cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-            return DSA_ERR_CUDA;
-        attr_set = true;
-    }
+    static DeviceFlags attr_set;
+    if (!set_smem_limit(topk_kernel, smem, attr_set)) return DSA_ERR_CUDA;
     LaunchScope ls(K_TOPK, s);
     topk_kernel<<<rows, kTkThreads, smem, s>>>(P);
     return launch_status();
@@ -276,13 +290,9 @@ template <int NT>
 dsa_status launch_attn_t(const AttnParams& P, cudaStream_t s) {
     const int smem = attn_smem_bytes(P.Hkv, NT);
     auto kern = sparse_attn_kernel<NT>;
-    static bool attr_set = false;
-    if (!attr_set) {
-        const int most = std::max(attn_smem_bytes(1, NT), std::max(attn_smem_bytes(2, NT), attn_smem_bytes(4, NT)));
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, most) != cudaSuccess)
-            return DSA_ERR_CUDA;
-        attr_set = true;
-    }
+    static DeviceFlags attr_set;
+    const int most = std::max(attn_smem_bytes(1, NT), std::max(attn_smem_bytes(2, NT), attn_smem_bytes(4, NT)));
+    if (!set_smem_limit(kern, most, attr_set)) return DSA_ERR_CUDA;
     LaunchScope ls(K_ATTN, s);
     kern<<<P.T * P.nsplit, kAttnThreads, smem, s>>>(P);
     return launch_status();
@@ -365,12 +375,12 @@ constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;  // 16 MiB
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 std::mutex g_noalloc_mu;
-void* g_noalloc_addr[256] = {};
+void* g_noalloc_addr[kMaxDevices] = {};
 
 // Device address of g_noalloc_scratch on the current device (looked up on first use).
 dsa_status noalloc_scratch(void** out) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 256) return DSA_ERR_CUDA;
+    const int dev = current_device();
+    if (dev < 0) return DSA_ERR_CUDA;
     std::lock_guard<std::mutex> lk(g_noalloc_mu);
     if (!g_noalloc_addr[dev]) {
         void* p = nullptr;
@@ -508,13 +518,8 @@ dsa_status dsa_indexer_kl(const void* q, const void* k, const void* qI, const vo
     if (C < std::min<int64_t>(L, TB)) return DSA_ERR_WORKSPACE;
     float* scores = static_cast<float*>(ws);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    static bool attr_set = false;
-    if (!attr_set) {
-        if (cudaFuncSetAttribute(indexer_kl_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kl_smem_bytes(4)) !=
-            cudaSuccess)
-            return DSA_ERR_CUDA;
-        attr_set = true;
-    }
+    static DeviceFlags attr_set;
+    if (!set_smem_limit(indexer_kl_kernel, kl_smem_bytes(4), attr_set)) return DSA_ERR_CUDA;
     for (int64_t t0 = 0; t0 < L; t0 += C) {
         const int n = (int)std::min<int64_t>(C, L - t0);
         st = run_indexer(static_cast<const __nv_bfloat16*>(qI) + t0 * HI * dI, kI,

@@ -16,6 +16,8 @@
  *     allocates device memory and never frees caller memory.  Tensors are contiguous,
  *     row-major, with the shapes given, and must be 16-byte aligned.
  *   - bf16 means IEEE bfloat16 stored as uint16; scores are fp32; indices are int32.
+ *   - Every call runs on the calling thread's current CUDA device (cudaSetDevice); its pointers
+ *     and `stream` must belong to that device.  A process may drive several devices in turn.
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL is the legacy default stream).
  *     The return value reports host-side validation and launch errors only.  When it is not
  *     DSA_OK nothing was launched (or, for DSA_ERR_CUDA, a launch failed).

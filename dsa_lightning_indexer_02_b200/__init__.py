@@ -5,13 +5,20 @@ raw device pointers, sizes and the current CUDA stream to the C entry point of t
 All computation runs in the library's CUDA kernels; there is no fallback of any kind: if the
 library is missing this module raises at import time.
 
-Shapes follow the C header:
+Shapes follow the C header (bf16 unless stated; every shape is checked before the call):
   dsa_index(qI [Lq,HI,64], kI [Lk,64], w [Lq,HI], q_pos0, scores fp32 [Lq, ld])
-  dsa_topk(scores fp32 [Lq, ld], q_pos0, k, idx int32 [Lq,k])
-  dsa_sparse_attn(q [Lq,Hq,128], k/v [Lk,Hkv,128], idx [Lq,topk], q_pos0, scale, out, lse=None)
-  dsa_prefill(q, k, v, qI, kI, w, topk, scale, out, idx_out=None, ws=None)
-  dsa_decode(q, qI, w, k_new, v_new, kI_new, k_cache, v_cache, kI_cache, ctx_len, topk, scale,
-             out, idx_out=None, ws=None, update_ctx=False)
+  dsa_topk(scores fp32 [Lq, ld], q_pos0, k, idx int32 [Lq,k], window=0)
+  dsa_sparse_attn(q [Lq,Hq,128], k/v [Lk,Hkv,128], idx int32 [Lq,topk], q_pos0, scale, out [Lq,Hq,128],
+                  lse fp32 [Lq,Hq] = None)
+  dsa_prefill(q [L,Hq,128], k/v [>=L,Hkv,128], qI [L,HI,64], kI [>=L,64], w [L,HI], topk, scale,
+              out [L,Hq,128], idx_out int32 [L,topk] = None, ws=None, window=0)
+  dsa_prefill_rows(q_rows [R,..], k, v, qI_rows [R,..], kI, w_rows [R,HI], row0, topk, scale, out_rows,
+                   idx_rows=None, ws=None, window=0)      (k/v/kI cover rows 0 .. row0+R-1)
+  dsa_indexer_kl(q [L,Hq,128], k [>=L,Hkv,128], qI [L,HI,64], kI [>=L,64], w [L,HI], scale, kl fp32 [>=L])
+  dsa_decode(q [B,Hq,128], qI [B,HI,64], w [B,HI], k_new/v_new [B,Hkv,128], kI_new [B,64],
+             k_cache/v_cache [B,Lmax,Hkv,128], kI_cache [B,Lmax,64], ctx_len int32 [B], topk, scale,
+             out [B,Hq,128], idx_out int32 [B,topk] = None, ws=None, update_ctx=False)
+Every tensor must be contiguous and on the current CUDA device.
 """
 from __future__ import annotations
 
@@ -105,40 +112,77 @@ def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
-def _need(t, dtype, name, ndim=None):
+def _need(t, dtype, name, shape):
+    """One tensor argument: its type, dtype, shape (None: any extent) and contiguity.  The
+    library reads every size from the leading operand, so an operand whose shape disagrees would
+    let a kernel read or write past it: refuse it here."""
     import torch
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name} must be a torch.Tensor")
-    if not t.is_cuda:
-        raise ValueError(f"{name} must be a CUDA tensor")
     if t.dtype != dtype:
         raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.dim() != len(shape) or any(e is not None and int(e) != n for e, n in zip(shape, t.shape)):
+        want = ", ".join("*" if e is None else str(int(e)) for e in shape)
+        raise ValueError(f"{name} must have shape [{want}], got {list(t.shape)}")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
-    if ndim is not None and t.dim() != ndim:
-        raise ValueError(f"{name} must have {ndim} dims, got shape {tuple(t.shape)}")
+
+
+def _at_least(t, name, dim, n):
+    if t.shape[dim] < n:
+        raise ValueError(f"{name}.shape[{dim}] must be >= {n}, got {t.shape[dim]}")
+
+
+def _on_device(**tensors):
+    """Every tensor argument on the current CUDA device (where the library launches)."""
+    import torch
+    ts = {k: t for k, t in tensors.items() if t is not None}
+    for k, t in ts.items():
+        if not t.is_cuda:
+            raise ValueError(f"{k} must be a CUDA tensor")
+    dev = torch.cuda.current_device()
+    for k, t in ts.items():
+        if t.device.index != dev:
+            raise ValueError(f"{k} is on {t.device}, the current device is cuda:{dev}")
+
+
+def _nbytes(t) -> int:
+    return t.numel() * t.element_size()
 
 
 def workspace_size(op: int, L: int, B: int = 1, Hq: int = 32, HI: int = 32, topk: int = 2048) -> int:
     return int(_lib.dsa_workspace_size(op, L, B, Hq, HI, topk))
 
 
-def dsa_index(qI, kI, w, q_pos0: int, scores, stream=None) -> None:
+def _workspace(ws, op, L, B, Hq, HI, topk, like):
     import torch
-    _need(qI, torch.bfloat16, "qI", 3), _need(kI, torch.bfloat16, "kI", 2)
-    _need(w, torch.bfloat16, "w", 2), _need(scores, torch.float32, "scores", 2)
+    if ws is None:
+        return torch.empty(workspace_size(op, L, B, Hq, HI, topk), dtype=torch.uint8, device=like.device)
+    if not isinstance(ws, torch.Tensor) or not ws.is_contiguous():
+        raise ValueError("ws must be a contiguous torch.Tensor")
+    return ws
+
+
+def dsa_index(qI, kI, w, q_pos0: int, scores, stream=None) -> None:
+    """scores[i, s] for the Lq rows of qI (positions q_pos0 + i) and every causal key s."""
+    import torch
+    bf = torch.bfloat16
+    _need(qI, bf, "qI", (None, None, None))
     Lq, HI, dI = qI.shape
+    _need(kI, bf, "kI", (None, dI)), _need(w, bf, "w", (Lq, HI)), _need(scores, torch.float32, "scores", (Lq, None))
+    _on_device(qI=qI, kI=kI, w=w, scores=scores)
     st = _lib.dsa_index(_ptr(qI), _ptr(kI), _ptr(w), Lq, kI.shape[0], HI, dI, q_pos0, _ptr(scores),
                         scores.shape[1], _stream(stream))
     _check(st, "dsa_index")
 
 
 def dsa_topk(scores, q_pos0: int, k: int, idx, window: int = 0, stream=None) -> None:
+    """idx[i] = the top-k keys of score row i (row i holds q_pos0 + i + 1 valid scores)."""
     import torch
-    _need(scores, torch.float32, "scores", 2), _need(idx, torch.int32, "idx", 2)
+    _need(scores, torch.float32, "scores", (None, None))
     Lq = scores.shape[0]
-    if idx.shape != (Lq, k):
-        raise ValueError(f"idx must be [{Lq}, {k}]")
+    _need(idx, torch.int32, "idx", (Lq, k))
+    _on_device(scores=scores, idx=idx)
     if window:
         st = _lib.dsa_topk_window(_ptr(scores), scores.shape[1], Lq, q_pos0, k, window, _ptr(idx), _stream(stream))
         _check(st, "dsa_topk_window")
@@ -148,62 +192,72 @@ def dsa_topk(scores, q_pos0: int, k: int, idx, window: int = 0, stream=None) -> 
 
 
 def dsa_sparse_attn(q, k, v, idx, q_pos0: int, scale: float, out, lse=None, stream=None) -> None:
+    """Attention of the Lq rows of q over the keys that idx selects for each row."""
     import torch
-    _need(q, torch.bfloat16, "q", 3), _need(k, torch.bfloat16, "k", 3), _need(v, torch.bfloat16, "v", 3)
-    _need(idx, torch.int32, "idx", 2), _need(out, torch.bfloat16, "out", 3)
-    if lse is not None:
-        _need(lse, torch.float32, "lse", 2)
+    bf = torch.bfloat16
+    _need(q, bf, "q", (None, None, None))
     Lq, Hq, D = q.shape
-    if out.shape != q.shape or v.shape != k.shape or idx.shape[0] != Lq:
-        raise ValueError("shape mismatch")
+    _need(k, bf, "k", (None, None, D))
+    _need(v, bf, "v", tuple(k.shape)), _need(idx, torch.int32, "idx", (Lq, None)), _need(out, bf, "out", (Lq, Hq, D))
+    if lse is not None:
+        _need(lse, torch.float32, "lse", (Lq, Hq))
+    _on_device(q=q, k=k, v=v, idx=idx, out=out, lse=lse)
     st = _lib.dsa_sparse_attn(_ptr(q), _ptr(k), _ptr(v), _ptr(idx), Lq, k.shape[0], q_pos0, Hq, k.shape[1], D,
                               idx.shape[1], float(scale), _ptr(out), _ptr(lse), _stream(stream))
     _check(st, "dsa_sparse_attn")
 
 
+def _prefill_operands(q, k, v, qI, kI, w, out, idx, topk, key_rows, names):
+    """Shapes shared by the prefill entry points: q/qI/w/out/idx hold the same query rows, k/v/kI
+    at least `key_rows` key rows."""
+    import torch
+    bf = torch.bfloat16
+    nq, nk, nv, nqI, nkI, nw, nout, nidx = names
+    _need(q, bf, nq, (None, None, None))
+    rows, Hq, D = q.shape
+    _need(k, bf, nk, (None, None, D))
+    _at_least(k, nk, 0, key_rows)
+    _need(v, bf, nv, tuple(k.shape)), _need(qI, bf, nqI, (rows, None, None))
+    HI, dI = qI.shape[1], qI.shape[2]
+    _need(kI, bf, nkI, (None, dI))
+    _at_least(kI, nkI, 0, key_rows)
+    _need(w, bf, nw, (rows, HI)), _need(out, bf, nout, (rows, Hq, D))
+    if idx is not None:
+        _need(idx, torch.int32, nidx, (rows, topk))
+    return Hq, D, HI, dI
+
+
 def dsa_prefill(q, k, v, qI, kI, w, topk: int, scale: float, out, idx_out=None, ws=None, window: int = 0,
                 stream=None) -> None:
-    import torch
-    for t, n in ((q, "q"), (k, "k"), (v, "v"), (qI, "qI"), (out, "out")):
-        _need(t, torch.bfloat16, n, 3)
-    _need(kI, torch.bfloat16, "kI", 2), _need(w, torch.bfloat16, "w", 2)
-    L, Hq, D = q.shape
-    HI, dI = qI.shape[1], qI.shape[2]
-    if ws is None:
-        ws = torch.empty(workspace_size(DSA_OP_PREFILL, L, 1, Hq, HI, topk), dtype=torch.uint8, device=q.device)
-    if idx_out is not None:
-        _need(idx_out, torch.int32, "idx_out", 2)
+    """Indexer, top-k and sparse attention for every row of one causal sequence of q.shape[0] tokens."""
+    L = q.shape[0] if hasattr(q, "shape") else 0
+    Hq, D, HI, dI = _prefill_operands(q, k, v, qI, kI, w, out, idx_out, topk, L,
+                                      ("q", "k", "v", "qI", "kI", "w", "out", "idx_out"))
+    _on_device(q=q, k=k, v=v, qI=qI, kI=kI, w=w, out=out, idx_out=idx_out, ws=ws)
+    ws = _workspace(ws, DSA_OP_PREFILL, L, 1, Hq, HI, topk, q)
     if window:
         st = _lib.dsa_prefill_window(_ptr(q), _ptr(k), _ptr(v), _ptr(qI), _ptr(kI), _ptr(w), L, Hq, k.shape[1], D,
                                      HI, dI, topk, window, float(scale), _ptr(out), _ptr(idx_out), _ptr(ws),
-                                     ws.numel() * ws.element_size(), _stream(stream))
+                                     _nbytes(ws), _stream(stream))
         _check(st, "dsa_prefill_window")
         return
     st = _lib.dsa_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(qI), _ptr(kI), _ptr(w), L, Hq, k.shape[1], D, HI, dI,
-                          topk, float(scale), _ptr(out), _ptr(idx_out), _ptr(ws), ws.numel() * ws.element_size(),
-                          _stream(stream))
+                          topk, float(scale), _ptr(out), _ptr(idx_out), _ptr(ws), _nbytes(ws), _stream(stream))
     _check(st, "dsa_prefill")
 
 
 def dsa_prefill_rows(q_rows, k, v, qI_rows, kI, w_rows, row0: int, topk: int, scale: float, out_rows,
                      idx_rows=None, ws=None, window: int = 0, stream=None) -> None:
     """Prefill of query rows row0 .. row0+len(q_rows)-1; k, v, kI cover at least those rows."""
-    import torch
-    for t, n in ((q_rows, "q_rows"), (k, "k"), (v, "v"), (qI_rows, "qI_rows"), (out_rows, "out_rows")):
-        _need(t, torch.bfloat16, n, 3)
-    _need(kI, torch.bfloat16, "kI", 2), _need(w_rows, torch.bfloat16, "w_rows", 2)
-    rows, Hq, D = q_rows.shape
-    HI, dI = qI_rows.shape[1], qI_rows.shape[2]
-    if k.shape[0] < row0 + rows or kI.shape[0] < row0 + rows:
-        raise ValueError("k/v/kI must cover rows up to row0 + rows")
-    if ws is None:
-        ws = torch.empty(workspace_size(DSA_OP_PREFILL, row0 + rows, 1, Hq, HI, topk), dtype=torch.uint8,
-                         device=q_rows.device)
-    if idx_rows is not None:
-        _need(idx_rows, torch.int32, "idx_rows", 2)
+    rows = q_rows.shape[0] if hasattr(q_rows, "shape") else 0
+    Hq, D, HI, dI = _prefill_operands(q_rows, k, v, qI_rows, kI, w_rows, out_rows, idx_rows, topk, row0 + rows,
+                                      ("q_rows", "k", "v", "qI_rows", "kI", "w_rows", "out_rows", "idx_rows"))
+    _on_device(q_rows=q_rows, k=k, v=v, qI_rows=qI_rows, kI=kI, w_rows=w_rows, out_rows=out_rows, idx_rows=idx_rows,
+               ws=ws)
+    ws = _workspace(ws, DSA_OP_PREFILL, row0 + rows, 1, Hq, HI, topk, q_rows)
     st = _lib.dsa_prefill_rows(_ptr(q_rows), _ptr(k), _ptr(v), _ptr(qI_rows), _ptr(kI), _ptr(w_rows), row0, rows, Hq,
                                k.shape[1], D, HI, dI, topk, window, float(scale), _ptr(out_rows), _ptr(idx_rows),
-                               _ptr(ws), ws.numel() * ws.element_size(), _stream(stream))
+                               _ptr(ws), _nbytes(ws), _stream(stream))
     _check(st, "dsa_prefill_rows")
 
 
@@ -211,38 +265,44 @@ def dsa_indexer_kl(q, k, qI, kI, w, scale: float, kl, ws=None, stream=None) -> N
     """Indexer warm-up target KL(P_t || Q_t) for every query row of one causal sequence into kl
     (float32 [L]); see dsa_indexer_kl in include/dsa.h."""
     import torch
-    _need(q, torch.bfloat16, "q", 3), _need(k, torch.bfloat16, "k", 3), _need(qI, torch.bfloat16, "qI", 3)
-    _need(kI, torch.bfloat16, "kI", 2), _need(w, torch.bfloat16, "w", 2), _need(kl, torch.float32, "kl", 1)
+    bf = torch.bfloat16
+    _need(q, bf, "q", (None, None, None))
     L, Hq, D = q.shape
+    _need(k, bf, "k", (None, None, D)), _at_least(k, "k", 0, L), _need(qI, bf, "qI", (L, None, None))
     HI, dI = qI.shape[1], qI.shape[2]
-    if k.shape[0] < L or kI.shape[0] < L or kl.shape[0] < L:
-        raise ValueError("k, kI and kl must cover the L query rows")
-    if ws is None:
-        ws = torch.empty(workspace_size(DSA_OP_INDEXER_KL, L, 1, Hq, HI, 1), dtype=torch.uint8, device=q.device)
+    _need(kI, bf, "kI", (None, dI)), _at_least(kI, "kI", 0, L), _need(w, bf, "w", (L, HI))
+    _need(kl, torch.float32, "kl", (None,)), _at_least(kl, "kl", 0, L)
+    _on_device(q=q, k=k, qI=qI, kI=kI, w=w, kl=kl, ws=ws)
+    ws = _workspace(ws, DSA_OP_INDEXER_KL, L, 1, Hq, HI, 1, q)
     st = _lib.dsa_indexer_kl(_ptr(q), _ptr(k), _ptr(qI), _ptr(kI), _ptr(w), L, Hq, k.shape[1], D, HI, dI,
-                             float(scale), _ptr(kl), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream))
+                             float(scale), _ptr(kl), _ptr(ws), _nbytes(ws), _stream(stream))
     _check(st, "dsa_indexer_kl")
 
 
 def dsa_decode(q, qI, w, k_new, v_new, kI_new, k_cache, v_cache, kI_cache, ctx_len, topk: int, scale: float, out,
                idx_out=None, ws=None, update_ctx: bool = False, stream=None) -> None:
+    """One decode step for B sequences: append the new token at ctx_len[b], then indexer, top-k
+    and sparse attention over positions 0 .. ctx_len[b]."""
     import torch
-    for t, n in ((q, "q"), (qI, "qI"), (k_new, "k_new"), (v_new, "v_new"), (out, "out")):
-        _need(t, torch.bfloat16, n, 3)
-    _need(w, torch.bfloat16, "w", 2), _need(kI_new, torch.bfloat16, "kI_new", 2)
-    _need(k_cache, torch.bfloat16, "k_cache", 4), _need(v_cache, torch.bfloat16, "v_cache", 4)
-    _need(kI_cache, torch.bfloat16, "kI_cache", 3), _need(ctx_len, torch.int32, "ctx_len", 1)
+    bf = torch.bfloat16
+    _need(q, bf, "q", (None, None, None))
     B, Hq, D = q.shape
+    _need(k_cache, bf, "k_cache", (B, None, None, D))
     Lmax, Hkv = k_cache.shape[1], k_cache.shape[2]
+    _need(v_cache, bf, "v_cache", (B, Lmax, Hkv, D)), _need(qI, bf, "qI", (B, None, None))
     HI, dI = qI.shape[1], qI.shape[2]
-    if ws is None:
-        ws = torch.empty(workspace_size(DSA_OP_DECODE, Lmax, B, Hq, HI, topk), dtype=torch.uint8, device=q.device)
+    _need(w, bf, "w", (B, HI)), _need(kI_cache, bf, "kI_cache", (B, Lmax, dI))
+    _need(k_new, bf, "k_new", (B, Hkv, D)), _need(v_new, bf, "v_new", (B, Hkv, D)), _need(kI_new, bf, "kI_new", (B, dI))
+    _need(ctx_len, torch.int32, "ctx_len", (B,)), _need(out, bf, "out", (B, Hq, D))
     if idx_out is not None:
-        _need(idx_out, torch.int32, "idx_out", 2)
+        _need(idx_out, torch.int32, "idx_out", (B, topk))
+    _on_device(q=q, qI=qI, w=w, k_new=k_new, v_new=v_new, kI_new=kI_new, k_cache=k_cache, v_cache=v_cache,
+               kI_cache=kI_cache, ctx_len=ctx_len, out=out, idx_out=idx_out, ws=ws)
+    ws = _workspace(ws, DSA_OP_DECODE, Lmax, B, Hq, HI, topk, q)
     st = _lib.dsa_decode(_ptr(q), _ptr(qI), _ptr(w), _ptr(k_new), _ptr(v_new), _ptr(kI_new), _ptr(k_cache),
                          _ptr(v_cache), _ptr(kI_cache), _ptr(ctx_len), B, Lmax, Hq, Hkv, D, HI, dI, topk,
-                         float(scale), int(bool(update_ctx)), _ptr(out), _ptr(idx_out), _ptr(ws),
-                         ws.numel() * ws.element_size(), _stream(stream))
+                         float(scale), int(bool(update_ctx)), _ptr(out), _ptr(idx_out), _ptr(ws), _nbytes(ws),
+                         _stream(stream))
     _check(st, "dsa_decode")
 
 

@@ -101,3 +101,74 @@ def test_torch_binding_rejects_cpu_tensors():
     with pytest.raises(ValueError):
         dsa.dsa_index(x, torch.zeros(4, 64, dtype=torch.bfloat16), torch.zeros(4, 32, dtype=torch.bfloat16), 0,
                       torch.zeros(4, 4))
+
+
+def _bf(*shape):
+    import torch
+    return torch.zeros(shape, dtype=torch.bfloat16)
+
+
+def _i32(*shape):
+    import torch
+    return torch.zeros(shape, dtype=torch.int32)
+
+
+def _f32(*shape):
+    import torch
+    return torch.zeros(shape, dtype=torch.float32)
+
+
+def _prefill_args(L=16, Hq=8, Hkv=2, D=128, HI=4, dI=64, k=8):
+    return dict(q=_bf(L, Hq, D), k=_bf(L, Hkv, D), v=_bf(L, Hkv, D), qI=_bf(L, HI, dI), kI=_bf(L, dI),
+                w=_bf(L, HI), topk=k, scale=0.1, out=_bf(L, Hq, D), idx_out=_i32(L, k))
+
+
+def _decode_args(B=2, Lmax=32, Hq=8, Hkv=2, D=128, HI=16, dI=64, k=8):
+    return dict(q=_bf(B, Hq, D), qI=_bf(B, HI, dI), w=_bf(B, HI), k_new=_bf(B, Hkv, D), v_new=_bf(B, Hkv, D),
+                kI_new=_bf(B, dI), k_cache=_bf(B, Lmax, Hkv, D), v_cache=_bf(B, Lmax, Hkv, D),
+                kI_cache=_bf(B, Lmax, dI), ctx_len=_i32(B), topk=k, scale=0.1, out=_bf(B, Hq, D),
+                idx_out=_i32(B, k))
+
+
+# (entry point, consistent arguments, {operand: a wrong-shaped replacement})
+_SHAPE_CASES = [
+    (dsa.dsa_index, dict(qI=_bf(8, 4, 64), kI=_bf(8, 64), w=_bf(8, 4), q_pos0=0, scores=_f32(8, 8)),
+     {"kI": _bf(8, 32), "w": _bf(8, 5), "scores": _f32(7, 8)}),
+    (dsa.dsa_topk, dict(scores=_f32(8, 8), q_pos0=0, k=4, idx=_i32(8, 4)),
+     {"idx": _i32(8, 5)}),
+    (dsa.dsa_sparse_attn, dict(q=_bf(8, 8, 128), k=_bf(8, 2, 128), v=_bf(8, 2, 128), idx=_i32(8, 4), q_pos0=0,
+                               scale=0.1, out=_bf(8, 8, 128), lse=_f32(8, 8)),
+     {"k": _bf(8, 2, 64), "v": _bf(9, 2, 128), "idx": _i32(7, 4), "out": _bf(8, 4, 128), "lse": _f32(8, 4)}),
+    (dsa.dsa_prefill, _prefill_args(),
+     {"k": _bf(15, 2, 128), "v": _bf(16, 1, 128), "qI": _bf(15, 4, 64), "kI": _bf(16, 32), "w": _bf(16, 3),
+      "out": _bf(16, 8, 64), "idx_out": _i32(16, 9)}),
+    (dsa.dsa_indexer_kl, dict(q=_bf(16, 8, 128), k=_bf(16, 2, 128), qI=_bf(16, 4, 64), kI=_bf(16, 64),
+                              w=_bf(16, 4), scale=0.1, kl=_f32(16)),
+     {"k": _bf(15, 2, 128), "qI": _bf(15, 4, 64), "kI": _bf(15, 64), "w": _bf(16, 8), "kl": _f32(15)}),
+    (dsa.dsa_decode, _decode_args(),
+     {"qI": _bf(3, 16, 64), "w": _bf(2, 8), "k_new": _bf(2, 1, 128), "v_new": _bf(2, 2, 64), "kI_new": _bf(2, 32),
+      "k_cache": _bf(2, 32, 2, 64), "v_cache": _bf(2, 31, 2, 128), "kI_cache": _bf(2, 32, 32), "ctx_len": _i32(3),
+      "out": _bf(2, 8, 64), "idx_out": _i32(2, 7)}),
+]
+
+
+@pytest.mark.parametrize("fn,args,bad", _SHAPE_CASES, ids=[c[0].__name__ for c in _SHAPE_CASES])
+def test_binding_checks_every_operand_shape(fn, args, bad):
+    """A consistent call gets past the shape checks (and stops at the CPU-tensor check); each
+    operand whose shape disagrees with the leading one is refused by name before any pointer is
+    passed on."""
+    with pytest.raises(ValueError, match="must be a CUDA tensor"):
+        fn(**args)
+    for name, wrong in bad.items():
+        with pytest.raises(ValueError, match=f"^{name}"):
+            fn(**{**args, name: wrong})
+
+
+def test_binding_prefill_rows_needs_keys_up_to_its_last_row():
+    a = _prefill_args()
+    rows = dict(q_rows=a["q"][:8], k=a["k"], v=a["v"], qI_rows=a["qI"][:8], kI=a["kI"], w_rows=a["w"][:8],
+                topk=8, scale=0.1, out_rows=a["out"][:8], idx_rows=a["idx_out"][:8])
+    with pytest.raises(ValueError, match="must be a CUDA tensor"):
+        dsa.dsa_prefill_rows(row0=8, **rows)
+    with pytest.raises(ValueError, match=r"^k\.shape\[0\] must be >= 17"):
+        dsa.dsa_prefill_rows(row0=9, **rows)

@@ -123,19 +123,21 @@ def cpu_baseline(cfg, x, budget_s: float = 15.0, seed: int = 7) -> dict:
     import oracle
     cores = oracle.threads()
     # one probe batch to size the sample so the whole leg takes about budget_s
-    rows = np.sort(synth.sample_rows(max(2, cores), cfg.L, seed=seed, key=0xC0DE))
+    probe_rows = np.sort(synth.sample_rows(max(2, cores), cfg.L, seed=seed, key=0xC0DE))
     t0 = time.perf_counter()
-    oracle.dsa_rows(x["q"][rows], x["qI"][rows], x["w"][rows], x["k"], x["v"], x["kI"], rows, cfg.k, cfg.scale)
+    oracle.dsa_rows(x["q"][probe_rows], x["qI"][probe_rows], x["w"][probe_rows], x["k"], x["v"], x["kI"], probe_rows,
+                    cfg.k, cfg.scale)
     probe = time.perf_counter() - t0
-    n = int(max(cores, min(4096, len(rows) * max(1.0, (budget_s - probe) / max(probe, 1e-3)))))
+    n = int(max(cores, min(4096, len(probe_rows) * max(1.0, (budget_s - probe) / max(probe, 1e-3)))))
     rows = np.sort(synth.sample_rows(n, cfg.L, seed=seed + 1, key=0xC0DE))
     t0 = time.perf_counter()
     oracle.dsa_rows(x["q"][rows], x["qI"][rows], x["w"][rows], x["k"], x["v"], x["kI"], rows, cfg.k, cfg.scale)
     el = time.perf_counter() - t0
     return {"value": n / el, "unit": UNIT, "cores": cores, "kind": "oracle",
             "sample": f"{n} query rows drawn uniformly from the {cfg.L}-token prefill (full path per row: "
-                      f"indexer over t+1 keys, sort-based top-{cfg.k}, attention), {el:.1f} s; "
-                      f"unbiased for tokens/s since rows are uniform in t"}
+                      f"indexer over t+1 keys, sort-based top-{cfg.k}, attention), {el:.1f} s after a "
+                      f"{probe:.1f} s sizing probe of {len(probe_rows)} rows; unbiased for tokens/s since rows "
+                      f"are uniform in t"}
 
 
 # ----------------------------------------------------------------------------- reference arm
@@ -189,7 +191,7 @@ def main():
                     help="query rows of the 32K workload for the KL measurement (default: all 32768)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
-    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--cpu-seconds", type=float, default=20.0)
     ap.add_argument("--chunk-rows", type=int, default=0,
                     help="limit the prefill workspace to this many score rows (small profiling cases)")
     args = ap.parse_args()

@@ -184,6 +184,8 @@ def main():
     ap.add_argument("--decode-steps", type=int, default=256)
     ap.add_argument("--decode-ctx", type=int, default=0, help="override the cached context (small profiling cases)")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--decode-only", action="store_true",
+                    help="measure only the decode step and print its object (profiling cases)")
     ap.add_argument("--no-kl", action="store_true", help="skip the indexer warm-up KL measurement")
     ap.add_argument("--kl-only", action="store_true",
                     help="measure only the indexer warm-up KL and print its object (profiling cases)")
@@ -226,6 +228,12 @@ def main():
         kl = run_kl(torch, dsa, synth.CONFIGS["32k"], barrier, max_over_ranks, peaks, rows=args.kl_rows)
         if rank == 0:
             print(json.dumps({"indexer_kl": kl}), flush=True)
+        return 0
+    if args.decode_only:
+        decode = run_decode(torch, dsa, decode_config(args), args.decode_steps, rank, world, barrier,
+                            max_over_ranks, peaks)
+        if rank == 0:
+            print(json.dumps({"decode": decode}), flush=True)
         return 0
     cfg = synth.CONFIGS[args.workload]
     x = synth.inputs(cfg, 0, cfg.L, seq=rank)
@@ -381,11 +389,8 @@ def main():
     # ---- decode: 16 sequences x 131072 cached tokens, 256 steps
     decode = None
     if not args.no_decode:
-        dcfg = synth.CONFIGS["decode"]
-        if args.decode_ctx:
-            import dataclasses
-            dcfg = dataclasses.replace(dcfg, L=args.decode_ctx, iid_from=args.decode_ctx)
-        decode = run_decode(torch, dsa, dcfg, args.decode_steps, rank, world, barrier, max_over_ranks, peaks)
+        decode = run_decode(torch, dsa, decode_config(args), args.decode_steps, rank, world, barrier,
+                            max_over_ranks, peaks)
 
     # ---- indexer warm-up KL target on the 32K workload (dense, tensor-core bound)
     kl = None
@@ -474,6 +479,15 @@ def run_kl(torch, dsa, cfg, barrier, max_over_ranks, peaks, reps: int = 3, rows:
                          "unit": "TFLOP/s", "frac": achieved / tpeak,
                          "algorithmic": "4 x Hq x D flop per causal (t, s) pair (two passes of Q.K)"},
             "mean_kl": float(kl.mean()), "mma": "warp-level m16n8k16 (mma.sync)"}
+
+
+def decode_config(args):
+    """The decode workload (16 sequences x 131072 cached tokens), or a shorter cached context."""
+    dcfg = synth.CONFIGS["decode"]
+    if args.decode_ctx:
+        import dataclasses
+        dcfg = dataclasses.replace(dcfg, L=args.decode_ctx, iid_from=args.decode_ctx)
+    return dcfg
 
 
 def run_decode(torch, dsa, cfg, steps, rank, world, barrier, max_over_ranks, peaks):

@@ -68,6 +68,13 @@ def prefill_work(cfg) -> dict:
     }
 
 
+def decode_step_bytes(cfg, ctx_mean: float) -> float:
+    """Algorithmic bytes of one decode step for cfg.batch sequences whose keys number ctx_mean on
+    average: the kI stream (2*dI bytes per key), the fp32 score row written and read back, the
+    K/V gather (k keys x Hkv x D x K and V x 2 bytes) and the idx row written and read back."""
+    return cfg.batch * (ctx_mean * cfg.dI * 2 + 2 * 4 * ctx_mean + cfg.k * cfg.Hkv * cfg.D * 2 * 2 + 2 * 4 * cfg.k)
+
+
 # ----------------------------------------------------------------------------- clocks
 class ClockSampler:
     def __init__(self, device_index: int):
@@ -553,9 +560,7 @@ def run_decode(torch, dsa, cfg, steps, rank, world, barrier, max_over_ranks, pea
     prof = dsa.profile_end()
     dcount = dsa.read_counters(reset=True)
     kmeans = {k: v["ms"] / steps for k, v in prof.items() if v["launches"]}
-    # algorithmic bytes per step: kI stream + score write/read + K/V gather + idx
-    ctx_mean = ctx0 + (steps - 1) / 2
-    bytes_step = B * (ctx_mean * cfg.dI * 2 + 2 * 4 * ctx_mean + cfg.k * cfg.Hkv * cfg.D * 2 * 2 + 2 * 4 * cfg.k)
+    bytes_step = decode_step_bytes(cfg, ctx0 + (steps - 1) / 2)
     return {"value": world * B * steps / (ms / 1e3), "unit": UNIT, "steps": steps, "batch": B, "ctx": ctx0,
             "ms_per_decode_step": ms / steps, "timing": "one CUDA graph of all steps, CUDA events around it",
             "kernel_ms_per_step": kmeans,

@@ -172,3 +172,34 @@ def test_binding_prefill_rows_needs_keys_up_to_its_last_row():
         dsa.dsa_prefill_rows(row0=8, **rows)
     with pytest.raises(ValueError, match=r"^k\.shape\[0\] must be >= 17"):
         dsa.dsa_prefill_rows(row0=9, **rows)
+
+
+def _c_kind(decl: str) -> str:
+    """Coarse ctypes kind of one C parameter or return type from include/dsa.h."""
+    d = " ".join(decl.replace("const", " ").split())
+    if "*" in d or d.startswith("dsa_stream_t"):
+        return "ptr"
+    base = d.split()[0]
+    return {"int": "int", "int64_t": "i64", "size_t": "size", "float": "float", "double": "double",
+            "dsa_status": "int", "void": "void"}[base]
+
+
+_CTYPES_KIND = {ctypes.c_void_p: "ptr", ctypes.c_char_p: "ptr", ctypes.c_int: "int", ctypes.c_int64: "i64",
+                ctypes.c_size_t: "size", ctypes.c_float: "float", ctypes.c_double: "double", None: "void"}
+
+
+def test_binding_signatures_match_the_header():
+    """Every prototype in include/dsa.h and the binding's ctypes signature of the same name agree
+    in return kind, argument count and each argument's kind (a pointer passed where the header
+    expects a size, or a dropped argument, would reach a kernel as a bad address)."""
+    import re
+    with open(dsa.HEADER_PATH) as f:
+        text = re.sub(r"/\*.*?\*/", "", f.read(), flags=re.S)
+    decls = re.findall(r"([A-Za-z_][\w \*]*?)\b(dsa_[a-z_]+)\s*\(([^)]*)\)\s*;", text)
+    assert len(decls) == len(dsa.header_symbols())
+    for ret, name, params in decls:
+        params = params.strip()
+        kinds = [] if params in ("", "void") else [_c_kind(p) for p in params.split(",")]
+        res, args = dsa._SIGS[name]
+        assert _CTYPES_KIND[res] == _c_kind(ret.strip()), name
+        assert [_CTYPES_KIND[a] for a in args] == kinds, name

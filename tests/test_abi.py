@@ -203,3 +203,35 @@ def test_binding_signatures_match_the_header():
         res, args = dsa._SIGS[name]
         assert _CTYPES_KIND[res] == _c_kind(ret.strip()), name
         assert [_CTYPES_KIND[a] for a in args] == kinds, name
+
+
+def test_host_validation_of_window_rows_and_noalloc_entry_points():
+    """The variants of prefill, top-k and decode refuse bad sizes, windows and workspaces on the
+    host, before any CUDA call."""
+    A = fake(0x10000)
+    f = 0.1
+    # top-k with a window: negative window, k = 0, rows past ld
+    assert lib.dsa_topk_window(A, 8, 8, 0, 4, -1, A, None) == dsa.DSA_ERR_INVALID_ARG
+    assert lib.dsa_topk_window(A, 8, 8, 0, 0, 16, A, None) == dsa.DSA_ERR_INVALID_ARG
+    assert lib.dsa_topk_window(A, 8, 8, 4, 4, 16, A, None) == dsa.DSA_ERR_INVALID_ARG
+    assert lib.dsa_topk_window(A, 8, 8, 0, 1 << 20, 16, A, None) == dsa.DSA_ERR_UNSUPPORTED
+    # prefill of a row range: empty range, negative row0 or window, missing workspace
+    shape = [32, 4, 128, 32, 64, 2048]                     # Hq, Hkv, D, HI, dI, topk
+    def rows(row0, n, window, ws=A, ws_bytes=1 << 40):
+        return lib.dsa_prefill_rows(*[A] * 6, row0, n, *shape, window, f, A, None, ws, ws_bytes, None)
+    assert rows(0, 0, 0) == dsa.DSA_ERR_INVALID_ARG
+    assert rows(-1, 8, 0) == dsa.DSA_ERR_INVALID_ARG
+    assert rows(0, 8, -5) == dsa.DSA_ERR_INVALID_ARG
+    assert rows(0, 8, 0, ws=None, ws_bytes=0) == dsa.DSA_ERR_WORKSPACE
+    assert rows(0, 4096, 0, ws_bytes=1024) == dsa.DSA_ERR_WORKSPACE
+    # windowed prefill: empty sequence, and the shape checks it shares with prefill
+    assert lib.dsa_prefill_window(*[A] * 6, 0, *shape, 100, f, A, None, A, 1 << 30, None) == dsa.DSA_ERR_INVALID_ARG
+    assert lib.dsa_prefill_window(*[A] * 6, 1024, 32, 4, 64, 32, 64, 2048, 100, f, A, None, A, 1 << 30, None) == \
+        dsa.DSA_ERR_UNSUPPORTED
+    # allocation-free decode: bad batch, and a step too large for its fixed scratch
+    dargs = [A] * 10
+    assert lib.dsa_decode_noalloc(*dargs, 0, 4096, 32, 4, 128, 32, 64, 2048, f, 0, A, None, None) == \
+        dsa.DSA_ERR_INVALID_ARG
+    assert lib.dsa_decode_noalloc(*dargs, 256, 1 << 22, 32, 4, 128, 32, 64, 2048, f, 0, A, None, None) == \
+        dsa.DSA_ERR_WORKSPACE
+    assert lib.dsa_launch_count() == 0

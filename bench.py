@@ -162,7 +162,7 @@ def run_reference(args):
     cfg = synth.CONFIGS[args.workload]
     x = synth.inputs(cfg, 0, cfg.L)
     vals = []
-    budget = max(5.0, 120.0 / max(1, args.steps + args.warmup))
+    budget = args.ref_seconds if args.ref_seconds else max(5.0, 120.0 / max(1, args.steps + args.warmup))
     cb = None
     for i in range(args.warmup + args.steps):
         cb = cpu_baseline(cfg, x, budget_s=budget, seed=11 + i)
@@ -201,6 +201,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
+    ap.add_argument("--ref-seconds", type=float, default=0.0,
+                    help="oracle seconds per reference-arm step (default: about 2 minutes per run)")
     ap.add_argument("--chunk-rows", type=int, default=0,
                     help="limit the prefill workspace to this many score rows (small profiling cases)")
     args = ap.parse_args()

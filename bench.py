@@ -56,15 +56,23 @@ def selected_keys(L: int, k: int) -> int:
     return m * (m + 1) // 2 + max(0, L - k) * k
 
 
-def prefill_work(cfg) -> dict:
-    """Algorithmic work of one prefill step (per kernel kind)."""
-    caus = causal_keys(0, cfg.L)
-    sel = selected_keys(cfg.L, cfg.k)
+def selected_keys_range(lo: int, hi: int, k: int) -> int:
+    """sum_{t=lo}^{hi-1} min(k, t+1)"""
+    return selected_keys(hi, k) - selected_keys(lo, k)
+
+
+def prefill_work(cfg, lo: int = 0, hi: int | None = None) -> dict:
+    """Algorithmic work of query rows [lo, hi) of one prefill (default: the whole sequence),
+    per kernel kind."""
+    hi = cfg.L if hi is None else hi
+    n = hi - lo
+    caus = causal_keys(lo, n)
+    sel = selected_keys_range(lo, hi, cfg.k)
     return {
         "indexer_flop": 2 * cfg.HI * cfg.dI * caus,
-        "topk_bytes": 4 * caus + 4 * cfg.k * cfg.L,
+        "topk_bytes": 4 * caus + 4 * cfg.k * n,
         "attn_gather_bytes": sel * cfg.Hkv * cfg.D * 2 * 2,
-        "attn_io_bytes": cfg.L * cfg.Hq * cfg.D * 2 * 2 + 4 * cfg.k * cfg.L,
+        "attn_io_bytes": n * cfg.Hq * cfg.D * 2 * 2 + 4 * cfg.k * n,
     }
 
 
@@ -148,10 +156,15 @@ def cpu_baseline(cfg, x, budget_s: float = 15.0, seed: int = 7) -> dict:
 
 
 # ----------------------------------------------------------------------------- reference arm
-def bench_config(cfg, workload: str, world: int) -> dict:
+def bench_config(cfg, workload: str, world: int, split: str = "seq") -> dict:
     """The `config` object of the JSON line, identical for both arms."""
+    if split == "rows":
+        par = (f"rows{world} (one sequence; causal-work-balanced query-row ranges per rank, K/V/kI "
+               "replicated; output rows assembled on every rank by one broadcast per range)")
+    else:
+        par = f"dp{world} (independent sequences)"
     return {"workload": f"prefill_{workload}", "L": cfg.L, "k": cfg.k, "Hq": cfg.Hq, "Hkv": cfg.Hkv, "D": cfg.D,
-            "HI": cfg.HI, "dI": cfg.dI, "batch": 1, "parallelism": f"dp{world} (independent sequences)",
+            "HI": cfg.HI, "dI": cfg.dI, "batch": 1, "parallelism": par,
             "l2": "inputs (1.8 GB) larger than L2; no flush"}
 
 
@@ -205,6 +218,12 @@ def main():
                     help="oracle seconds per reference-arm step (default: about 2 minutes per run)")
     ap.add_argument("--chunk-rows", type=int, default=0,
                     help="limit the prefill workspace to this many score rows (small profiling cases)")
+    ap.add_argument("--split", default="seq", choices=["seq", "rows"],
+                    help="under torchrun: seq = one independent sequence per rank (weak scaling); rows = one "
+                         "sequence whose query rows are split over the ranks (strong scaling)")
+    ap.add_argument("--profile-rows", default="",
+                    help="R0:N -- run only query rows R0..R0+N-1 of the workload through dsa_prefill_rows, "
+                         "once untimed and once more (a small case for ncu captures); prints its work units")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
@@ -213,7 +232,8 @@ def main():
     import torch.distributed as dist
 
     import dsa_lightning_indexer_02_b200 as dsa
-    from dsa_lightning_indexer_02_b200.sharding import reduce_max, weak_scaling_value
+    from dsa_lightning_indexer_02_b200.sharding import (assemble_row_ranges, causal_balanced_row_ranges, reduce_max,
+                                                        weak_scaling_value)
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -245,20 +265,33 @@ def main():
             print(json.dumps({"decode": decode}), flush=True)
         return 0
     cfg = synth.CONFIGS[args.workload]
-    x = synth.inputs(cfg, 0, cfg.L, seq=rank)
+    if args.profile_rows:
+        return run_profile_case(torch, dsa, cfg, args.profile_rows)
+    rows_mode = args.split == "rows"
+    # split=seq: each rank prefills its own independent sequence (seq = rank); split=rows: every
+    # rank holds the same sequence and prefills its causal-work-balanced range of query rows
+    x = synth.inputs(cfg, 0, cfg.L, seq=0 if rows_mode else rank)
+    ranges = causal_balanced_row_ranges(cfg.L, world, k=cfg.k, align=256 // cfg.HI) if rows_mode else None
+    lo, hi = ranges[rank] if rows_mode else (0, cfg.L)
     names = ("q", "k", "v", "qI", "kI", "w")
     host = {n: synth.to_torch(x[n]).pin_memory() for n in names}
     d = {n: host[n].cuda() for n in names}
     out = torch.empty((cfg.L, cfg.Hq, cfg.D), dtype=torch.bfloat16, device="cuda")
     idx = torch.empty((cfg.L, cfg.k), dtype=torch.int32, device="cuda")
-    ws_bytes = dsa.workspace_size(dsa.DSA_OP_PREFILL, cfg.L, 1, cfg.Hq, cfg.HI, cfg.k)
+    ws_bytes = dsa.workspace_size(dsa.DSA_OP_PREFILL, hi, 1, cfg.Hq, cfg.HI, cfg.k)
     if args.chunk_rows:
         ws_bytes = args.chunk_rows * ((cfg.L + 3) // 4 * 4) * 4 + 4096
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
     stream = torch.cuda.current_stream()
 
     def step():
-        dsa.dsa_prefill(d["q"], d["k"], d["v"], d["qI"], d["kI"], d["w"], cfg.k, cfg.scale, out, idx, ws)
+        if rows_mode:
+            if hi > lo:
+                dsa.dsa_prefill_rows(d["q"][lo:hi], d["k"][:hi], d["v"][:hi], d["qI"][lo:hi], d["kI"][:hi],
+                                     d["w"][lo:hi], lo, cfg.k, cfg.scale, out[lo:hi], idx[lo:hi], ws=ws)
+            assemble_row_ranges((out, idx), ranges, dist if world > 1 else None)
+        else:
+            dsa.dsa_prefill(d["q"], d["k"], d["v"], d["qI"], d["kI"], d["w"], cfg.k, cfg.scale, out, idx, ws)
 
     for _ in range(max(3, args.warmup)):
         step()
@@ -285,60 +318,22 @@ def main():
     if dsa.sync_status() != dsa.DSA_OK:
         raise SystemExit("device error during the timed region")
     ms_step = max_over_ranks(ev0.elapsed_time(ev1) / args.steps)
-    value = weak_scaling_value(cfg.L, world, ms_step / 1000.0)
+    value = (cfg.L if rows_mode else weak_scaling_value(cfg.L, world, 1.0)) / (ms_step / 1000.0)
     union16 = adjacent_union_stat(idx, cfg, torch)
     clk = clocks.summary()
 
-    # ---- per-kernel roofline (event-timed launches inside the timed region)
-    work = prefill_work(cfg)
-    hbm = peaks["hbm_gbs"]
-    tfl = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
-    kern = {}
-
-    def per_launch(kind):
-        p = prof[kind]
-        return p["ms"] / max(1, p["launches"]), p["launches"] / args.steps
-
-    ms_i, n_i = per_launch("indexer")
-    ms_t, n_t = per_launch("topk")
-    ms_a, n_a = per_launch("sparse_attn")
-    # algorithmic units per launch = per-step work / launches per step (chunks are equal-sized
-    # except for causal growth; the step totals are exact, per-launch figures are their mean)
-    fl_i = work["indexer_flop"] / n_i
-    kern["indexer"] = {"bound": "tensor", "achieved": fl_i / (ms_i / 1e3) / 1e12, "peak": tfl, "unit": "TFLOP/s",
-                       "ms_per_launch": ms_i, "launches_per_step": n_i}
-    by_t = work["topk_bytes"] / n_t
-    kern["topk"] = {"bound": "hbm", "achieved": by_t / (ms_t / 1e3) / 1e9, "peak": hbm, "unit": "GB/s",
-                    "ms_per_launch": ms_t, "launches_per_step": n_t}
-    by_a = (work["attn_gather_bytes"] + work["attn_io_bytes"]) / n_a
-    kern["sparse_attn"] = {"bound": "hbm", "achieved": by_a / (ms_a / 1e3) / 1e9, "peak": hbm, "unit": "GB/s",
-                           "ms_per_launch": ms_a, "launches_per_step": n_a,
-                           "note": "logical gathered K/V bytes + q/out/idx; L2 reuse can push it past HBM peak"}
-    for v in kern.values():
-        v["frac"] = v["achieved"] / v["peak"]
+    # ---- per-kernel roofline (event-timed launches inside the timed region, this rank's rows)
+    work = prefill_work(cfg, lo, hi)
+    kern = kernel_rooflines(prof, work, args.steps, peaks, args.workload, cfg)
+    for kv in kern.values():
+        kv["peak_source"] = f"{peak_src}: {kv['peak_source']}"
     dominant = max(kern, key=lambda kk: kern[kk]["ms_per_launch"] * kern[kk]["launches_per_step"])
-    # measured DRAM bytes per launch (ncu, committed under profiles/) while the sources still match
-    tr = {}
-    tpath = os.path.join(ROOT, "profiles", "traffic.json")
-    if os.path.exists(tpath):
-        with open(tpath) as f:
-            tr = json.load(f)
-    sha = lib_hash()
-    for name, kd in kern.items():
-        ent = tr.get(name)
-        kd["traffic"] = None
-        if ent and ent.get("lib_sha") == sha and ent.get("workload") == args.workload:
-            kd["traffic"] = ent["bytes_per_launch"]
-            # DRAM bandwidth actually drawn: measured bytes / this run's launch time
-            kd["dram_gbs"] = kd["traffic"] / (kd["ms_per_launch"] / 1e3) / 1e9
     kd = kern[dominant]
     roofline = {"bound": kd["bound"], "achieved": kd["achieved"], "peak": kd["peak"], "unit": kd["unit"],
-                "frac": kd["frac"], "traffic": kd["traffic"], "kernel": dominant,
-                "peak_source": f"{peak_src} ({'sustained bf16' if kd['bound'] == 'tensor' else 'HBM copy'})"}
-    if dominant == "sparse_attn":
-        roofline["note"] = ("achieved counts the logical gathered K/V bytes (the algorithmic unit); most "
-                            "gathered rows hit L2, so it exceeds the HBM copy rate; traffic is the DRAM "
-                            "bytes one launch really moves")
+                "frac": kd["frac"], "traffic": kd["traffic"], "kernel": dominant, "peak_source": kd["peak_source"]}
+    for extra in ("achieved_logical", "logical_frac", "traffic_scaled_from", "frac_sustained", "note"):
+        if extra in kd:
+            roofline[extra] = kd[extra]
 
     # ---- end to end through host buffers and the public row-range call: per block of rows, the
     # host->device copy of its inputs (and of the keys it adds), dsa_prefill_rows, and the
@@ -347,10 +342,13 @@ def main():
     if not args.no_e2e:
         hout = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
         hidx = torch.empty(idx.shape, dtype=idx.dtype, pin_memory=True)
-        h2d = sum(host[n].numel() * host[n].element_size() for n in names)
-        d2h = hout.numel() * 2 + hidx.numel() * 4
         R = 8192
-        blocks = [(r, min(cfg.L, r + R)) for r in range(0, cfg.L, R)]
+        blocks = [(r, min(hi, r + R)) for r in range(lo, hi, R)]
+        row_bytes = {n: host[n][0].numel() * host[n].element_size() for n in names}
+        # this rank's query rows of q/qI/w, and K/V/kI of every position up to its last row
+        h2d = sum(row_bytes[n] * (hi - lo) for n in ("q", "qI", "w")) + \
+            sum(row_bytes[n] * hi for n in ("k", "v", "kI"))
+        d2h = (hi - lo) * (out[0].numel() * 2 + idx[0].numel() * 4)
         s_in, s_cmp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
         # score rows of one block at the longest row length, plus alignment slack
         ws_rows = torch.empty(R * ((cfg.L + 3) // 4 * 4) * 4 + 4096, dtype=torch.uint8, device="cuda")
@@ -359,6 +357,10 @@ def main():
             ev_in = [torch.cuda.Event() for _ in blocks]
             ev_c = [torch.cuda.Event() for _ in blocks]
             s_in.wait_stream(stream)
+            if lo > 0:                       # the key prefix that rows before this rank's range hold
+                with torch.cuda.stream(s_in):
+                    for n in ("k", "v", "kI"):
+                        d[n][:lo].copy_(host[n][:lo], non_blocking=True)
             for i, (r0, r1) in enumerate(blocks):
                 with torch.cuda.stream(s_in):
                     for n in names:
@@ -387,10 +389,12 @@ def main():
         if dsa.sync_status() != dsa.DSA_OK:
             raise SystemExit("device error in the end-to-end leg")
         ms_e2e = max_over_ranks(ev0.elapsed_time(ev1) / args.steps)
-        e2e = {"value": weak_scaling_value(cfg.L, world, ms_e2e / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
-               "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e,
-               "how": f"dsa_prefill_rows over {len(blocks)} blocks of {R} rows; H2D, compute and D2H on three "
-                      "streams, pinned host buffers"}
+        e2e = {"value": (cfg.L if rows_mode else weak_scaling_value(cfg.L, world, 1.0)) / (ms_e2e / 1e3),
+               "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e,
+               "how": f"dsa_prefill_rows over {len(blocks)} blocks of up to {R} rows; H2D, compute and D2H on "
+                      "three streams, pinned host buffers" +
+                      ("; each rank copies in its own query rows and the key prefix they need, and copies "
+                       "out its own output rows" if rows_mode else "")}
 
     del d, host, out, idx, ws
     torch.cuda.empty_cache()
@@ -411,10 +415,10 @@ def main():
         cpu = cpu_baseline(cfg, x, budget_s=args.cpu_seconds)
 
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-            "warmup": max(3, args.warmup), "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16",
+            "warmup": max(3, args.warmup), "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "strong" if rows_mode else "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded; 512 frame + 64 text token layout, block-structured keys)",
-            "config": bench_config(cfg, args.workload, world),
+            "config": bench_config(cfg, args.workload, world, args.split),
             "roofline": roofline, "kernels": kern, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
             "clocks": clk, "decode": decode, "indexer_kl": kl, "adjacent_union_16": union16,
             "path_counters": counters}
@@ -435,6 +439,105 @@ def adjacent_union_stat(idx, cfg, torch, windows: int = 32) -> dict:
         rows = idx[int(t0):int(t0) + 16].cpu().numpy()
         sizes.append(len(np.unique(rows[rows >= 0])))
     return {"mean_unique": float(np.mean(sizes)), "naive": 16 * cfg.k, "windows": windows}
+
+
+# the prefill kernels' algorithmic unit (the denominator of the DRAM bytes per unit in
+# profiles/traffic.json): indexer causal score pairs, top-k algorithmic bytes, logical gathered bytes
+TRAFFIC_UNITS = {"indexer": "causal (t, s) score pairs", "topk": "algorithmic bytes",
+                 "sparse_attn": "logical gathered K/V bytes"}
+
+
+def traffic_units(cfg, work: dict) -> dict:
+    return {"indexer": work["indexer_flop"] / (2 * cfg.HI * cfg.dI), "topk": work["topk_bytes"],
+            "sparse_attn": work["attn_gather_bytes"]}
+
+
+def kernel_rooflines(prof: dict, work: dict, steps: int, peaks: dict, workload: str, cfg) -> dict:
+    """Per prefill kernel: mean CUDA-event launch time inside the timed region, achieved rate of
+    its algorithmic work, and the fraction of the measured peak for its bound.  The indexer is
+    compared with the burst bf16 GEMM rate (it runs at the maximum SM clock inside the step; the
+    sustained figure is given alongside).  Sparse attention's roofline is HBM: its fraction is the
+    DRAM bytes one launch really moves (ncu, small case scaled per logical gathered byte) over its
+    time; the logical gather rate, which L2 reuse lifts past the HBM copy rate, is reported
+    separately as achieved_logical / logical_frac."""
+    hbm = peaks["hbm_gbs"]
+    burst = peaks["bf16_tflops"]
+    sust = peaks.get("bf16_tflops_sustained", burst)
+    kern = {}
+
+    def per_launch(kind):
+        p = prof[kind]
+        return p["ms"] / max(1, p["launches"]), p["launches"] / steps
+
+    ms_i, n_i = per_launch("indexer")
+    ms_t, n_t = per_launch("topk")
+    ms_a, n_a = per_launch("sparse_attn")
+    # algorithmic units per launch = per-step work / launches per step (the step totals are exact;
+    # per-launch figures are their mean over the chunks)
+    ach_i = work["indexer_flop"] / n_i / (ms_i / 1e3) / 1e12
+    kern["indexer"] = {"bound": "tensor", "achieved": ach_i, "peak": burst, "unit": "TFLOP/s", "frac": ach_i / burst,
+                       "frac_sustained": ach_i / sust, "ms_per_launch": ms_i, "launches_per_step": n_i,
+                       "peak_source": "measured burst bf16 (MEASURED_PEAKS.json bf16_tflops); sustained alongside"}
+    ach_t = work["topk_bytes"] / n_t / (ms_t / 1e3) / 1e9
+    kern["topk"] = {"bound": "hbm", "achieved": ach_t, "peak": hbm, "unit": "GB/s", "frac": ach_t / hbm,
+                    "ms_per_launch": ms_t, "launches_per_step": n_t, "peak_source": "measured HBM copy"}
+    logical = (work["attn_gather_bytes"] + work["attn_io_bytes"]) / n_a / (ms_a / 1e3) / 1e9
+    kern["sparse_attn"] = {"bound": "hbm", "achieved": logical, "peak": hbm, "unit": "GB/s", "frac": logical / hbm,
+                           "achieved_logical": logical, "logical_frac": logical / hbm, "ms_per_launch": ms_a,
+                           "launches_per_step": n_a, "peak_source": "measured HBM copy"}
+    # DRAM bytes per launch: ncu counters of a small case of the same kernel, scaled by the
+    # launch's algorithmic units, used only while the kernel sources are unchanged
+    tr = {}
+    tpath = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(tpath):
+        with open(tpath) as f:
+            tr = json.load(f)
+    sha = lib_hash()
+    units = traffic_units(cfg, work)
+    n_per = {"indexer": n_i, "topk": n_t, "sparse_attn": n_a}
+    for name, kd in kern.items():
+        ent = tr.get(name)
+        kd["traffic"] = None
+        if ent and ent.get("lib_sha") == sha and ent.get("workload") == workload:
+            kd["traffic"] = ent["bytes_per_unit"] * units[name] / n_per[name]
+            kd["traffic_scaled_from"] = ent["case"]
+            kd["dram_gbs"] = kd["traffic"] / (kd["ms_per_launch"] / 1e3) / 1e9
+    ka = kern["sparse_attn"]
+    if ka["traffic"] is not None:
+        ka["achieved"] = ka["dram_gbs"]
+        ka["frac"] = ka["dram_gbs"] / hbm
+        ka["note"] = ("achieved/frac: DRAM bytes moved per launch over its time; most gathered rows hit L2, "
+                      "so the logical gather rate (achieved_logical) exceeds the HBM copy rate")
+    else:
+        ka["note"] = ("no DRAM capture for these sources: achieved/frac fall back to the logical gather rate, "
+                      "which L2 reuse lifts past the HBM copy rate")
+    return kern
+
+
+def run_profile_case(torch, dsa, cfg, spec: str) -> int:
+    """Query rows R0..R0+N-1 of the workload through dsa_prefill_rows with a workspace that holds
+    all N score rows (one launch of each kernel per call), once untimed and once more.  The small
+    case that ncu captures: a few GB on the device, one launch per kernel per call."""
+    r0, n = (int(v) for v in spec.split(":"))
+    hi = r0 + n
+    assert 0 <= r0 and n > 0 and hi <= cfg.L
+    d = {}
+    for name in ("k", "v", "kI"):
+        d[name] = synth.to_torch(synth.tensor(cfg, name, 0, hi)).cuda()
+    for name in ("q", "qI", "w"):
+        d[name] = synth.to_torch(synth.tensor(cfg, name, r0, n)).cuda()
+    out = torch.empty((n, cfg.Hq, cfg.D), dtype=torch.bfloat16, device="cuda")
+    idx = torch.empty((n, cfg.k), dtype=torch.int32, device="cuda")
+    ws = torch.empty(n * ((hi + 3) // 4 * 4) * 4 + 4096, dtype=torch.uint8, device="cuda")
+    for _ in range(2):
+        dsa.dsa_prefill_rows(d["q"], d["k"], d["v"], d["qI"], d["kI"], d["w"], r0, cfg.k, cfg.scale, out, idx, ws=ws)
+    torch.cuda.synchronize()
+    if dsa.sync_status() != dsa.DSA_OK:
+        raise SystemExit("device error in the profiling case")
+    work = prefill_work(cfg, r0, hi)
+    print(json.dumps({"profile_rows": [r0, n], "workload": cfg.name, "lib_sha": lib_hash(),
+                      "units_per_launch": traffic_units(cfg, work), "unit_names": TRAFFIC_UNITS}), flush=True)
+    return 0
 
 
 def lib_hash() -> str:
@@ -480,12 +583,13 @@ def run_kl(torch, dsa, cfg, barrier, max_over_ranks, peaks, reps: int = 3, rows:
     flop = 4.0 * cfg.Hq * cfg.D * pairs
     k_ms = prof["kl"]["ms"] / reps
     achieved = flop / (k_ms / 1e3) / 1e12
-    tpeak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    tpeak = peaks["bf16_tflops"]                     # the kernel is timed on its own: burst peak
+    tsust = peaks.get("bf16_tflops_sustained", tpeak)
     return {"workload": "prefill_32k" if L == cfg.L else f"prefill_32k_first_{L}", "value": L / (ms / 1e3),
             "unit": "tokens/s", "ms_per_sequence": ms,
             "kernel_ms": k_ms, "indexer_ms": prof["indexer"]["ms"] / reps,
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": tpeak,
-                         "unit": "TFLOP/s", "frac": achieved / tpeak,
+                         "unit": "TFLOP/s", "frac": achieved / tpeak, "frac_sustained": achieved / tsust,
                          "algorithmic": "4 x Hq x D flop per causal (t, s) pair (two passes of Q.K)"},
             "mean_kl": float(kl.mean()), "mma": "warp-level m16n8k16 (mma.sync)"}
 

@@ -617,10 +617,14 @@ dsa_status dsa_prefill(const void* q, const void* k, const void* v, const void* 
                               stream);
 }
 
-dsa_status dsa_decode(const void* q, const void* qI, const void* w, const void* k_new, const void* v_new,
-                      const void* kI_new, void* k_cache, void* v_cache, void* kI_cache, int32_t* ctx_len, int B,
-                      int64_t Lmax, int Hq, int Hkv, int D, int HI, int dI, int topk, float scale, int update_ctx,
-                      void* out, int32_t* idx_out, void* ws, size_t ws_bytes, dsa_stream_t stream) {
+}  // extern "C"
+
+namespace {
+// Host-side checks of a decode step's arguments (everything except the workspace).
+dsa_status check_decode_args(const void* q, const void* qI, const void* w, const void* k_new, const void* v_new,
+                             const void* kI_new, const void* k_cache, const void* v_cache, const void* kI_cache,
+                             const int32_t* ctx_len, int B, int64_t Lmax, int Hq, int Hkv, int D, int HI, int dI,
+                             int topk, float scale, const void* out, const int32_t* idx_out) {
     const void* ptrs[] = {q, qI, w, k_new, v_new, kI_new, k_cache, v_cache, kI_cache, ctx_len, out};
     for (const void* p : ptrs)
         if (!p || !aligned16(p)) return DSA_ERR_INVALID_ARG;
@@ -630,6 +634,19 @@ dsa_status dsa_decode(const void* q, const void* qI, const void* w, const void* 
     if (st != DSA_OK) return st;
     if (dI != kIdxBK || !hi_supported_decode(HI) || topk > kMaxTopk || Lmax > (int64_t)INT32_MAX)
         return DSA_ERR_UNSUPPORTED;
+    return DSA_OK;
+}
+}  // namespace
+
+extern "C" {
+
+dsa_status dsa_decode(const void* q, const void* qI, const void* w, const void* k_new, const void* v_new,
+                      const void* kI_new, void* k_cache, void* v_cache, void* kI_cache, int32_t* ctx_len, int B,
+                      int64_t Lmax, int Hq, int Hkv, int D, int HI, int dI, int topk, float scale, int update_ctx,
+                      void* out, int32_t* idx_out, void* ws, size_t ws_bytes, dsa_stream_t stream) {
+    dsa_status st = check_decode_args(q, qI, w, k_new, v_new, kI_new, k_cache, v_cache, kI_cache, ctx_len, B, Lmax,
+                                      Hq, Hkv, D, HI, dI, topk, scale, out, idx_out);
+    if (st != DSA_OK) return st;
     const DecodeWs L = decode_ws_layout(Lmax, B, Hq, topk, idx_out == nullptr);
     if (!ws || !aligned16(ws)) return DSA_ERR_WORKSPACE;
     if (ws_bytes < L.total) return DSA_ERR_WORKSPACE;
@@ -687,9 +704,12 @@ dsa_status dsa_decode_noalloc(const void* q, const void* qI, const void* w, cons
                               const void* kI_new, void* k_cache, void* v_cache, void* kI_cache, int32_t* ctx_len, int B,
                               int64_t Lmax, int Hq, int Hkv, int D, int HI, int dI, int topk, float scale,
                               int update_ctx, void* out, int32_t* idx_out, dsa_stream_t stream) {
-    if (B <= 0 || Lmax <= 0 || Hq <= 0 || topk <= 0 || Lmax > (int64_t)INT32_MAX || topk > kMaxTopk)
-        return DSA_ERR_INVALID_ARG;
-    // The same work as dsa_decode, with its workspace in the library's fixed scratch array.
+    // The same checks and work as dsa_decode, with its workspace in the library's fixed scratch
+    // array: argument errors are reported exactly as dsa_decode reports them, and only a valid
+    // step that needs more scratch than the array holds gets DSA_ERR_WORKSPACE.
+    dsa_status st0 = check_decode_args(q, qI, w, k_new, v_new, kI_new, k_cache, v_cache, kI_cache, ctx_len, B, Lmax,
+                                       Hq, Hkv, D, HI, dI, topk, scale, out, idx_out);
+    if (st0 != DSA_OK) return st0;
     if (decode_ws_layout(Lmax, B, Hq, topk, idx_out == nullptr).total > kNoAllocScratchBytes)
         return DSA_ERR_WORKSPACE;
     void* scratch = nullptr;

@@ -1,11 +1,13 @@
 """Host-side partitioning of the DSA hot path over ranks (one process per GPU).
 
-The path shards without a data-path collective:
+The path shards by query rows or by sequences:
   - prefill of one sequence: split the query rows into contiguous ranges of equal causal work
     (row t costs t+1 key scores in the indexer and min(k, t+1) gathered keys in attention), each
-    rank holding the whole K, V and kI prefix it needs;
-  - many sequences (prefill batches, decode): whole sequences per rank.
-The only collectives are for timing: a barrier and the max of the per-rank step times.
+    rank holding the whole K, V and kI prefix it needs; the ranks' output rows are then
+    assembled into the whole sequence on every rank (one broadcast per rank's range: the
+    ranges differ in length, so a padded all-gather would move up to twice the bytes);
+  - many sequences (prefill batches, decode): whole sequences per rank, no data-path collective.
+Timing uses a barrier and the max of the per-rank step times.
 """
 from __future__ import annotations
 
@@ -65,3 +67,19 @@ def weak_scaling_value(units_per_rank: float, world: int, max_seconds: float) ->
     if max_seconds <= 0 or not math.isfinite(max_seconds):
         raise ValueError("max_seconds must be positive and finite")
     return units_per_rank * world / max_seconds
+
+
+def assemble_row_ranges(tensors, ranges: list[tuple[int, int]], dist=None) -> None:
+    """Make rows [lo, hi) of every tensor in `tensors` (all indexed by query row along dim 0)
+    hold rank r's values for each r's range (lo, hi) = ranges[r], on every rank: rank r
+    broadcasts its own rows to the others, in rank order, so every rank issues the same
+    collectives in the same order.  Without a process group (or with one rank) nothing moves."""
+    if dist is None or not dist.is_available() or not dist.is_initialized() or dist.get_world_size() == 1:
+        return
+    if len(ranges) != dist.get_world_size():
+        raise ValueError("one row range per rank")
+    for r, (lo, hi) in enumerate(ranges):
+        if hi <= lo:
+            continue
+        for t in tensors:
+            dist.broadcast(t[lo:hi], src=r)

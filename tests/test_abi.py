@@ -234,4 +234,17 @@ def test_host_validation_of_window_rows_and_noalloc_entry_points():
         dsa.DSA_ERR_INVALID_ARG
     assert lib.dsa_decode_noalloc(*dargs, 256, 1 << 22, 32, 4, 128, 32, 64, 2048, f, 0, A, None, None) == \
         dsa.DSA_ERR_WORKSPACE
+    # argument errors before the scratch-size check, with dsa_decode's codes
+    assert lib.dsa_decode_noalloc(*dargs, 256, 1 << 22, 32, 4, 128, 32, 64, 1 << 20, f, 0, A, None, None) == \
+        dsa.DSA_ERR_UNSUPPORTED
+    assert lib.dsa_decode_noalloc(*dargs, 256, 1 << 22, 32, 4, 128, 24, 64, 2048, f, 0, A, None, None) == \
+        dsa.DSA_ERR_UNSUPPORTED
+    assert lib.dsa_decode_noalloc(None, *dargs[1:], 256, 1 << 22, 32, 4, 128, 32, 64, 2048, f, 0, A, None, None) == \
+        dsa.DSA_ERR_INVALID_ARG
+    assert lib.dsa_decode_noalloc(*dargs, 256, 1 << 22, 32, 4, 128, 32, 64, 2048, f, 0, fake(0x10008), None, None) == \
+        dsa.DSA_ERR_INVALID_ARG
+    # the decode workload (16 sequences of 131072 + 256 positions) fits the fixed array even with
+    # the index rows kept in it
+    assert dsa.workspace_size(dsa.DSA_OP_DECODE, 131072 + 256, 16, 32, 32, 2048) <= \
+        int(lib.dsa_decode_noalloc_scratch_bytes())
     assert lib.dsa_launch_count() == 0

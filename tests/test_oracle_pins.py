@@ -94,6 +94,30 @@ def test_indexer_weight_scaling_invariance():
     assert np.array_equal(i1, i2)
 
 
+def test_row_absmax_and_tau_on_a_designed_row():
+    """dsa_rows reports, per row, absmax = max_s |score(t, s)| (the absolute floor of the parity
+    band) and tau = the score of the last selected key.  Hand case: one head picking channel 0,
+    keys with channel-0 values 1, 3, -4, 0.5: ReLU'd dots 1, 3, 0, 0.5.  With w = -2 the scores
+    are -2, -6, 0, -1, so the largest magnitude belongs to a NEGATIVE score (a max of the signed
+    scores would give 0); with w = +2 they are 2, 6, 0, 1."""
+    dI, D = 4, 128
+    kI = bf16_bits([[1, 0, 0, 0], [3, 0, 0, 0], [-4, 0, 0, 0], [0.5, 0, 0, 0]])
+    qI = bf16_bits([[[1, 0, 0, 0]]] * 2)                         # rows t = 0 and t = 3
+    rng = np.random.default_rng(9)
+    q = rand_bf16(rng, (2, 1, D))
+    k = rand_bf16(rng, (4, 1, D))
+    v = rand_bf16(rng, (4, 1, D))
+    t_rows = np.array([0, 3])
+    for wv, absmax, tau, sel in ((-2.0, [2.0, 6.0], [-2.0, -1.0], [2, 3]), (2.0, [2.0, 6.0], [2.0, 2.0], [1, 0])):
+        w = bf16_bits([[wv], [wv]])
+        r = oracle.dsa_rows(q, qI, w, k, v, kI, t_rows, 2, 1.0, keep_scores=True)
+        assert r["absmax"].tolist() == absmax, wv
+        assert r["tau"].tolist() == tau, wv
+        assert r["idx"][0].tolist() == [0, -1]                  # one causal key at t = 0
+        assert r["idx"][1].tolist() == sel, wv
+        assert r["scores"][1, :4].tolist() == [wv * 1, wv * 3, 0.0, wv * 0.5]
+
+
 # ----------------------------------------------------------------------------- top-k
 
 

@@ -5,8 +5,9 @@ memory pool owns the GPU, or a latency-critical path that must not pay cudaMallo
 device synchronisation.  dsa_decode_noalloc runs the same decode step as dsa_decode with its
 scratch in a fixed array inside the library.  This test calls it through the C ABI and checks,
 on two decode steps in a row, that it gives what dsa_decode gives on an identical copy of the
-state (same index sets, outputs within the tolerances of the other parity tests), and that a
-problem too large for the fixed array is refused without a launch.
+state (same index sets, outputs within the tolerances of the other parity tests), both when the
+caller passes idx_out and when the index rows stay in the fixed array, and that a problem too
+large for the fixed array is refused without a launch (argument errors first, as dsa_decode).
 
 This file is named so that pytest collects it last.
 """
@@ -37,7 +38,10 @@ def call_noalloc(new, kc, vc, kIc, ctx, cfg, out, idx, update_ctx=1):
                                         update_ctx, ptr(out), ptr(idx), stream)
 
 
-def test_noalloc_decode_matches_dsa_decode_on_two_steps(cuda_ok):
+@pytest.mark.parametrize("own_idx", [True, False], ids=["idx_out", "idx_in_scratch"])
+def test_noalloc_decode_matches_dsa_decode_on_two_steps(cuda_ok, own_idx):
+    """With idx_out given, and with idx_out NULL (the index rows then live in the fixed array
+    between the top-k and the attention kernels): two steps in a row give dsa_decode's results."""
     cfg = synth.CONFIGS["32k"]
     B, Lmax, steps = 4, 6144, 2
     ctx0 = np.array([5, 1500, 2047, 6000])
@@ -65,13 +69,14 @@ def test_noalloc_decode_matches_dsa_decode_on_two_steps(cuda_ok):
         dsa.dsa_decode(new["q"], new["qI"], new["w"], new["k"], new["v"], new["kI"], *state_a, ctx_a, cfg.k,
                        cfg.scale, out_a, idx_a, ws=ws, update_ctx=True)
         out_b = torch.full_like(out_a, float("nan"))
-        idx_b = torch.full_like(idx_a, -7)
+        idx_b = torch.full_like(idx_a, -7) if own_idx else None
         st = call_noalloc(new, *state_b, ctx_b, cfg, out_b, idx_b)
         assert st == dsa.DSA_OK, dsa.status_string(st)
         assert dsa.sync_status() == dsa.DSA_OK
         assert torch.equal(ctx_a, ctx_b) and np.array_equal(ctx_b.cpu().numpy(), pos + 1)
-        for b in range(B):
-            assert sorted(idx_a[b].tolist()) == sorted(idx_b[b].tolist()), (j, b)
+        if own_idx:
+            for b in range(B):
+                assert sorted(idx_a[b].tolist()) == sorted(idx_b[b].tolist()), (j, b)
         assert_output_ok(bf16_tensor_to_f64(out_b), bf16_tensor_to_f64(out_a), f"step {j}")
         for a, b_ in zip(state_a, state_b):              # the appended cache rows agree too
             assert torch.equal(a.view(torch.int16), b_.view(torch.int16))
@@ -92,5 +97,14 @@ def test_noalloc_decode_refuses_problems_beyond_its_scratch(cuda_ok):
                                       ptr(one), ptr(ctx), B, Lmax, cfg.Hq, cfg.Hkv, cfg.D, cfg.HI, cfg.dI, cfg.k,
                                       ctypes.c_float(cfg.scale), 0, ptr(one), None, stream)
     assert st == dsa.DSA_ERR_WORKSPACE
+    # argument errors come first, exactly as dsa_decode reports them
+    st = dsa.lib().dsa_decode_noalloc(ptr(one), ptr(one), ptr(one), ptr(one), ptr(one), ptr(one), ptr(one), ptr(one),
+                                      ptr(one), ptr(ctx), B, Lmax, cfg.Hq, cfg.Hkv, cfg.D, cfg.HI, cfg.dI, 1 << 20,
+                                      ctypes.c_float(cfg.scale), 0, ptr(one), None, stream)
+    assert st == dsa.DSA_ERR_UNSUPPORTED
+    st = dsa.lib().dsa_decode_noalloc(None, ptr(one), ptr(one), ptr(one), ptr(one), ptr(one), ptr(one), ptr(one),
+                                      ptr(one), ptr(ctx), B, Lmax, cfg.Hq, cfg.Hkv, cfg.D, cfg.HI, cfg.dI, cfg.k,
+                                      ctypes.c_float(cfg.scale), 0, ptr(one), None, stream)
+    assert st == dsa.DSA_ERR_INVALID_ARG
     assert dsa.launch_count() == n0
     assert dsa.sync_status() == dsa.DSA_OK

@@ -259,7 +259,7 @@ dsa_status run_topk(const float* scores, int64_t ld, int rows, int64_t q_pos0, c
     const int smem = (int)sizeof(TopkSmem);
     // Few long rows: a cluster of CTAs per row; otherwise one CTA per row.
     if ((long long)rows * kTkCluster <= 2LL * sms && n_max > 4LL * kTkCap) {
-        const int csmem = smem + kTkCap * 8;
+        const int csmem = smem;
         static DeviceFlags cattr;
         if (!set_smem_limit(topk_cluster_kernel, csmem, cattr)) return DSA_ERR_CUDA;
         cudaLaunchConfig_t cfg = {};
@@ -412,7 +412,7 @@ int dsa_version(void) { return kVersion; }
 dsa_status dsa_index(const void* qI, const void* kI, const void* w, int Lq, int64_t Lk, int HI, int dI,
                      int64_t q_pos0, float* scores, int64_t ld_scores, dsa_stream_t stream) {
     if (!qI || !kI || !w || !scores) return DSA_ERR_INVALID_ARG;
-    if (!aligned16(qI) || !aligned16(kI) || !aligned16(scores)) return DSA_ERR_INVALID_ARG;
+    if (!aligned16(qI) || !aligned16(kI) || !aligned16(w) || !aligned16(scores)) return DSA_ERR_INVALID_ARG;
     if (Lq <= 0 || Lk <= 0 || HI <= 0 || dI <= 0 || q_pos0 < 0) return DSA_ERR_INVALID_ARG;
     if (q_pos0 + Lq > Lk || ld_scores < q_pos0 + Lq || ld_scores % 4 != 0) return DSA_ERR_INVALID_ARG;
     if (dI != kIdxBK || !hi_supported_prefill(HI)) return DSA_ERR_UNSUPPORTED;

@@ -15,8 +15,10 @@
 // Roles (one CTA per SM, persistent):
 //   warp 0        TMA producer: the unit's Q tile (once per unit) and a ring of kI tiles
 //   warp 1        TMEM allocator + single-thread tcgen05.mma issuer
-//   warps 2..     epilogue: tcgen05.ld, ReLU, weight FMA, head sum, score store;
-//                 NWG warpgroups split the BN columns between them
+//   warps 2-3     idle (they complete the role warpgroup)
+//   warps 4..     epilogue: tcgen05.ld, ReLU, weight FMA, head sum, score store;
+//                 NWG warpgroups split the BN columns between them and keep the unit's weights
+//                 for their columns in registers
 // Two TMEM accumulators (2 x BN fp32 columns) let the MMA of tile j+1 overlap the epilogue of
 // tile j.  Work units are (problem p, query block qb, key-tile range); prefill uses one problem
 // and whole causal key ranges, decode uses one problem per sequence and splits its keys.
@@ -100,7 +102,8 @@ __device__ __forceinline__ int indexer_unit_of(int round, int cta, int grid) {
 template <int CHUNK>
 __device__ __forceinline__ void tmem_ld_chunk(uint32_t taddr, float (&v)[CHUNK]) {
     if constexpr (CHUNK == 32) tmem_ld_32x32b_x32(taddr, v);
-    else tmem_ld_32x32b_x16(taddr, v);
+    else if constexpr (CHUNK == 16) tmem_ld_32x32b_x16(taddr, v);
+    else tmem_ld_32x32b_x8(taddr, v);
 }
 
 // c + a * b on packed fp32 pairs (one fma.rn.f32x2).
@@ -140,21 +143,18 @@ __device__ __forceinline__ float head_sum(const float* v, const float* w) {
 #pragma unroll
         for (int i = 0; i < NA; ++i) acc[i] = make_float2(0.f, 0.f);
         if constexpr (N % 4 == 0) {
-            // weights four at a time: one 16-byte shared load (a warp-wide broadcast) per 4 heads
 #pragma unroll
             for (int q = 0; q < N / 4; ++q) {
-                const float4 w4 = *reinterpret_cast<const float4*>(w + 4 * q);
                 const float2 x0 = relu_pair_alu(v[4 * q], v[4 * q + 1]);
                 const float2 x1 = relu2_pair_fma(v[4 * q + 2], v[4 * q + 3]);
-                acc[(2 * q) % NA] = ffma2(x0, make_float2(w4.x, w4.y), acc[(2 * q) % NA]);
-                acc[(2 * q + 1) % NA] = ffma2(x1, make_float2(w4.z, w4.w), acc[(2 * q + 1) % NA]);
+                acc[(2 * q) % NA] = ffma2(x0, make_float2(w[4 * q], w[4 * q + 1]), acc[(2 * q) % NA]);
+                acc[(2 * q + 1) % NA] = ffma2(x1, make_float2(w[4 * q + 2], w[4 * q + 3]), acc[(2 * q + 1) % NA]);
             }
         } else {
 #pragma unroll
             for (int p = 0; p < NP; ++p) {
                 const float2 x = make_float2(fmaxf(v[2 * p], 0.f), fmaxf(v[2 * p + 1], 0.f));
-                const float2 ww = *reinterpret_cast<const float2*>(w + 2 * p);
-                acc[p % NA] = ffma2(x, ww, acc[p % NA]);
+                acc[p % NA] = ffma2(x, make_float2(w[2 * p], w[2 * p + 1]), acc[p % NA]);
             }
         }
         float r = 0.f;
@@ -164,16 +164,16 @@ __device__ __forceinline__ float head_sum(const float* v, const float* w) {
     }
 }
 
-// carry[0..3] += packed partial sums of w[h] * max(v[h], 0) over one chunk of N heads.
+// carry[0..1] += packed partial sums of w[h] * max(v[h], 0) over one chunk of N heads.  `w` points
+// into a register array (every index is a compile-time constant after unrolling).
 template <int N>
-__device__ __forceinline__ void head_sum_acc(const float* v, const float* w, float2 (&carry)[4]) {
+__device__ __forceinline__ void head_sum_acc(const float* v, const float* w, float2 (&carry)[2]) {
 #pragma unroll
     for (int q = 0; q < N / 4; ++q) {
-        const float4 w4 = *reinterpret_cast<const float4*>(w + 4 * q);
         const float2 x0 = relu_pair_alu(v[4 * q], v[4 * q + 1]);
         const float2 x1 = relu2_pair_fma(v[4 * q + 2], v[4 * q + 3]);
-        carry[(2 * q) % 4] = ffma2(x0, make_float2(w4.x, w4.y), carry[(2 * q) % 4]);
-        carry[(2 * q + 1) % 4] = ffma2(x1, make_float2(w4.z, w4.w), carry[(2 * q + 1) % 4]);
+        carry[0] = ffma2(x0, make_float2(w[4 * q], w[4 * q + 1]), carry[0]);
+        carry[1] = ffma2(x1, make_float2(w[4 * q + 2], w[4 * q + 3]), carry[1]);
     }
 }
 
@@ -184,35 +184,42 @@ struct IndexerCfg {
     // of the per-token reduction chains
     static constexpr int NWG = (BN >= 256 && BN / 4 >= HI) ? 4 : (BN >= 128 && BN / 2 >= HI) ? 2 : 1;
     static constexpr int COLS_WG = BN / NWG;
-    static constexpr int CHUNK = COLS_WG >= 32 ? 32 : 16;
+    // TMEM loads of 8 columns: the warpgroup's COLS_WG weights live in registers for a whole
+    // work unit, so the loads stay small
+    static constexpr int CHUNK = 8;
     static constexpr int NCHUNK = COLS_WG / CHUNK;
-    static constexpr int THREADS = 64 + NWG * 128;
+    // warpgroup 0 holds the roles (warp 0 TMA, warp 1 MMA, warps 2-3 idle); warpgroups 1..NWG the
+    // epilogue.  With four epilogue warpgroups the roles hand registers to the epilogue
+    // (setmaxnreg): launched at 96 per thread (20 warps, 5 per SM sub-partition), the role
+    // warpgroup drops to 32 and the epilogue rises to 112 -- 4*32*32 + 16*32*112 = 640*96, and
+    // per sub-partition 32*(32 + 4*112) <= 16384 -- which keeps a unit's 64 weights in registers.
+    static constexpr int THREADS = 128 + NWG * 128;
+    static constexpr bool REGSPLIT = NWG == 4;
+    static constexpr int ROLE_REGS = 32, EPI_REGS = 112;
     static constexpr int A_BYTES = kIdxBM * kIdxBK * 2;  // 16 KB
     static constexpr int B_BYTES = BN * kIdxBK * 2;
     static constexpr int TMEM_COLS = (2 * BN <= 32) ? 32 : (2 * BN <= 64) ? 64 : (2 * BN <= 128) ? 128 : (2 * BN <= 256) ? 256 : 512;
     // shared memory layout (offsets from a 1024-aligned base)
     static constexpr int OFF_A = 0;
     static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
-    static constexpr int OFF_W = OFF_B + 2 * B_BYTES;       // per epilogue warp: 2 x COLS_WG weights
-    static constexpr int OFF_BAR = OFF_W + NWG * 4 * 2 * COLS_WG * 4;
+    static constexpr int OFF_BAR = OFF_B + 2 * B_BYTES;
     static constexpr int NBAR = 2 * STAGES + 8;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int SMEM = OFF_MISC + 16 + 1024;  // + alignment slack
     static_assert(BN % HI == 0 && BN >= 16 && BN <= 256 && BN % 16 == 0, "bad BN");
     static_assert(HI <= COLS_WG, "a token's heads must stay inside one warpgroup");
     static_assert(HI <= CHUNK || HI % CHUNK == 0, "bad HI");
+    static_assert(COLS_WG % 8 == 0 && COLS_WG <= 64, "weights: whole 16-byte groups, at most 64 registers");
 };
 
 template <int HI, int BN, int STAGES>
-__global__ void __launch_bounds__(IndexerCfg<HI, BN, STAGES>::THREADS, 1)
-    indexer_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
+__global__ void __launch_bounds__(IndexerCfg<HI, BN, STAGES>::THREADS, 1) indexer_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                    const IndexerParams P) {
     using C = IndexerCfg<HI, BN, STAGES>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sA = smem + C::OFF_A;
     uint8_t* sB = smem + C::OFF_B;
-    float* sW = reinterpret_cast<float*>(smem + C::OFF_W);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
     uint64_t* a_full = bars;
     uint64_t* a_empty = bars + STAGES;
@@ -275,7 +282,9 @@ __global__ void __launch_bounds__(IndexerCfg<HI, BN, STAGES>::THREADS, 1)
     const uint32_t tmem_base = *tmem_slot;
     const int grid = gridDim.x, cta = blockIdx.x;
 
-    if (warp == 0) {
+    if (warp < 4) {
+      if constexpr (C::REGSPLIT) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(C::ROLE_REGS));
+      if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
             int st = 0;
@@ -308,7 +317,7 @@ __global__ void __launch_bounds__(IndexerCfg<HI, BN, STAGES>::THREADS, 1)
                 for (int i = 0; i < 2; ++i) wait_parity(&q_full[i], i < qbuf ? q_ph : q_ph ^ 1, 0x104, nullptr);
             }
         }
-    } else if (warp == 1) {
+      } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             constexpr uint32_t idesc = idesc_bf16_f32<kIdxBM, BN>();
@@ -343,32 +352,48 @@ __global__ void __launch_bounds__(IndexerCfg<HI, BN, STAGES>::THREADS, 1)
                 if (++qbuf == 2) { qbuf = 0; q_ph ^= 1; }
             }
         }
+      }
     } else {
+        if constexpr (C::REGSPLIT) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(C::EPI_REGS));
         // ------------------------------------------------------------ epilogue warpgroups
-        const int et = threadIdx.x - 64;            // 0 .. NWG*128-1
+        const int et = threadIdx.x - 128;           // 0 .. NWG*128-1
         const int wg = et >> 7;                     // column half
         const int quarter = warp & 3;               // TMEM lanes this warp may access
         const int key_in_tile = quarter * 32 + lane;
-        int ab = 0, ubuf = 0;
+        int ab = 0;
         uint32_t acc_ph = 0;
         for (int rd = 0;; ++rd) {
             const int u = indexer_unit_of(rd, cta, grid);
             if (u >= P.num_units) break;
             const IndexerUnit U = indexer_unit<C::TB>(P, u);
             if (U.kt0 >= U.kt1) continue;
-            // Weights of this unit's tokens for this warpgroup's columns (column c = token*HI + head),
-            // one private copy per warp so that only __syncwarp is needed.
-            float* w_s = sW + ((warp - 2) * 2 + ubuf) * C::COLS_WG;
-            for (int cc = lane; cc < C::COLS_WG; cc += 32) {
-                const int c = wg * C::COLS_WG + cc;
-                const int tok = c / HI;
-                float wv = 0.f;
-                if (tok < U.rows)
-                    wv = __bfloat162float(P.w[((long long)U.p * P.Lq + (long long)U.qb * C::TB + tok) * HI + (c % HI)]) *
-                         weight_store_scale<HI>(c % HI);
-                w_s[cc] = wv;
+            // This unit's weights for this warpgroup's columns (column c = token*HI + head), held in
+            // registers for all of the unit's key tiles: columns [c, c+8) are 8 consecutive bf16 of
+            // w (the unit's tokens are consecutive rows), one 16-byte load each; tokens past the
+            // unit's rows get weight 0.
+            float wr[C::COLS_WG];
+            {
+                const __nv_bfloat16* wu = P.w + ((long long)U.p * P.Lq + (long long)U.qb * C::TB) * HI;
+#pragma unroll
+                for (int cc = 0; cc < C::COLS_WG; cc += 8) {
+                    const int c = wg * C::COLS_WG + cc;
+                    if ((c + 7) / HI < U.rows) {
+                        const uint4 raw = __ldg(reinterpret_cast<const uint4*>(wu + c));
+                        const uint32_t wv[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            const uint32_t bits = (e & 1) ? (wv[e >> 1] & 0xFFFF0000u) : (wv[e >> 1] << 16);
+                            wr[cc + e] = __uint_as_float(bits) * weight_store_scale<HI>((c + e) % HI);
+                        }
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 8; ++e)
+                            wr[cc + e] = (c + e) / HI < U.rows
+                                             ? __bfloat162float(wu[c + e]) * weight_store_scale<HI>((c + e) % HI)
+                                             : 0.f;
+                    }
+                }
             }
-            __syncwarp();
             bool ok = true;
             for (int kt = U.kt0; kt < U.kt1; ++kt) {
                 ok = wait_parity(&acc_full[ab], acc_ph, 0x301, abort_flag);
@@ -376,15 +401,19 @@ __global__ void __launch_bounds__(IndexerCfg<HI, BN, STAGES>::THREADS, 1)
                 ok = __all_sync(0xffffffffu, ok);
                 if (!ok) break;
                 tc_fence_after();
-                const long long s = (long long)kt * kIdxBM + key_in_tile;
+                // key positions fit in 32 bits (the entry points refuse Lk > INT32_MAX)
+                const int s = kt * kIdxBM + key_in_tile;
                 const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + ab * BN + wg * C::COLS_WG;
-                const long long row0 = (long long)U.p * P.Lq + (long long)U.qb * C::TB;
+                // this lane's score of the unit's first token (row0) and key s; token j adds j*ld
+                float* const srow = P.scores + ((long long)U.p * P.Lq + (long long)U.qb * C::TB) * P.ld + s;
+                // s <= tq0 + tok also keeps s < Lk: a valid token's position is below Lk
+                const int tq0 = (int)U.tq0;
                 // TMEM loads run one chunk ahead of the math: ld(c+1) is in flight while chunk c is
                 // reduced; the accumulator is released right after the last load completes.
                 float va[C::CHUNK], vb[C::CHUNK];
-                float2 carry[4];
+                float2 carry[2];
 #pragma unroll
-                for (int i = 0; i < 4; ++i) carry[i] = make_float2(0.f, 0.f);
+                for (int i = 0; i < 2; ++i) carry[i] = make_float2(0.f, 0.f);
                 tmem_ld_chunk<C::CHUNK>(taddr, va);
                 tmem_ld_wait();
 #pragma unroll
@@ -401,19 +430,18 @@ __global__ void __launch_bounds__(IndexerCfg<HI, BN, STAGES>::THREADS, 1)
                     if constexpr (HI <= C::CHUNK) {
 #pragma unroll
                         for (int j = 0; j < C::CHUNK / HI; ++j) {
-                            const float a = head_sum<HI>(cur + j * HI, w_s + cw + j * HI);
+                            const float a = head_sum<HI>(cur + j * HI, wr + cw + j * HI);
                             const int tok = (wg * C::COLS_WG + cw) / HI + j;
-                            if (tok < U.rows && s <= U.tq0 + tok && s < P.Lk) P.scores[(row0 + tok) * P.ld + s] = a;
+                            if (tok < U.rows && s <= tq0 + tok) srow[(long long)tok * P.ld] = a;
                         }
                     } else {
-                        head_sum_acc<C::CHUNK>(cur, w_s + cw, carry);
+                        head_sum_acc<C::CHUNK>(cur, wr + cw, carry);
                         if ((wg * C::COLS_WG + cw + C::CHUNK) % HI == 0) {
-                            const float a = (carry[0].x + carry[0].y) + (carry[1].x + carry[1].y) +
-                                            (carry[2].x + carry[2].y) + (carry[3].x + carry[3].y);
+                            const float a = (carry[0].x + carry[0].y) + (carry[1].x + carry[1].y);
                             const int tok = (wg * C::COLS_WG + cw) / HI;
-                            if (tok < U.rows && s <= U.tq0 + tok && s < P.Lk) P.scores[(row0 + tok) * P.ld + s] = a;
+                            if (tok < U.rows && s <= tq0 + tok) srow[(long long)tok * P.ld] = a;
 #pragma unroll
-                            for (int i = 0; i < 4; ++i) carry[i] = make_float2(0.f, 0.f);
+                            for (int i = 0; i < 2; ++i) carry[i] = make_float2(0.f, 0.f);
                         }
                     }
                     if (ch + 1 < C::NCHUNK) tmem_ld_wait();
@@ -421,7 +449,6 @@ __global__ void __launch_bounds__(IndexerCfg<HI, BN, STAGES>::THREADS, 1)
                 if (++ab == 2) { ab = 0; acc_ph ^= 1; }
             }
             if (!ok) break;
-            ubuf ^= 1;
         }
     }
 

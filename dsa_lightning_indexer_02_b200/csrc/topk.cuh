@@ -48,6 +48,14 @@ constexpr int kTkUnroll = 8;                  // float4 loads in flight per lane
 constexpr int kTkCluster = 8;                 // CTAs per row in the cluster kernel
 constexpr int kTkMaxRegions = kTkCluster * kTkWarps;
 
+// The 128 threads (4 warps) of a CTA that select one row; tid is the thread's index in the CTA.
+struct Grp {
+    int tid;
+    __device__ __forceinline__ int lane() const { return tid & 31; }
+    __device__ __forceinline__ int warp() const { return tid >> 5; }
+    __device__ __forceinline__ void sync() const { __syncthreads(); }
+};
+
 struct TopkParams {
     const float* scores;  // row r at scores + r*ld (16-byte aligned rows)
     long long ld;
@@ -111,12 +119,12 @@ __device__ __forceinline__ uint32_t warp_incl_scan(uint32_t x) {
 }
 
 // Exclusive block prefix sum (4 warps); returns the block total.
-__device__ __forceinline__ uint32_t block_excl_scan(TopkSmem& S, uint32_t v, uint32_t& total) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+__device__ __forceinline__ uint32_t block_excl_scan(TopkSmem& S, const Grp& G, uint32_t v, uint32_t& total) {
+    const int lane = G.lane(), warp = G.warp();
     const uint32_t x = warp_incl_scan(v);
-    __syncthreads();
+    G.sync();
     if (lane == 31) S.red[warp] = x;
-    __syncthreads();
+    G.sync();
     uint32_t before = 0, tot = 0;
 #pragma unroll
     for (int w = 0; w < kTkWarps; ++w) {
@@ -129,25 +137,25 @@ __device__ __forceinline__ uint32_t block_excl_scan(TopkSmem& S, uint32_t v, uin
 
 // Bin b of S.hist[0, nbins) with (count above b) < need <= (count above b) + hist[b]; result in
 // S.sel_bin / S.sel_gt.  nbins <= kTkBins; needs the histogram total >= need.
-__device__ __forceinline__ void find_threshold_bin(TopkSmem& S, int nbins, uint32_t need) {
+__device__ __forceinline__ void find_threshold_bin(TopkSmem& S, const Grp& G, int nbins, uint32_t need) {
     constexpr int kMaxPer = kTkBins / kTkThreads;
     const int per = (nbins + kTkThreads - 1) / kTkThreads;
-    const int lo = threadIdx.x * per;
+    const int lo = G.tid * per;
     uint32_t mine = 0;
 #pragma unroll
     for (int b = 0; b < kMaxPer; ++b)
         if (b < per && lo + b < nbins) mine += S.hist[lo + b];
     // suffix sums over threads (a higher thread owns higher bins)
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int lane = G.lane(), warp = G.warp();
     uint32_t x = mine;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
         const uint32_t y = __shfl_down_sync(0xffffffffu, x, o);
         if (lane + o < 32) x += y;
     }
-    __syncthreads();
+    G.sync();
     if (lane == 0) S.red[warp] = x;
-    __syncthreads();
+    G.sync();
     uint32_t above = x - mine;
 #pragma unroll
     for (int w = 0; w < kTkWarps; ++w) above += (w > warp) ? S.red[w] : 0u;
@@ -163,11 +171,11 @@ __device__ __forceinline__ void find_threshold_bin(TopkSmem& S, int nbins, uint3
             cum += h;
         }
     }
-    __syncthreads();
+    G.sync();
 }
 
-__device__ __forceinline__ void clear_hist(TopkSmem& S, int nbins) {
-    for (int b = threadIdx.x; b < nbins; b += kTkThreads) S.hist[b] = 0;
+__device__ __forceinline__ void clear_hist(TopkSmem& S, const Grp& G, int nbins) {
+    for (int b = G.tid; b < nbins; b += kTkThreads) S.hist[b] = 0;
 }
 
 // T0 from m sample keys in S.cand_key[0, m): a lower bound on the key at rank rs (counted from
@@ -177,11 +185,12 @@ __device__ __forceinline__ void clear_hist(TopkSmem& S, int nbins) {
 // holding rank rs again into up to 1024 parts.  Every sample key >= T0 is counted, so at least
 // rs samples are >= T0.  Bins that follow the data (rather than fixed top bits of the key) keep
 // the shared-memory atomics spread out when the scores sit in a narrow range.
-__device__ __forceinline__ uint32_t sample_threshold(TopkSmem& S, int m, uint32_t rs) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    __syncthreads();  // the samples were written by other threads
+__device__ __forceinline__ uint32_t sample_threshold(TopkSmem& S, const Grp& G, int m, uint32_t rs,
+                                                    uint32_t* kmax_out = nullptr) {
+    const int lane = G.lane(), warp = G.warp();
+    G.sync();  // the samples were written by other threads
     uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
-    for (int e = threadIdx.x; e < m; e += kTkThreads) {
+    for (int e = G.tid; e < m; e += kTkThreads) {
         const uint32_t key = S.cand_key[e];
         if (key) {
             kmin = min(kmin, key);
@@ -197,49 +206,57 @@ __device__ __forceinline__ uint32_t sample_threshold(TopkSmem& S, int m, uint32_
         S.hist[warp] = kmin;
         S.hist[kTkWarps + warp] = kmax;
     }
-    __syncthreads();
+    G.sync();
 #pragma unroll
     for (int w = 0; w < kTkWarps; ++w) {
         kmin = min(kmin, S.hist[w]);
         kmax = max(kmax, S.hist[kTkWarps + w]);
     }
-    __syncthreads();
+    G.sync();
     if (kmin > kmax) kmin = kmax = 0u;  // every sample masked
+    if (kmax_out) *kmax_out = kmax;
     const uint32_t span = kmax - kmin;
     const int sh1 = (span >> 10) ? 32 - __clz(span >> 10) : 0;  // (span >> sh1) < 1024
-    clear_hist(S, kTkBins);
-    __syncthreads();
-    for (int e = threadIdx.x; e < m; e += kTkThreads) {
+    clear_hist(S, G, kTkBins);
+    G.sync();
+    for (int e = G.tid; e < m; e += kTkThreads) {
         const uint32_t key = S.cand_key[e];
         atomicAdd(&S.hist[min((key > kmin ? key - kmin : 0u) >> sh1, (uint32_t)kTkBins - 1u)], 1u);
     }
-    __syncthreads();
-    find_threshold_bin(S, kTkBins, rs);
+    G.sync();
+    find_threshold_bin(S, G, kTkBins, rs);
     const uint32_t b1 = S.sel_bin, need = rs - S.sel_gt;
     if (sh1 == 0) return kmin + b1;  // bins of single key values: exact
     const int sh2 = sh1 > 10 ? sh1 - 10 : 0;
     const uint32_t base = b1 << sh1;
-    clear_hist(S, kTkBins);
-    __syncthreads();
-    for (int e = threadIdx.x; e < m; e += kTkThreads) {
+    clear_hist(S, G, kTkBins);
+    G.sync();
+    for (int e = G.tid; e < m; e += kTkThreads) {
         const uint32_t key = S.cand_key[e];
         const uint32_t d = key > kmin ? key - kmin : 0u;
         if (min(d >> sh1, (uint32_t)kTkBins - 1u) == b1) atomicAdd(&S.hist[min((d - base) >> sh2, (uint32_t)kTkBins - 1u)], 1u);
     }
-    __syncthreads();
-    find_threshold_bin(S, kTkBins, need);
+    G.sync();
+    find_threshold_bin(S, G, kTkBins, need);
     return kmin + base + (S.sel_bin << sh2);
 }
 
 // Stream float4 groups [g_lo, g_hi) of a row whose keys e_lo <= e < n compete and compact the
 // scores >= F0 into this warp's region, in index order.  Warp w takes the 128-byte pieces p
 // (keys 32p .. 32p+31 of the row) with p % 4 == w: region w.
+// Each batch of kTkUnroll float4 loads per lane is filtered as a whole: the per-float4 candidate
+// counts of a lane (0..4 each) ride in the bytes of two registers through one warp-wide
+// inclusive scan (5 shuffle steps), which gives every lane the position of each of its
+// candidates -- independent work for the whole batch instead of a ballot chain per load.
+// With chist, every candidate also adds one to bin min((key - hT0) >> hsh, kTkBins - 1) of the
+// 1024-bin histogram chist (which may live in another CTA's shared memory).
 // Returns how many scores of this warp qualified (may exceed the region; the excess is dropped).
-__device__ __forceinline__ uint32_t stream_collect(TopkSmem& S, const float4* row4, int g_lo, int g_hi, int e_lo,
-                                                   int n, float F0, int region_base) {
+__device__ __forceinline__ uint32_t stream_collect(TopkSmem& S, const Grp& G, const float4* row4, int g_lo, int g_hi,
+                                                   int e_lo, int n, float F0, int region_base,
+                                                   uint32_t* chist = nullptr, uint32_t hT0 = 0, int hsh = 0) {
+    static_assert(kTkUnroll == 8, "the packed scan holds 8 counts");
     const int g_first = g_lo;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const uint32_t lanes_below = (1u << lane) - 1u;
+    const int lane = G.lane(), warp = G.warp();
     // float4 offset inside a 128-float4 round: piece (lane/8)*4 + warp, float4 lane%8 of it
     const int lane_off = (lane >> 3) * 32 + warp * 8 + (lane & 7);
     // float4 groups whose four keys all lie in [e_lo, n): [g_in_lo, g_in_hi)
@@ -258,6 +275,8 @@ __device__ __forceinline__ uint32_t stream_collect(TopkSmem& S, const float4* ro
             const int g = g0 + u * 128 + lane_off;
             v[u] = (interior || g < g_hi) ? __ldcs(row4 + g) : make_float4(0.f, 0.f, 0.f, 0.f);
         }
+        uint32_t m[kTkUnroll];
+        uint32_t c_lo = 0, c_hi = 0;  // candidate counts of float4 u in byte u (u < 4) or byte u-4
 #pragma unroll
         for (int u = 0; u < kTkUnroll; ++u) {
             const int g = g0 + u * 128 + lane_off;
@@ -271,35 +290,48 @@ __device__ __forceinline__ uint32_t stream_collect(TopkSmem& S, const float4* ro
                 for (int j = 0; j < 4; ++j)
                     if (f[j] >= F0 && g * 4 + j < n && g * 4 + j >= e_lo && g >= g_first) mask |= 1u << j;
             }
-            // compaction in (lane, j) order = index order: the exclusive prefix of the per-lane
-            // counts from ballots (one ballot when no lane has more than one candidate)
-            const uint32_t c = __popc(mask);
-            const uint32_t any = __ballot_sync(0xffffffffu, c != 0);
-            if (any == 0) continue;
-            uint32_t excl, tot;
-            if (__ballot_sync(0xffffffffu, c > 1) == 0) {
-                excl = __popc(any & lanes_below);
-                tot = __popc(any);
-            } else {
-                const uint32_t b0 = __ballot_sync(0xffffffffu, c & 1u), b1 = __ballot_sync(0xffffffffu, c & 2u),
-                               b2 = __ballot_sync(0xffffffffu, c & 4u);
-                excl = __popc(b0 & lanes_below) + 2 * __popc(b1 & lanes_below) + 4 * __popc(b2 & lanes_below);
-                tot = __popc(b0) + 2 * __popc(b1) + 4 * __popc(b2);
+            m[u] = mask;
+            if (u < 4) c_lo |= (uint32_t)__popc(mask) << (8 * u);
+            else c_hi |= (uint32_t)__popc(mask) << (8 * (u - 4));
+        }
+        if (__ballot_sync(0xffffffffu, (c_lo | c_hi) != 0) == 0) continue;
+        // inclusive scan over lanes of the packed counts (each prefix <= 128 fits its byte)
+        uint32_t s_lo = c_lo, s_hi = c_hi;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y_lo = __shfl_up_sync(0xffffffffu, s_lo, o), y_hi = __shfl_up_sync(0xffffffffu, s_hi, o);
+            if (lane >= o) {
+                s_lo += y_lo;
+                s_hi += y_hi;
             }
-            if (mask) {
-                uint32_t pos = cnt + excl;
+        }
+        const uint32_t t_lo = __shfl_sync(0xffffffffu, s_lo, 31), t_hi = __shfl_sync(0xffffffffu, s_hi, 31);
+        const uint32_t e_lo8 = s_lo - c_lo, e_hi8 = s_hi - c_hi;  // exclusive prefixes, bytewise
+        // candidates of float4 u follow those of every lane's float4s before u (index order)
+        uint32_t base = cnt;
+#pragma unroll
+        for (int u = 0; u < kTkUnroll; ++u) {
+            const uint32_t excl = ((u < 4 ? e_lo8 : e_hi8) >> (8 * (u & 3))) & 0xFFu;
+            const uint32_t tot = ((u < 4 ? t_lo : t_hi) >> (8 * (u & 3))) & 0xFFu;
+            if (m[u]) {
+                const int g = g0 + u * 128 + lane_off;
+                const float f[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+                uint32_t pos = base + excl;
 #pragma unroll
                 for (int j = 0; j < 4; ++j)
-                    if (mask & (1u << j)) {
+                    if (m[u] & (1u << j)) {
+                        const uint32_t key = score_key(f[j]);
                         if (pos < (uint32_t)kTkRegion) {
-                            S.cand_key[region_base + pos] = score_key(f[j]);
+                            S.cand_key[region_base + pos] = key;
                             S.cand_idx[region_base + pos] = g * 4 + j;
                         }
+                        if (chist) atomicAdd(chist + min((key - hT0) >> hsh, (uint32_t)kTkBins - 1u), 1u);
                         ++pos;
                     }
             }
-            cnt += tot;
+            base += tot;
         }
+        cnt = base;
     }
     return cnt;
 }
@@ -312,8 +344,8 @@ __device__ __forceinline__ uint32_t stream_collect(TopkSmem& S, const float4* ro
 constexpr int kTkSmallBin = 64;
 constexpr int kTkBatch = 4;  // shared-memory loads batched per thread in the refinement passes
 
-__device__ __forceinline__ bool refine_and_emit(TopkSmem& S, uint32_t lo, int k, int* out) {
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+__device__ __forceinline__ bool refine_and_emit(TopkSmem& S, const Grp& G, uint32_t lo, int k, int* out) {
+    const int tid = G.tid, lane = G.lane(), warp = G.warp();
     const int nreg = S.nreg;
     // The passes below hoist each region's pointers and count into registers and batch their
     // shared-memory loads (kTkBatch per thread ahead of the use), so that they overlap instead of
@@ -328,9 +360,9 @@ __device__ __forceinline__ bool refine_and_emit(TopkSmem& S, uint32_t lo, int k,
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    __syncthreads();
+    G.sync();
     if (lane == 0) S.red[warp] = mx;
-    __syncthreads();
+    G.sync();
     uint32_t R = 0;
 #pragma unroll
     for (int w = 0; w < kTkWarps; ++w) R = max(R, S.red[w]);
@@ -341,9 +373,9 @@ __device__ __forceinline__ bool refine_and_emit(TopkSmem& S, uint32_t lo, int k,
     while (fixed > 0) {
         const int sh = fixed > 10 ? fixed - 10 : 0;
         const int nbins = 1 << (fixed - sh);
-        __syncthreads();
-        clear_hist(S, nbins);
-        __syncthreads();
+        G.sync();
+        clear_hist(S, G, nbins);
+        G.sync();
         for (int r = 0; r < nreg; ++r) {
             const uint32_t* kp = S.reg_kp[r];
             const int cnt = S.reg_cnt[r];
@@ -361,15 +393,15 @@ __device__ __forceinline__ bool refine_and_emit(TopkSmem& S, uint32_t lo, int k,
                 }
             }
         }
-        __syncthreads();
-        find_threshold_bin(S, nbins, need);
+        G.sync();
+        find_threshold_bin(S, G, nbins, need);
         need -= S.sel_gt;
         cnt_b = S.hist[S.sel_bin];
         pv |= S.sel_bin << sh;
         fixed = sh;
         if (cnt_b <= (uint32_t)kTkSmallBin) break;  // uniform: every thread read the same count
     }
-    __syncthreads();
+    G.sync();
     // boundary bin: offsets d with d >> fixed == pv >> fixed; kept outright: d >> fixed > pv >> fixed
     if (cnt_b > (uint32_t)(kTkBins / 2)) return false;
     const uint32_t bin = fixed >= 32 ? 0u : (pv >> fixed);
@@ -382,7 +414,7 @@ __device__ __forceinline__ bool refine_and_emit(TopkSmem& S, uint32_t lo, int k,
     uint32_t* bloc = S.hist + kTkBins / 2;        // region << 16 | position
     auto loc_idx = [&](uint32_t l) { return S.reg_ip[l >> 16][l & 0xFFFFu]; };
     if (tid == 0) S.sel_bin = 0;
-    __syncthreads();
+    G.sync();
     for (int r = 0; r < nreg; ++r) {
         const uint32_t* kp = S.reg_kp[r];
         const int cnt = S.reg_cnt[r];
@@ -404,7 +436,7 @@ __device__ __forceinline__ bool refine_and_emit(TopkSmem& S, uint32_t lo, int k,
             }
         }
     }
-    __syncthreads();
+    G.sync();
     bool drop[(kTkBins / 2 + kTkThreads - 1) / kTkThreads];
 #pragma unroll
     for (int j = 0; j < (int)(sizeof(drop) / sizeof(drop[0])); ++j) {
@@ -421,13 +453,13 @@ __device__ __forceinline__ bool refine_and_emit(TopkSmem& S, uint32_t lo, int k,
             drop[j] = rank >= need;
         }
     }
-    __syncthreads();  // every rank used the original indices
+    G.sync();  // every rank used the original indices
 #pragma unroll
     for (int j = 0; j < (int)(sizeof(drop) / sizeof(drop[0])); ++j) {
         const uint32_t a = tid + j * kTkThreads;
         if (a < cnt_b && drop[j]) S.reg_ip[bloc[a] >> 16][bloc[a] & 0xFFFFu] = -1;
     }
-    __syncthreads();
+    G.sync();
     auto kept = [&](uint32_t key, int ix) {
         const uint32_t d = key - lo;
         return above(d) || (in_bin(d) && ix >= 0);
@@ -444,7 +476,7 @@ __device__ __forceinline__ bool refine_and_emit(TopkSmem& S, uint32_t lo, int k,
         for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
         if (lane == 0) S.reg_gt[r] = (int)c;
     }
-    __syncthreads();
+    G.sync();
     for (int r = warp; r < nreg; r += kTkWarps) {
         uint32_t base = 0;
         for (int q = 0; q < r; ++q) base += (uint32_t)S.reg_gt[q];
@@ -475,23 +507,23 @@ __device__ __forceinline__ bool refine_and_emit(TopkSmem& S, uint32_t lo, int k,
 // Exact radix select over the row in global memory (the fallback): histogram passes of
 // 10 + 10 + 10 + 2 bits fix tau and the number of ties to keep, a scan finds the last kept tie,
 // then the kept keys are written in the same order as the fast path (region by region).
-__device__ __noinline__ void topk_global(TopkSmem& S, const float* row, int lo, int n, int k, int* out) {
-    const int tid = threadIdx.x;
+__device__ __noinline__ void topk_global(TopkSmem& S, const Grp& G, const float* row, int lo, int n, int k, int* out) {
+    const int tid = G.tid;
     uint32_t pval = 0, need = (uint32_t)k;
     int fixed = 32;
     while (fixed > 0) {
         const int width = fixed >= 10 ? 10 : fixed;
         const int sh = fixed - width;
         const int nbins = 1 << width;
-        __syncthreads();
-        clear_hist(S, nbins);
-        __syncthreads();
+        G.sync();
+        clear_hist(S, G, nbins);
+        G.sync();
         for (int e = lo + tid; e < n; e += kTkThreads) {
             const uint32_t key = score_key(row[e]);
             if (fixed >= 32 || (key >> fixed) == (pval >> fixed)) atomicAdd(&S.hist[(key >> sh) & (nbins - 1)], 1u);
         }
-        __syncthreads();
-        find_threshold_bin(S, nbins, need);
+        G.sync();
+        find_threshold_bin(S, G, nbins, need);
         need -= S.sel_gt;
         pval |= S.sel_bin << sh;
         fixed = sh;
@@ -505,9 +537,9 @@ __device__ __noinline__ void topk_global(TopkSmem& S, const float* row, int lo, 
         const int e = e0 + tid;
         const uint32_t eq = (e < n && score_key(row[e]) == tau) ? 1u : 0u;
         uint32_t total;
-        const uint32_t ex = block_excl_scan(S, eq, total);
+        const uint32_t ex = block_excl_scan(S, G, eq, total);
         if (eq && eq_seen + ex == ties - 1) S.sel_gt = (uint32_t)e + 1;  // the last kept tie
-        __syncthreads();
+        G.sync();
         eq_seen += total;
         if (eq_seen >= ties) {
             tie_end = (int)S.sel_gt;
@@ -525,7 +557,7 @@ __device__ __noinline__ void topk_global(TopkSmem& S, const float* row, int lo, 
             const uint32_t key = (mine && e >= lo && e < n) ? score_key(row[e]) : 0u;
             const bool keep = mine && e >= lo && e < n && (key > tau || (key == tau && e < tie_end));
             uint32_t total;
-            const uint32_t ex = block_excl_scan(S, keep ? 1u : 0u, total);
+            const uint32_t ex = block_excl_scan(S, G, keep ? 1u : 0u, total);
             if (keep) out[written + ex] = e;
             written += total;
         }
@@ -539,8 +571,8 @@ __device__ __forceinline__ uint32_t rank_target(long long m, long long n, int k)
 
 // Sample s4 evenly spaced float4 of float4 range [g_lo, g_hi) into keys[base .. base + 4*s4); all
 // of a thread's loads are issued before any is used.
-__device__ __forceinline__ void take_samples(uint32_t* keys, int base, const float4* row4, int g_lo, int g_hi, int e_lo,
-                                             int n, int s4) {
+__device__ __forceinline__ void take_samples(const Grp& G, uint32_t* keys, int base, const float4* row4, int g_lo,
+                                             int g_hi, int e_lo, int n, int s4) {
     constexpr int kPer = kTkMaxSample4 / kTkThreads;
     float4 v[kPer];
     int gg[kPer];
@@ -548,13 +580,13 @@ __device__ __forceinline__ void take_samples(uint32_t* keys, int base, const flo
     const unsigned long long step = ((unsigned long long)(g_hi - g_lo) << 32) / (unsigned)max(s4, 1);
 #pragma unroll
     for (int u = 0; u < kPer; ++u) {
-        const int i = threadIdx.x + u * kTkThreads;
+        const int i = G.tid + u * kTkThreads;
         gg[u] = g_lo + (int)(((unsigned long long)i * step) >> 32);
         v[u] = (i < s4 && gg[u] < g_hi) ? row4[gg[u]] : make_float4(0.f, 0.f, 0.f, 0.f);
     }
 #pragma unroll
     for (int u = 0; u < kPer; ++u) {
-        const int i = threadIdx.x + u * kTkThreads;
+        const int i = G.tid + u * kTkThreads;
         if (i >= s4) continue;
         const int g = gg[u];
         const float f[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
@@ -579,6 +611,7 @@ __global__ void __launch_bounds__(kTkThreads, 6) topk_kernel(const TopkParams P)
     extern __shared__ __align__(1024) uint8_t topk_smem[];
     TopkSmem& S = *reinterpret_cast<TopkSmem*>(topk_smem);
     const int r = blockIdx.x, tid = threadIdx.x, warp = tid >> 5;
+    const Grp G{tid};
     const int n = (int)row_length(P, r, tid == 0);
     const int lo = row_first_key(P, n), ne = n - lo;  // competing keys: [lo, n)
     const int k = P.k;
@@ -599,11 +632,11 @@ __global__ void __launch_bounds__(kTkThreads, 6) topk_kernel(const TopkParams P)
         uint32_t T0 = 0;
         if (ne > kTkCap) {
             if (attempt > 0) __syncthreads();
-            take_samples(S.cand_key, 0, row4, g0, n4, lo, n, s4);
-            T0 = sample_threshold(S, (int)m, rs);
+            take_samples(G, S.cand_key, 0, row4, g0, n4, lo, n, s4);
+            T0 = sample_threshold(S, G, (int)m, rs);
         }
         // ---- one streaming pass: scores >= T0 into the 4 warp regions
-        const uint32_t c = stream_collect(S, row4, g0, n4, lo, n, key_floor_float(T0), warp * kTkRegion);
+        const uint32_t c = stream_collect(S, G, row4, g0, n4, lo, n, key_floor_float(T0), warp * kTkRegion);
         if ((tid & 31) == 0) {
             S.reg_kp[warp] = S.cand_key + warp * kTkRegion;
             S.reg_ip[warp] = S.cand_idx + warp * kTkRegion;
@@ -620,27 +653,58 @@ __global__ void __launch_bounds__(kTkThreads, 6) topk_kernel(const TopkParams P)
             fits = fits && S.reg_gt[w] <= kTkRegion;
         }
         fits = fits && total >= (uint32_t)k;
-        done = fits && refine_and_emit(S, T0, k, out);
+        done = fits && refine_and_emit(S, G, T0, k, out);
         if (!done) rs = retarget(rs, total, m, k);
         if (tid == 0) {
             atomicAdd(&g_counters[0], attempt == 0 ? 1ull : 0ull);
             if (!done) atomicAdd(&g_counters[1 + 3 * attempt], 1ull);  // [1] first miss, [4] second miss
         }
     }
-    if (!done) topk_global(S, row, lo, n, k, out);
+    if (!done) topk_global(S, G, row, lo, n, k, out);
 }
 
-// Few long rows (decode): a cluster of kTkCluster CTAs per row.  Each CTA samples and streams
-// 1/kTkCluster of the row; the sample keys go to CTA 0, which sets the threshold, gathers every
-// CTA's candidate regions through distributed shared memory, then refines and writes the row.
-// Dynamic shared memory: sizeof(TopkSmem) + kTkCap * 8 bytes (CTA 0's gather buffer).
+// Few long rows (decode): a cluster of kTkCluster CTAs per row, each sampling and streaming
+// 1/kTkCluster of the row.  CTA 0 turns the samples (sent to it through distributed shared
+// memory) into the threshold T0, aimed at rank 2k so that a miss is rare, and into the scale of a
+// histogram of the candidates' key offsets from T0.  Every CTA streams its segment into its own
+// warp regions and adds each candidate to CTA 0's histogram (distributed shared-memory atomics).
+// The refinement is then spread over the cluster: CTA 0 finds the bin that holds the k-th key
+// (narrowing it with further distributed histogram rounds while it holds more than kTkBndMax
+// keys), the CTAs send that bin's members to CTA 0, which ranks them and broadcasts the exact
+// cutoff (key, index); each CTA counts its kept keys per region, the counts are exchanged, and
+// every CTA writes its own kept keys at its offsets.  The output order is the one-CTA kernel's:
+// region w of the row is region w of CTA 0, then of CTA 1, ... (contiguous segments).  A miss
+// (the candidates do not hold k keys, or a region overflows) re-aims and streams once more; a
+// final bin of more than kTkBndMax equal keys, or a second miss, takes the exact radix select
+// on CTA 0.  Dynamic shared memory: sizeof(TopkSmem).
+constexpr int kTkBndMax = 256;
+
+struct TopkClusterShared {
+    int kept[kTkCluster][kTkWarps];  // kept keys per (CTA, region); every CTA writes its row into all
+    uint32_t bkey[kTkBndMax];         // boundary-bin members (CTA 0)
+    int bidx[kTkBndMax];
+    int bn;                           // boundary-bin members received (CTA 0)
+    uint32_t T0, sh;                  // threshold key and candidate-histogram shift (broadcast)
+    uint32_t pv, need, cnt_b;         // refinement state (broadcast): prefix of the bin, keys still
+    int fixed;                        // needed from it, its size, low offset bits not yet fixed
+    uint32_t cut_key;                 // last kept key of the boundary bin (broadcast)
+    int cut_idx;
+};
+
+__device__ __forceinline__ uint32_t rank_target_2k(long long m, long long n, int k) {
+    // aim at rank 2k of the row, i.e. rank 2k * m / n of the m samples
+    return (uint32_t)max(1LL, min(m - 1, (2LL * k * m + n - 1) / n));
+}
+
 __global__ void __launch_bounds__(kTkThreads, 1) topk_cluster_kernel(const TopkParams P) {
     extern __shared__ __align__(1024) uint8_t topk_smem[];
+    __shared__ TopkClusterShared C;
     __shared__ int src_cnt[kTkMaxRegions];
     TopkSmem& S = *reinterpret_cast<TopkSmem*>(topk_smem);
     cg::cluster_group cluster = cg::this_cluster();
     const int crank = (int)cluster.block_rank();
     const int r = blockIdx.x / kTkCluster, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const Grp G{tid};
     const int n = (int)row_length(P, r, tid == 0 && crank == 0);
     const int lo = row_first_key(P, n), ne = n - lo;  // competing keys: [lo, n)
     const int k = P.k;
@@ -657,113 +721,179 @@ __global__ void __launch_bounds__(kTkThreads, 1) topk_cluster_kernel(const TopkP
     const int seg = ((n4 - (gw & ~31) + kTkCluster - 1) / kTkCluster + 31) & ~31;
     const int g_lo = min(n4, max(gw, (gw & ~31) + crank * seg)), g_hi = min(n4, (gw & ~31) + (crank + 1) * seg);
     TopkSmem* S0 = cluster.map_shared_rank(&S, 0);
+    TopkClusterShared* C0 = cluster.map_shared_rank(&C, 0);
 
     const int s4 = sample_count4(n4 - gw, kTkCluster);  // per CTA
     const long long m = 4LL * s4 * kTkCluster;
-    uint32_t rs = (uint32_t)rank_target(m, ne, k);
+    uint32_t rs = rank_target_2k(m, ne, k);
     bool done = false;
-    for (int attempt = 0; attempt < 2; ++attempt) {
-        // ---- samples of every segment into CTA 0, which computes T0 and hands it to every CTA
-        take_samples(S0->cand_key, 4 * crank * s4, row4, g_lo, g_hi, lo, n, s4);
+    for (int attempt = 0; attempt < 2 && !done; ++attempt) {
+        // ---- samples of every segment into CTA 0, which sets T0 and the histogram scale
+        take_samples(G, S0->cand_key, 4 * crank * s4, row4, g_lo, g_hi, lo, n, s4);
         cluster.sync();
         if (crank == 0) {
-            const uint32_t t0 = sample_threshold(S, (int)m, rs);
-            if (tid < kTkCluster) cluster.map_shared_rank(&S, tid)->T0 = t0;
-        }
-        cluster.sync();
-        const uint32_t T0 = S.T0;
-
-        // ---- stream this CTA's segment into its warp regions
-        const uint32_t c = stream_collect(S, row4, g_lo, g_hi, lo, n, key_floor_float(T0), warp * kTkRegion);
-        if ((tid & 31) == 0) S.reg_gt[warp] = (int)c;
-        cluster.sync();
-
-        if (crank == 0) {
-            if (tid < kTkMaxRegions) src_cnt[tid] = cluster.map_shared_rank(&S, tid / kTkWarps)->reg_gt[tid % kTkWarps];
-            __syncthreads();
-            uint32_t total = 0;
-            bool fits = true;
-            for (int q = 0; q < kTkMaxRegions; ++q) {
-                total += (uint32_t)src_cnt[q];
-                fits = fits && src_cnt[q] <= kTkRegion;
-            }
-            fits = fits && total >= (uint32_t)k && total <= (uint32_t)kTkCap;
-            if (fits) {
-                // gather every CTA's regions into a local buffer, region-major (region w of CTA 0,
-                // of CTA 1, ...); region w of the row then stays one ascending run, as in the
-                // one-CTA kernel
-                uint32_t* gkey = reinterpret_cast<uint32_t*>(topk_smem + sizeof(TopkSmem));
-                int* gidx = reinterpret_cast<int*>(gkey + kTkCap);
-                __shared__ int src_pre[kTkMaxRegions + 1];
-                if (tid == 0) {
-                    int acc = 0;
-                    for (int q = 0; q < kTkMaxRegions; ++q) {  // q = warp * kTkCluster + cta
-                        src_pre[q] = acc;
-                        acc += src_cnt[(q % kTkCluster) * kTkWarps + q / kTkCluster];
-                    }
-                    src_pre[kTkMaxRegions] = acc;
-                }
-                __syncthreads();
-                // warp w copies source regions q = w, w + 4, ...: consecutive lanes read
-                // consecutive entries of one remote region (coalesced), four per lane in flight
-                for (int q = warp; q < kTkMaxRegions; q += kTkWarps) {
-                    const int c = q % kTkCluster, w = q / kTkCluster;
-                    const int cnt = src_pre[q + 1] - src_pre[q], dst0 = src_pre[q];
-                    const TopkSmem* Src = cluster.map_shared_rank(&S, c);
-                    const uint32_t* sk = Src->cand_key + w * kTkRegion;
-                    const int* si = Src->cand_idx + w * kTkRegion;
-                    for (int e0 = 0; e0 < cnt; e0 += 32 * kTkBatch) {
-                        uint32_t kk[kTkBatch];
-                        int ii[kTkBatch];
-#pragma unroll
-                        for (int j = 0; j < kTkBatch; ++j) {
-                            const int e = e0 + 32 * j + lane;
-                            if (e < cnt) {
-                                kk[j] = sk[e];
-                                ii[j] = si[e];
-                            }
-                        }
-#pragma unroll
-                        for (int j = 0; j < kTkBatch; ++j) {
-                            const int e = e0 + 32 * j + lane;
-                            if (e < cnt) {
-                                gkey[dst0 + e] = kk[j];
-                                gidx[dst0 + e] = ii[j];
-                            }
-                        }
-                    }
-                }
-                __syncthreads();
-                if (tid < kTkWarps) {
-                    S.reg_kp[tid] = gkey + src_pre[tid * kTkCluster];
-                    S.reg_ip[tid] = gidx + src_pre[tid * kTkCluster];
-                    S.reg_cnt[tid] = src_pre[(tid + 1) * kTkCluster] - src_pre[tid * kTkCluster];
-                }
-                if (tid == 0) S.nreg = kTkWarps;
-                __syncthreads();
-                done = refine_and_emit(S, T0, k, out);
-            }
-            if (tid == 0) {
-                atomicAdd(&g_counters[2], attempt == 0 ? 1ull : 0ull);
-                if (!done) atomicAdd(&g_counters[3 + 2 * attempt], 1ull);  // [3] first miss, [5] second miss
-                S.sel_gt = done ? 1u : 0u;
-                S.T0 = retarget(rs, total, m, k);
-            }
-            __syncthreads();
-            // tell every CTA whether to go again (and with which rank)
+            uint32_t kmax = 0;
+            const uint32_t t0 = sample_threshold(S, G, (int)m, rs, &kmax);
+            // bins of width 2^sh over [T0, kmax] fill at most half the histogram: keys up to twice
+            // the sampled range above T0 still get bins of their own
+            const uint32_t span = kmax > t0 ? kmax - t0 : 0u;
+            const uint32_t sh = (span >> 9) ? 32 - __clz(span >> 9) : 0;
+            clear_hist(S, G, kTkBins);
             if (tid < kTkCluster) {
-                TopkSmem* D = cluster.map_shared_rank(&S, tid);
-                D->sel_bin = S.sel_gt;
-                D->red[0] = S.T0;
+                TopkClusterShared* D = cluster.map_shared_rank(&C, tid);
+                D->T0 = t0;
+                D->sh = sh;
             }
         }
-        cluster.sync();  // CTA 0's gather of every region is complete; the verdict is everywhere
-        done = S.sel_bin != 0u;
-        rs = S.red[0];
-        if (done) break;
+        cluster.sync();  // T0 everywhere, CTA 0's histogram cleared
+        const uint32_t T0 = C.T0, sh = C.sh;
+
+        // ---- stream this CTA's segment into its warp regions and CTA 0's candidate histogram
+        const uint32_t c = stream_collect(S, G, row4, g_lo, g_hi, lo, n, key_floor_float(T0), warp * kTkRegion,
+                                          S0->hist, T0, (int)sh);
+        if (lane == 0) S.reg_gt[warp] = (int)c;
+        cluster.sync();
+        if (tid < kTkMaxRegions) src_cnt[tid] = cluster.map_shared_rank(&S, tid / kTkWarps)->reg_gt[tid % kTkWarps];
+        __syncthreads();
+        uint32_t total = 0;
+        bool fits = true;
+        for (int q = 0; q < kTkMaxRegions; ++q) {
+            total += (uint32_t)src_cnt[q];
+            fits = fits && src_cnt[q] <= kTkRegion;
+        }
+        fits = fits && total >= (uint32_t)k;  // uniform over the cluster
+        if (crank == 0 && tid == 0) {
+            atomicAdd(&g_counters[2], attempt == 0 ? 1ull : 0ull);
+            if (!fits && attempt == 0) atomicAdd(&g_counters[3], 1ull);  // first miss
+        }
+        if (!fits) {
+            rs = retarget(rs, total, m, k);
+            cluster.sync();  // every CTA has read the counts before the next attempt rewrites them
+            continue;
+        }
+
+        // ---- distributed refinement: the bin holding the k-th key, narrowed while it is large
+        if (crank == 0) {
+            find_threshold_bin(S, G, kTkBins, (uint32_t)k);
+            if (tid < kTkCluster) {
+                TopkClusterShared* D = cluster.map_shared_rank(&C, tid);
+                D->pv = S.sel_bin << sh;
+                D->fixed = (int)sh;
+                D->need = (uint32_t)k - S.sel_gt;
+                // a clamped top bin has no prefix: treat it as too large to resolve (exact fallback)
+                D->cnt_b = S.sel_bin == (uint32_t)kTkBins - 1u ? 0xFFFFFFFFu : S.hist[S.sel_bin];
+            }
+        }
+        cluster.sync();
+        while (C.cnt_b != 0xFFFFFFFFu && C.cnt_b > (uint32_t)kTkBndMax && C.fixed > 0) {  // uniform
+            const int fixed = C.fixed;
+            const uint32_t pv = C.pv;
+            const int sh2 = fixed > 10 ? fixed - 10 : 0;
+            const int nb = 1 << (fixed - sh2);
+            if (crank == 0) clear_hist(S, G, nb);
+            cluster.sync();
+            for (int w = 0; w < kTkWarps; ++w) {
+                const int cw = min(S.reg_gt[w], kTkRegion);
+                for (int e = tid; e < cw; e += kTkThreads) {
+                    const uint32_t d = S.cand_key[w * kTkRegion + e] - T0;
+                    if ((d >> fixed) == (pv >> fixed)) atomicAdd(&S0->hist[(d >> sh2) & (nb - 1)], 1u);
+                }
+            }
+            cluster.sync();
+            if (crank == 0) {
+                find_threshold_bin(S, G, nb, C.need);
+                if (tid < kTkCluster) {
+                    TopkClusterShared* D = cluster.map_shared_rank(&C, tid);
+                    D->need = C.need - S.sel_gt;
+                    D->cnt_b = S.hist[S.sel_bin];
+                    D->pv = pv | (S.sel_bin << sh2);
+                    D->fixed = sh2;
+                }
+            }
+            cluster.sync();
+        }
+        if (C.cnt_b > (uint32_t)kTkBndMax) break;  // more equal keys than the ranking handles: exact fallback
+        const int fixed = C.fixed;
+        const uint32_t pv = C.pv;
+        auto in_bin = [&](uint32_t d) { return fixed >= 32 || (d >> fixed) == (pv >> fixed); };
+        auto above = [&](uint32_t d) { return fixed < 32 && (d >> fixed) > (pv >> fixed); };
+        // ---- the boundary bin's members to CTA 0, which ranks them and broadcasts the cutoff
+        if (crank == 0 && tid == 0) C.bn = 0;
+        cluster.sync();
+        for (int w = 0; w < kTkWarps; ++w) {
+            const int cw = min(S.reg_gt[w], kTkRegion);
+            for (int e = tid; e < cw; e += kTkThreads) {
+                const uint32_t key = S.cand_key[w * kTkRegion + e];
+                if (in_bin(key - T0)) {
+                    const int p = atomicAdd(&C0->bn, 1);
+                    if (p < kTkBndMax) {
+                        C0->bkey[p] = key;
+                        C0->bidx[p] = S.cand_idx[w * kTkRegion + e];
+                    }
+                }
+            }
+        }
+        cluster.sync();
+        if (crank == 0) {
+            const int bn = min(C.bn, kTkBndMax);
+            const uint32_t need = C.need;
+            for (int a = tid; a < bn; a += kTkThreads) {
+                const uint32_t ka = C.bkey[a];
+                const int ia = C.bidx[a];
+                uint32_t rank = 0;
+                for (int b = 0; b < bn; ++b) {
+                    const uint32_t kb = C.bkey[b];
+                    rank += (kb > ka) || (kb == ka && C.bidx[b] < ia);
+                }
+                if (rank == need - 1u)  // exactly one member: the last kept one
+                    for (int q = 0; q < kTkCluster; ++q) {
+                        TopkClusterShared* D = cluster.map_shared_rank(&C, q);
+                        D->cut_key = ka;
+                        D->cut_idx = ia;
+                    }
+            }
+        }
+        cluster.sync();
+        const uint32_t cut_key = C.cut_key;
+        const int cut_idx = C.cut_idx;
+        auto kept = [&](uint32_t key, int ix) {
+            const uint32_t d = key - T0;
+            return above(d) || (in_bin(d) && (key > cut_key || (key == cut_key && ix <= cut_idx)));
+        };
+        // ---- kept keys per region, exchanged; each CTA writes its own at the row's offsets
+        {
+            const int cw = min(S.reg_gt[warp], kTkRegion);
+            uint32_t cntk = 0;
+            for (int e = lane; e < cw; e += 32)
+                cntk += kept(S.cand_key[warp * kTkRegion + e], S.cand_idx[warp * kTkRegion + e]);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) cntk += __shfl_xor_sync(0xffffffffu, cntk, o);
+            if (lane < kTkCluster) cluster.map_shared_rank(&C, lane)->kept[crank][warp] = (int)cntk;
+        }
+        cluster.sync();
+        {
+            uint32_t base = 0;
+            for (int w = 0; w < warp; ++w)
+                for (int q = 0; q < kTkCluster; ++q) base += (uint32_t)C.kept[q][w];
+            for (int q = 0; q < crank; ++q) base += (uint32_t)C.kept[q][warp];
+            const int cw = min(S.reg_gt[warp], kTkRegion);
+            for (int e0 = 0; e0 < cw; e0 += 32) {
+                const int e = e0 + lane;
+                const int ix = e < cw ? S.cand_idx[warp * kTkRegion + e] : 0;
+                const bool keep = e < cw && kept(S.cand_key[warp * kTkRegion + e], ix);
+                const uint32_t bk = __ballot_sync(0xffffffffu, keep);
+                if (keep) out[base + __popc(bk & ((1u << lane) - 1u))] = ix;
+                base += __popc(bk);
+            }
+        }
+        done = true;
     }
-    if (crank == 0 && !done) topk_global(S, row, lo, n, k, out);
-    cluster.sync();  // peers keep their shared memory alive until CTA 0 is done with it
+    if (!done && crank == 0) {
+        if (tid == 0) atomicAdd(&g_counters[5], 1ull);  // exact fallback
+        topk_global(S, G, row, lo, n, k, out);
+    }
+    cluster.sync();  // peers keep their shared memory alive until every remote access is done
 }
+
 
 }  // namespace dsa

@@ -252,8 +252,9 @@ dsa_status dsa_profile_end(int64_t *launches, double *total_ms);
  * Diagnostic path counters, accumulated on the device since load or the last reset:
  *   [0] top-k rows handled by the one-CTA-per-row kernel; [1] of those, rows whose first sampled
  *   threshold missed (a second estimate and pass followed); [4] rows whose second estimate also
- *   missed (exact radix select over the row); [2], [3], [5] the same for rows handled by a CTA
- *   cluster.  Copies up to n counters (n <= DSA_NUM_COUNTERS) into out after synchronising the
+ *   missed (exact radix select over the row); [2] rows handled by a CTA cluster (few long rows,
+ *   decode), [3] of those, rows whose first threshold missed, [5] rows that took the exact radix
+ *   select on the cluster's first CTA (a second miss, or more than 256 equal keys at the cutoff).  Copies up to n counters (n <= DSA_NUM_COUNTERS) into out after synchronising the
  *   device; if reset != 0 the counters are zeroed afterwards.  Returns DSA_ERR_CUDA on failure.
  */
 #define DSA_NUM_COUNTERS 8

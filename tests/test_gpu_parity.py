@@ -624,3 +624,67 @@ def test_decode_sixteen_heads_per_kv_group(cuda_ok):
         assert mm["structural"] == 0 and mm["out_of_band"] == 0, (b, mm)
         own, _ = oracle.sparse_attn_rows(bits(q[b:b + 1]), k_all, v_all, got_idx[b:b + 1], scale)
         assert_output_ok(got_out[b:b + 1], own, f"decode G=16 b={b}")
+
+
+@pytest.mark.parametrize("kind,k,window", [("gauss", 2048, 0), ("gauss", 300, 0), ("ties", 2048, 0),
+                                           ("zeros", 2048, 0), ("gauss", 2048, 20000), ("frames", 2048, 0),
+                                           ("gauss", 4096, 0), ("decoy", 2048, 0)])
+def test_topk_many_long_rows_exact_order(cuda_ok, kind, k, window):
+    """A launch of many long rows (more than one per SM, as a prefill chunk) through the one-CTA
+    kernel (the path counter proves it): every row equals the oracle's set in the documented
+    order, entry by entry.  Gaussian scores, frame-correlated scores, heavy integer ties (the
+    re-aimed second pass and the exact fallback), signed zeros, a sliding window, k at the
+    candidate capacity, and decoys (raised scores at a regular stride of 4-key groups, a pattern
+    that biases the sampled threshold)."""
+    rng = np.random.default_rng(23 + k + window)
+    rows, q_pos0 = 400, 60000 if kind == "decoy" else 30000
+    n_max = q_pos0 + rows
+    ld = (n_max + 3) // 4 * 4
+    if kind == "gauss":
+        s = (rng.standard_normal((rows, ld)) * 10).astype(np.float32)
+    elif kind == "frames":                     # blocks of 512 keys sharing an offset
+        s = (rng.standard_normal((rows, ld)) + np.repeat(rng.standard_normal((rows, ld // 512 + 1)) * 3, 512,
+                                                         axis=1)[:, :ld]).astype(np.float32)
+    elif kind == "ties":
+        s = rng.integers(-2, 3, size=(rows, ld)).astype(np.float32)
+    elif kind == "decoy":
+        s = rng.standard_normal((rows, ld)).astype(np.float32)
+        g = np.arange(ld // 4)
+        s.reshape(rows, -1, 4)[:, g % 14 == 0, :] += 40.0
+    else:
+        s = np.where(rng.random((rows, ld)) < 0.5, np.float32(0.0), np.float32(-0.0))
+        s[:, ::13] = 2.0
+    idx = torch.full((rows, k), -5, dtype=torch.int32, device="cuda")
+    dsa.read_counters(reset=True)
+    dsa.dsa_topk(torch.from_numpy(s).cuda(), q_pos0, k, idx, window=window)
+    assert dsa.sync_status() == dsa.DSA_OK
+    cnt = dsa.read_counters(reset=True)
+    assert cnt["topk_rows"] == rows and cnt["topk_cluster_rows"] == 0, cnt
+    n = q_pos0 + np.arange(rows) + 1
+    want, _ = oracle.topk_rows(s.astype(np.float64), n, k, window=window)
+    got = idx.cpu().numpy()
+    for r in range(rows):
+        lo = max(0, int(n[r]) - window) if window > 0 else 0
+        expect = canonical_order(want[r], int(n[r]) - lo, lo, k)
+        assert got[r].tolist() == expect, (kind, k, window, r)
+    if kind in ("ties", "zeros"):
+        assert cnt["topk_retry"] > 0 and cnt["topk_global"] > 0   # both fallback passes ran
+
+
+def test_topk_cluster_and_one_cta_kernels_agree(cuda_ok):
+    """The same long rows through the one-CTA kernel (a launch of many rows) and the cluster
+    kernel (a few rows per launch, 8 CTAs each) give identical outputs, entry by entry."""
+    rng = np.random.default_rng(29)
+    rows, q_pos0, k = 300, 40000, 2048
+    ld = (q_pos0 + rows + 3) // 4 * 4
+    s = torch.from_numpy((rng.standard_normal((rows, ld)) * 5).astype(np.float32)).cuda()
+    a = torch.empty((rows, k), dtype=torch.int32, device="cuda")
+    b = torch.empty_like(a)
+    dsa.read_counters(reset=True)
+    dsa.dsa_topk(s, q_pos0, k, a)
+    for r0 in range(0, rows, 12):                        # 12 rows x 8 CTAs <= 2 per SM: clusters
+        dsa.dsa_topk(s[r0:r0 + 12], q_pos0 + r0, k, b[r0:r0 + 12])
+    assert dsa.sync_status() == dsa.DSA_OK
+    cnt = dsa.read_counters(reset=True)
+    assert cnt["topk_rows"] == rows and cnt["topk_cluster_rows"] == rows, cnt
+    assert torch.equal(a, b)

@@ -179,13 +179,16 @@ dsa_status launch_indexer_t(const CUtensorMap& mq, const CUtensorMap& mk, const 
     return launch_status();
 }
 
+// Query tokens per indexer work block: a 256-column tile of whole tokens (prefill), or the one new
+// token of a sequence (decode).
+int indexer_tb(int HI, bool decode) { return decode ? 1 : 256 / HI; }
+
 // Shared by dsa_index (P = 1) and the decode step (P = B, one query each).
 dsa_status run_indexer(const void* qI, const void* kI, const __nv_bfloat16* w, int P_, int Lq, int64_t q_pos0,
                        const int* ctx_len, int64_t Lk, int HI, float* scores, int64_t ld, cudaStream_t s,
                        int64_t window = 0, const IndexerParams* append = nullptr) {
     const bool decode = ctx_len != nullptr;
-    const int BN = decode ? HI : 256;
-    const int TB = BN / HI;
+    const int TB = indexer_tb(HI, decode);
     IndexerParams P{};
     P.P = P_;
     P.Lq = Lq;
@@ -222,7 +225,7 @@ dsa_status run_indexer(const void* qI, const void* kI, const __nv_bfloat16* w, i
     }
     P.num_units = P_ * P.num_qb * P.nsplit;
     const uint64_t qrows = (uint64_t)Lq * HI;
-    const uint32_t qbox = (uint32_t)std::min<uint64_t>(BN, qrows);
+    const uint32_t qbox = (uint32_t)std::min<uint64_t>((uint64_t)TB * HI, qrows);  // one block's qI rows
     const uint32_t kbox = (uint32_t)std::min<int64_t>(kIdxBM, Lk);
     P.q_box_bytes = qbox * 128u;
     P.k_box_bytes = kbox * 128u;
@@ -353,13 +356,18 @@ DecodeWs decode_ws_layout(int64_t Lmax, int B, int Hq, int topk, bool need_idx) 
 
 int64_t prefill_ld(int64_t L) { return (int64_t)align_up((size_t)L, 4); }
 
-// Query rows per chunk for a workspace of ws_bytes holding C score rows of ld floats (and, with
-// idx_per_row > 0, an index region of C rows after them at a 256-byte boundary): the most that
+// Bytes of a chunk of C query rows: C score rows of ld floats, then (idx_per_row > 0) C index
+// rows starting at a 256-byte boundary.
+size_t chunk_bytes(int64_t C, int64_t ld, int64_t idx_per_row) {
+    return align_up((size_t)C * ld * 4, 256) + (size_t)C * idx_per_row * 4;
+}
+
+// Query rows per chunk for a workspace of ws_bytes laid out as chunk_bytes says: the most that
 // fit, whole query blocks of TB rows unless the chunk covers every remaining row.  0 = too small.
 int64_t chunk_rows(size_t ws_bytes, int64_t ld, int64_t idx_per_row, int64_t rows, int TB) {
-    const size_t per_row = (size_t)ld * 4 + (size_t)idx_per_row * 4;
+    const size_t per_row = (size_t)(ld + idx_per_row) * 4;
     int64_t C = std::min<int64_t>(rows, (int64_t)(ws_bytes / per_row));
-    while (C > 0 && align_up((size_t)C * ld * 4, 256) + (size_t)C * idx_per_row * 4 > ws_bytes) --C;
+    while (C > 0 && chunk_bytes(C, ld, idx_per_row) > ws_bytes) --C;
     if (C < rows && C >= TB) C = C / TB * TB;
     return C;
 }
@@ -490,7 +498,7 @@ size_t dsa_workspace_size(int op, int64_t L, int B, int Hq, int HI, int topk) {
         int64_t rows = (int64_t(4) << 30) / (ld * 4);
         rows = std::max<int64_t>(256, rows / 256 * 256);
         rows = std::min<int64_t>(rows, L);
-        return align_up((size_t)rows * ld * 4, 256) + align_up((size_t)rows * topk * 4, 256);
+        return align_up(chunk_bytes(rows, ld, topk), 256);
     }
     case DSA_OP_DECODE:
         if (B <= 0 || Hq <= 0) return 0;
@@ -513,7 +521,7 @@ dsa_status dsa_indexer_kl(const void* q, const void* k, const void* qI, const vo
         return DSA_ERR_UNSUPPORTED;
     if (!ws || !aligned16(ws)) return DSA_ERR_WORKSPACE;
     const int64_t ld = prefill_ld(L);
-    const int TB = 256 / HI;
+    const int TB = indexer_tb(HI, false);
     const int64_t C = chunk_rows(ws_bytes, ld, 0, L, TB);
     if (C < std::min<int64_t>(L, TB)) return DSA_ERR_WORKSPACE;
     float* scores = static_cast<float*>(ws);
@@ -560,8 +568,9 @@ dsa_status dsa_prefill_rows(const void* q, const void* k, const void* v, const v
         return DSA_ERR_UNSUPPORTED;
     if (!ws || !aligned16(ws)) return DSA_ERR_WORKSPACE;
     const int64_t ld = prefill_ld(Lk);
-    const int TB = 256 / HI;
-    const int64_t C = chunk_rows(ws_bytes, ld, idx_out ? 0 : topk, rows, TB);
+    const int TB = indexer_tb(HI, false);
+    const int64_t ipr = idx_out ? 0 : topk;
+    const int64_t C = chunk_rows(ws_bytes, ld, ipr, rows, TB);
     if (C < std::min<int64_t>(rows, TB)) return DSA_ERR_WORKSPACE;
     float* scores = static_cast<float*>(ws);
     int32_t* idx_ws = idx_out ? nullptr
@@ -666,8 +675,8 @@ dsa_status dsa_decode(const void* q, const void* qI, const void* w, const void* 
     app.cache_kI = static_cast<uint4*>(kI_cache);
     app.kv16 = Hkv * D / 8;
     app.kI16 = dI / 8;
-    st = run_indexer(qI, kI_cache, static_cast<const __nv_bfloat16*>(w), B, 1, 0, ctx_len, Lmax, HI, scores, ld, s,
-                     0, &app);
+    st = run_indexer(qI, kI_cache, static_cast<const __nv_bfloat16*>(w), B, 1, 0, ctx_len, Lmax, HI, scores, ld, s, 0,
+                     &app);
     if (st != DSA_OK) return st;
     st = run_topk(scores, ld, B, 0, ctx_len, Lmax, topk, idx, s);
     if (st != DSA_OK) return st;

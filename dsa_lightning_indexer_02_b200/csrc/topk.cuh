@@ -504,10 +504,11 @@ __device__ __forceinline__ bool refine_and_emit(TopkSmem& S, const Grp& G, uint3
     return true;
 }
 
-// Exact radix select over the row in global memory (the fallback): histogram passes of
+// Exact radix select over the row (the fallback; row(e) gives the score of key e): histogram passes of
 // 10 + 10 + 10 + 2 bits fix tau and the number of ties to keep, a scan finds the last kept tie,
 // then the kept keys are written in the same order as the fast path (region by region).
-__device__ __noinline__ void topk_global(TopkSmem& S, const Grp& G, const float* row, int lo, int n, int k, int* out) {
+template <class RowAt>
+__device__ __noinline__ void topk_global(TopkSmem& S, const Grp& G, RowAt row, int lo, int n, int k, int* out) {
     const int tid = G.tid;
     uint32_t pval = 0, need = (uint32_t)k;
     int fixed = 32;
@@ -519,7 +520,7 @@ __device__ __noinline__ void topk_global(TopkSmem& S, const Grp& G, const float*
         clear_hist(S, G, nbins);
         G.sync();
         for (int e = lo + tid; e < n; e += kTkThreads) {
-            const uint32_t key = score_key(row[e]);
+            const uint32_t key = score_key(row(e));
             if (fixed >= 32 || (key >> fixed) == (pval >> fixed)) atomicAdd(&S.hist[(key >> sh) & (nbins - 1)], 1u);
         }
         G.sync();
@@ -535,7 +536,7 @@ __device__ __noinline__ void topk_global(TopkSmem& S, const Grp& G, const float*
     int tie_end = n;  // keys == tau with index < tie_end are kept
     for (int e0 = lo; e0 < n; e0 += kTkThreads) {
         const int e = e0 + tid;
-        const uint32_t eq = (e < n && score_key(row[e]) == tau) ? 1u : 0u;
+        const uint32_t eq = (e < n && score_key(row(e)) == tau) ? 1u : 0u;
         uint32_t total;
         const uint32_t ex = block_excl_scan(S, G, eq, total);
         if (eq && eq_seen + ex == ties - 1) S.sel_gt = (uint32_t)e + 1;  // the last kept tie
@@ -554,7 +555,7 @@ __device__ __noinline__ void topk_global(TopkSmem& S, const Grp& G, const float*
             const int p = p0 + (tid >> 5);
             const int e = p * 32 + (tid & 31);
             const bool mine = (p & 3) == region;
-            const uint32_t key = (mine && e >= lo && e < n) ? score_key(row[e]) : 0u;
+            const uint32_t key = (mine && e >= lo && e < n) ? score_key(row(e)) : 0u;
             const bool keep = mine && e >= lo && e < n && (key > tau || (key == tau && e < tie_end));
             uint32_t total;
             const uint32_t ex = block_excl_scan(S, G, keep ? 1u : 0u, total);
@@ -660,7 +661,7 @@ __global__ void __launch_bounds__(kTkThreads, 6) topk_kernel(const TopkParams P)
             if (!done) atomicAdd(&g_counters[1 + 3 * attempt], 1ull);  // [1] first miss, [4] second miss
         }
     }
-    if (!done) topk_global(S, G, row, lo, n, k, out);
+    if (!done) topk_global(S, G, [row](int e) { return row[e]; }, lo, n, k, out);
 }
 
 // Few long rows (decode): a cluster of kTkCluster CTAs per row, each sampling and streaming
@@ -696,30 +697,29 @@ __device__ __forceinline__ uint32_t rank_target_2k(long long m, long long n, int
     return (uint32_t)max(1LL, min(m - 1, (2LL * k * m + n - 1) / n));
 }
 
-__global__ void __launch_bounds__(kTkThreads, 1) topk_cluster_kernel(const TopkParams P) {
-    extern __shared__ __align__(1024) uint8_t topk_smem[];
-    __shared__ TopkClusterShared C;
-    __shared__ int src_cnt[kTkMaxRegions];
-    TopkSmem& S = *reinterpret_cast<TopkSmem*>(topk_smem);
-    cg::cluster_group cluster = cg::this_cluster();
-    const int crank = (int)cluster.block_rank();
-    const int r = blockIdx.x / kTkCluster, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const Grp G{tid};
-    const int n = (int)row_length(P, r, tid == 0 && crank == 0);
-    const int lo = row_first_key(P, n), ne = n - lo;  // competing keys: [lo, n)
-    const int k = P.k;
-    int* out = P.idx + (long long)r * k;
-    if (ne <= k) {  // uniform over the cluster
-        if (crank == 0)
-            for (int j = tid; j < k; j += kTkThreads) out[j] = j < ne ? lo + j : -1;
-        return;
-    }
-    const float* row = P.scores + (long long)r * P.ld;
-    const float4* row4 = reinterpret_cast<const float4*>(row);
+// Float4 groups [g_lo, g_hi) of a row's competing keys [lo, n) that CTA `crank` of a cluster
+// samples and streams: segments of whole groups of 4 pieces (32 float4), so that regions keep
+// their meaning across CTAs.  Returns the segment length in float4 groups.
+__device__ __forceinline__ int cluster_segment(int lo, int n, int crank, int& g_lo, int& g_hi) {
     const int n4 = (n + 3) >> 2, gw = lo >> 2;
-    // segments of whole groups of 4 pieces (32 float4), so regions keep their meaning across CTAs
     const int seg = ((n4 - (gw & ~31) + kTkCluster - 1) / kTkCluster + 31) & ~31;
-    const int g_lo = min(n4, max(gw, (gw & ~31) + crank * seg)), g_hi = min(n4, (gw & ~31) + (crank + 1) * seg);
+    g_lo = min(n4, max(gw, (gw & ~31) + crank * seg));
+    g_hi = min(n4, (gw & ~31) + (crank + 1) * seg);
+    return seg;
+}
+
+// One row's selection by the cluster (every thread of every CTA calls it): ne = n - lo > k.
+// row4[g] is the row's float4 group g (this CTA reads its segment [g_lo, g_hi)); row_at(e) gives
+// any key's score to CTA 0's exact fallback.
+template <class RowAt>
+__device__ __forceinline__ void cluster_select(TopkSmem& S, TopkClusterShared& C, int* src_cnt,
+                                               cg::cluster_group& cluster, const float4* row4, int g_lo, int g_hi,
+                                               int lo, int n, int k, int* out, RowAt row_at) {
+    const int crank = (int)cluster.block_rank();
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const Grp G{tid};
+    const int ne = n - lo;
+    const int n4 = (n + 3) >> 2, gw = lo >> 2;
     TopkSmem* S0 = cluster.map_shared_rank(&S, 0);
     TopkClusterShared* C0 = cluster.map_shared_rank(&C, 0);
 
@@ -890,9 +890,33 @@ __global__ void __launch_bounds__(kTkThreads, 1) topk_cluster_kernel(const TopkP
     }
     if (!done && crank == 0) {
         if (tid == 0) atomicAdd(&g_counters[5], 1ull);  // exact fallback
-        topk_global(S, G, row, lo, n, k, out);
+        topk_global(S, G, row_at, lo, n, k, out);
     }
     cluster.sync();  // peers keep their shared memory alive until every remote access is done
+}
+
+__global__ void __launch_bounds__(kTkThreads, 1) topk_cluster_kernel(const TopkParams P) {
+    extern __shared__ __align__(1024) uint8_t topk_smem[];
+    __shared__ TopkClusterShared C;
+    __shared__ int src_cnt[kTkMaxRegions];
+    TopkSmem& S = *reinterpret_cast<TopkSmem*>(topk_smem);
+    cg::cluster_group cluster = cg::this_cluster();
+    const int crank = (int)cluster.block_rank();
+    const int r = blockIdx.x / kTkCluster, tid = threadIdx.x;
+    const int n = (int)row_length(P, r, tid == 0 && crank == 0);
+    const int lo = row_first_key(P, n), ne = n - lo;  // competing keys: [lo, n)
+    const int k = P.k;
+    int* out = P.idx + (long long)r * k;
+    if (ne <= k) {  // uniform over the cluster
+        if (crank == 0)
+            for (int j = tid; j < k; j += kTkThreads) out[j] = j < ne ? lo + j : -1;
+        return;
+    }
+    const float* row = P.scores + (long long)r * P.ld;
+    int g_lo, g_hi;
+    cluster_segment(lo, n, crank, g_lo, g_hi);
+    cluster_select(S, C, src_cnt, cluster, reinterpret_cast<const float4*>(row), g_lo, g_hi, lo, n, k, out,
+                   [row](int e) { return row[e]; });
 }
 
 

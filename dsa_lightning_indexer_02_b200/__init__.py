@@ -49,6 +49,7 @@ _SIGS = {
     "dsa_topk": (_i, [_p, _i64, _i, _i64, _i, _p, _p, _sz, _p]),
     "dsa_topk_window": (_i, [_p, _i64, _i, _i64, _i, _i64, _p, _p]),
     "dsa_sparse_attn": (_i, [_p, _p, _p, _p, _i, _i64, _i64, _i, _i, _i, _i, _f, _p, _p, _p]),
+    "dsa_sparse_attn_dedup": (_i, [_p, _p, _p, _p, _i, _i64, _i64, _i, _i, _i, _i, _f, _p, _p, _p]),
     "dsa_prefill": (_i, [_p, _p, _p, _p, _p, _p, _i64, _i, _i, _i, _i, _i, _i, _f, _p, _p, _p, _sz, _p]),
     "dsa_prefill_rows": (_i, [_p, _p, _p, _p, _p, _p, _i64, _i64, _i, _i, _i, _i, _i, _i, _i64, _f, _p, _p, _p,
                               _sz, _p]),
@@ -62,6 +63,7 @@ _SIGS = {
     "dsa_indexer_kl": (_i, [_p, _p, _p, _p, _p, _i64, _i, _i, _i, _i, _i, _f, _p, _p, _sz, _p]),
     "dsa_workspace_size": (_sz, [_i, _i64, _i, _i, _i, _i]),
     "dsa_sync_status": (_i, [_p]),
+    "dsa_error_site": (ctypes.c_uint, []),
     "dsa_profile_begin": (None, []),
     "dsa_profile_end": (_i, [_p, _p]),
     "dsa_launch_count": (_i64, []),
@@ -207,6 +209,22 @@ def dsa_sparse_attn(q, k, v, idx, q_pos0: int, scale: float, out, lse=None, stre
     _check(st, "dsa_sparse_attn")
 
 
+def dsa_sparse_attn_dedup(q, k, v, idx, q_pos0: int, scale: float, out, lse=None, stream=None) -> None:
+    """dsa_sparse_attn computed per block of adjacent rows over the union of their index sets."""
+    import torch
+    bf = torch.bfloat16
+    _need(q, bf, "q", (None, None, None))
+    Lq, Hq, D = q.shape
+    _need(k, bf, "k", (None, None, D))
+    _need(v, bf, "v", tuple(k.shape)), _need(idx, torch.int32, "idx", (Lq, None)), _need(out, bf, "out", (Lq, Hq, D))
+    if lse is not None:
+        _need(lse, torch.float32, "lse", (Lq, Hq))
+    _on_device(q=q, k=k, v=v, idx=idx, out=out, lse=lse)
+    st = _lib.dsa_sparse_attn_dedup(_ptr(q), _ptr(k), _ptr(v), _ptr(idx), Lq, k.shape[0], q_pos0, Hq, k.shape[1], D,
+                                    idx.shape[1], float(scale), _ptr(out), _ptr(lse), _stream(stream))
+    _check(st, "dsa_sparse_attn_dedup")
+
+
 def _prefill_operands(q, k, v, qI, kI, w, out, idx, topk, key_rows, names):
     """Shapes shared by the prefill entry points: q/qI/w/out/idx hold the same query rows, k/v/kI
     at least `key_rows` key rows."""
@@ -308,6 +326,11 @@ def dsa_decode(q, qI, w, k_new, v_new, kI_new, k_cache, v_cache, kI_cache, ctx_l
 
 def sync_status(stream=None) -> int:
     return int(_lib.dsa_sync_status(_stream(stream)))
+
+
+def error_site() -> int:
+    """Site code (and loop index) of the last device error recorded; 0 if none."""
+    return int(_lib.dsa_error_site())
 
 
 def profile_begin() -> None:

@@ -9,7 +9,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 SRC = os.path.join(HERE, "csrc", "dsa_lib.cu")
 LIB = os.path.join(HERE, "libdsa.so")
-DEPS = [os.path.join(HERE, "csrc", f) for f in ("dsa_lib.cu", "ptx.cuh", "indexer.cuh", "topk.cuh", "attn.cuh", "kl.cuh")]
+DEPS = [os.path.join(HERE, "csrc", f) for f in ("dsa_lib.cu", "ptx.cuh", "indexer.cuh", "topk.cuh", "attn.cuh", "attn_dedup.cuh", "kl.cuh")]
 DEPS.append(os.path.join(ROOT, "include", "dsa.h"))
 
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",

@@ -12,6 +12,7 @@
 #include <vector>
 
 #include "attn.cuh"
+#include "attn_dedup.cuh"
 #include "kl.cuh"
 #include "dsa.h"
 #include "indexer.cuh"
@@ -301,6 +302,47 @@ dsa_status launch_attn_t(const AttnParams& P, cudaStream_t s) {
     return launch_status();
 }
 
+// ------------------------------------------------------------------ dedup attention launch
+// q bf16 [T][Hq][128] as a 3D map {128, Hq, T}; box {64, G, TBA}: the 128 (token, head) rows of one
+// KV group and block, one 64-dim half per load, 128-byte swizzle.
+bool make_dedup_q_map(CUtensorMap* m, const void* q, int T, int Hq, int G, int TBA) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)kAttnD, (cuuint64_t)Hq, (cuuint64_t)T};
+    cuuint64_t strides[2] = {(cuuint64_t)kAttnD * 2, (cuuint64_t)Hq * kAttnD * 2};
+    cuuint32_t box[3] = {64, (cuuint32_t)G, (cuuint32_t)TBA};
+    cuuint32_t es[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(q), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int G>
+dsa_status launch_dedup_t(const CUtensorMap& qm, const DedupParams& P, cudaStream_t s) {
+    auto kern = attn_dedup_kernel<G>;
+    static DeviceFlags attr_set;
+    if (!set_smem_limit(kern, kDdSmemBytes, attr_set)) return DSA_ERR_CUDA;
+    LaunchScope ls(K_ATTN, s);
+    kern<<<P.nblk * P.Hkv, kDdThreads, kDdSmemBytes, s>>>(qm, P);
+    return launch_status();
+}
+
+// Query heads per KV group the dedup kernel supports: 128 / G adjacent tokens fill one 128-row tile.
+bool dedup_supported(int Hq, int Hkv) { return Hkv > 0 && Hq % Hkv == 0 && (Hq / Hkv == 8 || Hq / Hkv == 16); }
+
+dsa_status run_attn_dedup(const void* q, DedupParams P, cudaStream_t s) {
+    const int G = P.Hq / P.Hkv;
+    const int TBA = kDdRows / G;
+    P.nblk = (P.T + TBA - 1) / TBA;
+    CUtensorMap qm;
+    if (!make_dedup_q_map(&qm, q, P.T, P.Hq, G, TBA)) return DSA_ERR_CUDA;
+    switch (G) {
+    case 8: return launch_dedup_t<8>(qm, P, s);
+    case 16: return launch_dedup_t<16>(qm, P, s);
+    }
+    return DSA_ERR_UNSUPPORTED;
+}
+
 dsa_status run_attn(const AttnParams& P, cudaStream_t s) {
     const int G = P.Hq / P.Hkv;
     if (G <= 8) return launch_attn_t<1>(P, s);
@@ -477,6 +519,35 @@ dsa_status dsa_sparse_attn(const void* q, const void* k, const void* v, const in
     P.nsplit = 1;
     P.part = nullptr;
     return run_attn(P, reinterpret_cast<cudaStream_t>(stream));
+}
+
+dsa_status dsa_sparse_attn_dedup(const void* q, const void* k, const void* v, const int32_t* idx, int Lq, int64_t Lk,
+                                 int64_t q_pos0, int Hq, int Hkv, int D, int topk, float scale, void* out, float* lse,
+                                 dsa_stream_t stream) {
+    if (!q || !k || !v || !idx || !out) return DSA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(idx) || !aligned16(out))
+        return DSA_ERR_INVALID_ARG;
+    if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return DSA_ERR_INVALID_ARG;
+    if (Lq <= 0 || Lk <= 0 || q_pos0 < 0 || topk <= 0 || !(scale == scale)) return DSA_ERR_INVALID_ARG;
+    dsa_status st = check_attn_shape(Hq, Hkv, D);
+    if (st != DSA_OK) return st;
+    if (!dedup_supported(Hq, Hkv) || topk > kMaxTopk || Lk > (int64_t)kDdMaxWin * kDdWin)
+        return DSA_ERR_UNSUPPORTED;
+    DedupParams P{};
+    P.k = static_cast<const __nv_bfloat16*>(k);
+    P.v = static_cast<const __nv_bfloat16*>(v);
+    P.idx = idx;
+    P.topk = topk;
+    P.T = Lq;
+    P.q_pos0 = q_pos0;
+    P.n_keys = Lk;
+    P.window = 0;
+    P.Hq = Hq;
+    P.Hkv = Hkv;
+    P.scale_log2 = scale * 1.4426950408889634f;
+    P.out = static_cast<__nv_bfloat16*>(out);
+    P.lse = lse;
+    return run_attn_dedup(q, P, reinterpret_cast<cudaStream_t>(stream));
 }
 
 size_t dsa_workspace_size(int op, int64_t L, int B, int Hq, int HI, int topk) {
@@ -741,6 +812,12 @@ dsa_status dsa_sync_status(dsa_stream_t stream) {
     if (err & DSA_DEV_ERR_TIMEOUT) return DSA_ERR_TIMEOUT;
     if (err & DSA_DEV_ERR_BOUNDS) return DSA_ERR_DEVICE_INPUT;
     return DSA_OK;
+}
+
+unsigned int dsa_error_site(void) {
+    unsigned int where = 0;
+    if (cudaMemcpyFromSymbol(&where, g_dev_error_where, sizeof(where)) != cudaSuccess) return 0;
+    return where;
 }
 
 void dsa_profile_begin(void) {

@@ -85,6 +85,36 @@ __device__ __forceinline__ bool wait_parity(uint64_t* bar, uint32_t parity, unsi
     }
 }
 
+// try_wait with a suspend-time hint: a waiting thread sleeps (up to `ns`) until the phase completes
+// instead of spinning, so warps that wait long leave the issue slots to the warps that compute.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(ns)
+        : "memory");
+    return ok != 0;
+}
+
+// wait_parity with sleeping tries (same time limit and abort behaviour).
+__device__ __forceinline__ bool wait_parity_sleep(uint64_t* bar, uint32_t parity, unsigned where,
+                                                  volatile int* abort_flag = nullptr, uint32_t ns = 2000) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const unsigned long long t0 = globaltimer_ns();
+    while (true) {
+        if (mbar_try_wait_sleep(bar, parity, ns)) return true;
+        if (abort_flag && *abort_flag) return false;
+        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            record_error(DSA_DEV_ERR_TIMEOUT, where);
+            if (abort_flag) *abort_flag = 1;
+            return false;
+        }
+    }
+}
+
 // ------------------------------------------------------------------ TMA (no multicast)
 __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y, int z) {
     asm volatile(
@@ -186,6 +216,38 @@ __device__ __forceinline__ void tmem_ld_32x32b_x8(uint32_t taddr, float (&v)[8])
 
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
+// 32 lanes x 32 consecutive fp32 columns from registers: thread i of the warp writes lane (base + i).
+__device__ __forceinline__ void tmem_st_32x32b_x32(uint32_t taddr, const float (&v)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+        "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+        "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+        "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
+        "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+        "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+        "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])), "r"(__float_as_uint(v[17])),
+        "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])), "r"(__float_as_uint(v[20])),
+        "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])), "r"(__float_as_uint(v[23])),
+        "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])),
+        "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])),
+        "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+        : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// Make this thread's generic-proxy shared-memory writes visible to later async-proxy reads
+// (tcgen05.mma operands) once they are published through an mbarrier.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Barrier over a subset of the CTA's warps (ids 1..15; id 0 is __syncthreads).
+__device__ __forceinline__ void named_bar_sync(int id, int threads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
 // Shared-memory matrix descriptor: K-major tile whose rows are 128 bytes, 128-byte swizzle,
 // 8-row groups 1024 bytes apart (the layout TMA writes with CU_TENSOR_MAP_SWIZZLE_128B).
 __device__ __forceinline__ uint64_t smem_desc_k128_sw128(const void* tile) {
@@ -199,6 +261,21 @@ __device__ __forceinline__ uint64_t smem_desc_k128_sw128(const void* tile) {
     return d;
 }
 
+// Shared-memory matrix descriptor: MN-major tile with 128-byte swizzle.  Each 128-byte row holds
+// 64 consecutive MN elements of one K index; 8 consecutive K indices form a 1024-byte group
+// (stride byte offset), and the next 64 MN elements start `mn_stride` bytes further (leading byte
+// offset).
+__device__ __forceinline__ uint64_t smem_desc_mn_sw128(const void* tile, uint32_t mn_stride) {
+    const uint64_t addr = smem_u32(tile);
+    uint64_t d = 0;
+    d |= (addr >> 4) & 0x3FFFull;                      // start address
+    d |= (uint64_t)((mn_stride >> 4) & 0x3FFFu) << 16; // leading byte offset: next 64 MN elements
+    d |= (1024ull >> 4) << 32;                         // stride byte offset: next 8 K indices
+    d |= 1ull << 46;                                   // descriptor version for sm_100
+    d |= 2ull << 61;                                   // 128-byte swizzle
+    return d;
+}
+
 // Instruction descriptor, kind::f16: bf16 x bf16 -> fp32, both operands K-major.
 template <int M, int N>
 __host__ __device__ constexpr uint32_t idesc_bf16_f32() {
@@ -207,6 +284,11 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32() {
            | (1u << 10)                    // B format: bf16
            | (uint32_t(N >> 3) << 17)      // N / 8
            | (uint32_t(M >> 4) << 24);     // M / 16
+}
+// The same with B MN-major (B's N elements contiguous in shared memory).
+template <int M, int N>
+__host__ __device__ constexpr uint32_t idesc_bf16_f32_bmn() {
+    return idesc_bf16_f32<M, N>() | (1u << 16);
 }
 
 // ------------------------------------------------------------------ Ampere-style async copies
@@ -244,6 +326,12 @@ __device__ __forceinline__ void mma_16816(float (&c)[4], const uint32_t (&a)[4],
 __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
     uint32_t y;
     asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+    return y;
+}
+// 2^x by the hardware approximation (ex2.approx.ftz: 2^-inf = 0, subnormal results flush to 0).
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
 }
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

@@ -115,6 +115,21 @@ dsa_status dsa_sparse_attn(const void *q, const void *k, const void *v, const in
                            dsa_stream_t stream);
 
 /*
+ * Step 3 with adjacent-query deduplication (page gsyq.cn section 八): the same result as
+ * dsa_sparse_attn, computed per block of 128/G adjacent rows (G = Hq/Hkv query heads per KV group)
+ * over the union of the block's index sets: each union key's K/V rows are gathered once per KV
+ * group, S = Q.K^T and O += P.V run as 128-row tensor-core tiles of the block's (row, head) pairs,
+ * and each row's softmax masks the union keys it did not select.  Arguments and their layouts as
+ * dsa_sparse_attn.  An index repeated within a row counts once (dsa_topk never repeats one).
+ * Outputs differ from dsa_sparse_attn only by fp32 summation order and the bf16 rounding of the
+ * probabilities.  Rows may list their keys in any order.
+ * Errors: as dsa_sparse_attn; DSA_ERR_UNSUPPORTED unless G is 8 or 16, or if Lk > 2^21.
+ */
+dsa_status dsa_sparse_attn_dedup(const void *q, const void *k, const void *v, const int32_t *idx, int Lq, int64_t Lk,
+                                 int64_t q_pos0, int Hq, int Hkv, int D, int topk, float scale, void *out,
+                                 float *lse, dsa_stream_t stream);
+
+/*
  * Steps 1-3 fused over a whole causal sequence of length L (prefill).  Processes query rows in
  * chunks whose score rows fit the workspace (more workspace = fewer, larger chunks; results do
  * not depend on the chunk size).
@@ -235,6 +250,13 @@ size_t dsa_workspace_size(int op, int64_t L, int B, int Hq, int HI, int topk);
  * DSA_ERR_TIMEOUT, DSA_ERR_DEVICE_INPUT or DSA_ERR_CUDA (a sticky CUDA error).
  */
 dsa_status dsa_sync_status(dsa_stream_t stream);
+
+/*
+ * Diagnostics: the code of the last device-side check or bounded wait that recorded an error
+ * (low 12 bits: the site; higher bits: the loop index there, where the site has one); 0 if none
+ * since the library was loaded.  Not cleared by dsa_sync_status.
+ */
+unsigned int dsa_error_site(void);
 
 /*
  * Per-kernel timing.  dsa_profile_begin() starts recording a CUDA event pair around every

@@ -69,6 +69,18 @@ def test_host_validation_without_gpu():
     assert lib.dsa_sparse_attn(A, A, A, A, 4, 4, 0, 32, 4, 128, 0, f, A, None, None) == dsa.DSA_ERR_INVALID_ARG
     nan = ctypes.c_float(float("nan"))
     assert lib.dsa_sparse_attn(A, A, A, A, 4, 4, 0, 32, 4, 128, 16, nan, A, None, None) == dsa.DSA_ERR_INVALID_ARG
+    # dedup attention: the per-token checks, and G = Hq / Hkv must be 8 or 16
+    assert lib.dsa_sparse_attn_dedup(A, A, A, A, 4, 4, 0, 32, 4, 64, 16, f, A, None, None) == dsa.DSA_ERR_UNSUPPORTED
+    assert lib.dsa_sparse_attn_dedup(A, A, A, A, 4, 4, 0, 16, 4, 128, 16, f, A, None, None) == dsa.DSA_ERR_UNSUPPORTED
+    assert lib.dsa_sparse_attn_dedup(A, A, A, A, 4, 4, 0, 8, 4, 128, 16, f, A, None, None) == dsa.DSA_ERR_UNSUPPORTED
+    assert lib.dsa_sparse_attn_dedup(A, A, A, A, 0, 4, 0, 32, 4, 128, 16, f, A, None, None) == dsa.DSA_ERR_INVALID_ARG
+    assert lib.dsa_sparse_attn_dedup(A, A, A, A, 4, 4, 0, 32, 4, 128, 0, f, A, None, None) == dsa.DSA_ERR_INVALID_ARG
+    assert lib.dsa_sparse_attn_dedup(None, A, A, A, 4, 4, 0, 32, 4, 128, 16, f, A, None, None) == \
+        dsa.DSA_ERR_INVALID_ARG
+    assert lib.dsa_sparse_attn_dedup(A, A, A, A, 4, 4, 0, 32, 4, 128, 16, nan, A, None, None) == \
+        dsa.DSA_ERR_INVALID_ARG
+    assert lib.dsa_sparse_attn_dedup(A, A, A, A, 4, (1 << 31) - 100, 0, 32, 4, 128, 16, f, A, None, None) == \
+        dsa.DSA_ERR_UNSUPPORTED
     # prefill: workspace missing / too small
     args = [A] * 6 + [1024, 32, 4, 128, 32, 64, 2048, f, A, None]
     assert lib.dsa_prefill(*args, None, 0, None) == dsa.DSA_ERR_WORKSPACE
@@ -139,6 +151,9 @@ _SHAPE_CASES = [
     (dsa.dsa_sparse_attn, dict(q=_bf(8, 8, 128), k=_bf(8, 2, 128), v=_bf(8, 2, 128), idx=_i32(8, 4), q_pos0=0,
                                scale=0.1, out=_bf(8, 8, 128), lse=_f32(8, 8)),
      {"k": _bf(8, 2, 64), "v": _bf(9, 2, 128), "idx": _i32(7, 4), "out": _bf(8, 4, 128), "lse": _f32(8, 4)}),
+    (dsa.dsa_sparse_attn_dedup, dict(q=_bf(8, 16, 128), k=_bf(8, 2, 128), v=_bf(8, 2, 128), idx=_i32(8, 4),
+                                     q_pos0=0, scale=0.1, out=_bf(8, 16, 128), lse=_f32(8, 16)),
+     {"k": _bf(8, 2, 64), "v": _bf(9, 2, 128), "idx": _i32(7, 4), "out": _bf(8, 8, 128), "lse": _f32(8, 8)}),
     (dsa.dsa_prefill, _prefill_args(),
      {"k": _bf(15, 2, 128), "v": _bf(16, 1, 128), "qI": _bf(15, 4, 64), "kI": _bf(16, 32), "w": _bf(16, 3),
       "out": _bf(16, 8, 64), "idx_out": _i32(16, 9)}),
@@ -180,11 +195,14 @@ def _c_kind(decl: str) -> str:
     if "*" in d or d.startswith("dsa_stream_t"):
         return "ptr"
     base = d.split()[0]
+    if d.startswith("unsigned int"):
+        return "uint"
     return {"int": "int", "int64_t": "i64", "size_t": "size", "float": "float", "double": "double",
             "dsa_status": "int", "void": "void"}[base]
 
 
-_CTYPES_KIND = {ctypes.c_void_p: "ptr", ctypes.c_char_p: "ptr", ctypes.c_int: "int", ctypes.c_int64: "i64",
+_CTYPES_KIND = {ctypes.c_void_p: "ptr", ctypes.c_char_p: "ptr", ctypes.c_int: "int", ctypes.c_uint: "uint",
+                ctypes.c_int64: "i64",
                 ctypes.c_size_t: "size", ctypes.c_float: "float", ctypes.c_double: "double", None: "void"}
 
 

@@ -212,6 +212,7 @@ def main():
     ap.add_argument("--kl-rows", type=int, default=0,
                     help="query rows of the 32K workload for the KL measurement (default: all 32768)")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-dedup", action="store_true", help="skip the adjacent-query dedup attention measurement")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
     ap.add_argument("--ref-seconds", type=float, default=0.0,
@@ -410,6 +411,11 @@ def main():
     if not args.no_kl:
         kl = run_kl(torch, dsa, synth.CONFIGS["32k"], barrier, max_over_ranks, peaks, rows=args.kl_rows)
 
+    # ---- adjacent-query dedup attention against the per-token kernel (last 8192 rows)
+    dedup = None
+    if not args.no_dedup and rank == 0 and world == 1:
+        dedup = run_dedup(torch, dsa, cfg)
+
     cpu = None
     if rank == 0 and not args.no_cpu and world == 1:
         cpu = cpu_baseline(cfg, x, budget_s=args.cpu_seconds)
@@ -420,7 +426,7 @@ def main():
             "data": "synthetic (seeded; 512 frame + 64 text token layout, block-structured keys)",
             "config": bench_config(cfg, args.workload, world, args.split),
             "roofline": roofline, "kernels": kern, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
-            "clocks": clk, "decode": decode, "indexer_kl": kl, "adjacent_union_16": union16,
+            "clocks": clk, "decode": decode, "indexer_kl": kl, "adjacent_union_16": union16, "attn_dedup": dedup,
             "path_counters": counters}
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -439,6 +445,59 @@ def adjacent_union_stat(idx, cfg, torch, windows: int = 32) -> dict:
         rows = idx[int(t0):int(t0) + 16].cpu().numpy()
         sizes.append(len(np.unique(rows[rows >= 0])))
     return {"mean_unique": float(np.mean(sizes)), "naive": 16 * cfg.k, "windows": windows}
+
+
+def run_dedup(torch, dsa, cfg, rows: int = 8192, reps: int = 3) -> dict:
+    """dsa_sparse_attn_dedup against dsa_sparse_attn on the workload's last `rows` query rows:
+    (a) with their own top-k index sets, (b) with index sets that have the pages' adjacent-query
+    overlap (each block of 16 adjacent rows draws its rows' 2048 keys from one pool of 8000 keys,
+    about 7900 distinct per block; rows in the top-k's region order).  Per case: ms per launch of
+    each kernel (CUDA events, median of `reps` after one untimed call), the mean number of distinct
+    keys per 16 adjacent rows, and the largest output difference between the two kernels."""
+    L, C = cfg.L, rows
+    t0 = L - C
+    d = {n: synth.to_torch(synth.tensor(cfg, n, 0, L)).cuda() for n in ("k", "v", "kI")}
+    r = {n: synth.to_torch(synth.tensor(cfg, n, t0, C)).cuda() for n in ("q", "qI", "w")}
+    o1 = torch.empty((C, cfg.Hq, cfg.D), dtype=torch.bfloat16, device="cuda")
+    o2 = torch.empty_like(o1)
+    own = torch.empty((C, cfg.k), dtype=torch.int32, device="cuda")
+    dsa.dsa_prefill_rows(r["q"], d["k"], d["v"], r["qI"], d["kI"], r["w"], t0, cfg.k, cfg.scale, o1, own)
+    g = torch.Generator(device="cuda")
+    g.manual_seed(7)
+    nb, pool = C // 16, 8000
+    pools = torch.argsort(torch.rand(nb, t0, device="cuda", generator=g), dim=1)[:, :pool]
+    pick = torch.argsort(torch.rand(C, pool, device="cuda", generator=g), dim=1)[:, :cfg.k]
+    ov = torch.gather(pools.repeat_interleave(16, dim=0), 1, pick).to(torch.int32)
+    region_key = ((ov // 32) % 4).to(torch.int64) * (1 << 40) + ov.to(torch.int64)
+    ov = torch.gather(ov, 1, torch.argsort(region_key, dim=1)).contiguous()
+    del pools, pick, region_key
+
+    def timed(fn):
+        fn()
+        torch.cuda.synchronize()
+        if dsa.sync_status() != dsa.DSA_OK:
+            raise SystemExit("device error in the dedup measurement")
+        ts = []
+        for _ in range(reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        return float(np.median(ts))
+
+    res = {"rows": [t0, L]}
+    for name, ii in (("own_topk", own), ("pages_overlap", ov)):
+        ms_t = timed(lambda: dsa.dsa_sparse_attn(r["q"], d["k"], d["v"], ii, t0, cfg.scale, o1))
+        ms_d = timed(lambda: dsa.dsa_sparse_attn_dedup(r["q"], d["k"], d["v"], ii, t0, cfg.scale, o2))
+        blocks = ii[: 16 * 64].cpu().numpy().reshape(64, 16 * cfg.k)
+        res[name] = {"per_token_ms": round(ms_t, 4), "dedup_ms": round(ms_d, 4),
+                     "union16_mean": float(np.mean([len(np.unique(b[b >= 0])) for b in blocks])),
+                     "max_abs_diff": float((o1.float() - o2.float()).abs().max())}
+    del d, r, o1, o2, own, ov
+    torch.cuda.empty_cache()
+    return res
 
 
 # the prefill kernels' algorithmic unit (the denominator of the DRAM bytes per unit in
@@ -591,7 +650,7 @@ def run_kl(torch, dsa, cfg, barrier, max_over_ranks, peaks, reps: int = 3, rows:
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": tpeak,
                          "unit": "TFLOP/s", "frac": achieved / tpeak, "frac_sustained": achieved / tsust,
                          "algorithmic": "4 x Hq x D flop per causal (t, s) pair (two passes of Q.K)"},
-            "mean_kl": float(kl.mean()), "mma": "warp-level m16n8k16 (mma.sync)"}
+            "mean_kl": float(kl.mean()), "mma": "tcgen05 (TMEM accumulators, TMA operands)"}
 
 
 def decode_config(args):

@@ -343,6 +343,92 @@ dsa_status run_attn_dedup(const void* q, DedupParams P, cudaStream_t s) {
     return DSA_ERR_UNSUPPORTED;
 }
 
+// ------------------------------------------------------------------ warm-up KL launches
+// k bf16 [Lk][Hkv][128] as a 3D map {128, Hkv, Lk}; box {64, 1, 128}: 128 keys of one KV group, one
+// 64-dim half per load, 128-byte swizzle.
+bool make_k_tile_map(CUtensorMap* m, const void* k, int64_t Lk, int Hkv) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)kAttnD, (cuuint64_t)Hkv, (cuuint64_t)Lk};
+    cuuint64_t strides[2] = {(cuuint64_t)kAttnD * 2, (cuuint64_t)Hkv * kAttnD * 2};
+    cuuint32_t box[3] = {64, 1, (cuuint32_t)kKlKeys};
+    cuuint32_t es[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(k), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool kl_shape_supported(int Hq, int Hkv) {
+    return (Hq == 8 || Hq == 16 || Hq == 32 || Hq == 64) && (Hkv == 1 || Hkv == 2 || Hkv == 4) && Hq % Hkv == 0 &&
+           Hq / Hkv >= 2;
+}
+
+template <int G>
+dsa_status launch_kl_lse_t(const CUtensorMap& qm, const CUtensorMap& km, const KlLseParams& P, cudaStream_t s) {
+    auto kern = kl_lse_kernel<G>;
+    static DeviceFlags attr_set;
+    if (!set_smem_limit(kern, kKlLseSmem, attr_set)) return DSA_ERR_CUDA;
+    LaunchScope ls(K_KL, s);
+    kern<<<P.nblk * P.Hkv, kKlThreads, kKlLseSmem, s>>>(qm, km, P);
+    return launch_status();
+}
+
+template <int HQ, int HKV>
+dsa_status launch_kl_div_t(const CUtensorMap& qm, const CUtensorMap& km, const KlDivParams& P, cudaStream_t s) {
+    auto kern = kl_div_kernel<HQ, HKV>;
+    static DeviceFlags attr_set;
+    if (!set_smem_limit(kern, kKlDivSmem, attr_set)) return DSA_ERR_CUDA;
+    LaunchScope ls(K_KL, s);
+    kern<<<P.nblk, kKlThreads, kKlDivSmem, s>>>(qm, km, P);
+    return launch_status();
+}
+
+// Both passes for n query rows at positions t0 .. t0+n-1 whose indexer score rows are in `scores`.
+dsa_status run_kl(const __nv_bfloat16* q, const void* k, const float* scores, int64_t ld, int n, int64_t t0, int Hq,
+                  int Hkv, float scale, float* lse2, float* kl, cudaStream_t s) {
+    const int G = Hq / Hkv;
+    CUtensorMap km, qa, qb;
+    if (!make_k_tile_map(&km, k, t0 + n, Hkv)) return DSA_ERR_CUDA;
+    KlLseParams A{};
+    A.T = n;
+    A.q_pos0 = t0;
+    A.Hq = Hq;
+    A.Hkv = Hkv;
+    A.scale_log2 = scale * 1.4426950408889634f;
+    A.lse2 = lse2;
+    A.nblk = (n + 128 / G - 1) / (128 / G);
+    if (!make_dedup_q_map(&qa, q, n, Hq, G, 128 / G)) return DSA_ERR_CUDA;
+    dsa_status st = DSA_ERR_UNSUPPORTED;
+    switch (G) {
+    case 2: st = launch_kl_lse_t<2>(qa, km, A, s); break;
+    case 4: st = launch_kl_lse_t<4>(qa, km, A, s); break;
+    case 8: st = launch_kl_lse_t<8>(qa, km, A, s); break;
+    case 16: st = launch_kl_lse_t<16>(qa, km, A, s); break;
+    case 32: st = launch_kl_lse_t<32>(qa, km, A, s); break;
+    case 64: st = launch_kl_lse_t<64>(qa, km, A, s); break;
+    }
+    if (st != DSA_OK) return st;
+    KlDivParams B{};
+    B.scores = scores;
+    B.ld = ld;
+    B.T = n;
+    B.q_pos0 = t0;
+    B.scale_log2 = A.scale_log2;
+    B.lse2 = lse2;
+    B.kl = kl;
+    const int TB = 256 / Hq;
+    B.nblk = (n + TB - 1) / TB;
+    if (!make_dedup_q_map(&qb, q, n, Hq, G, TB)) return DSA_ERR_CUDA;
+#define DSA_KL_DIV(HQ_, HKV_) \
+    if (Hq == HQ_ && Hkv == HKV_) return launch_kl_div_t<HQ_, HKV_>(qb, km, B, s);
+    DSA_KL_DIV(8, 1) DSA_KL_DIV(8, 2) DSA_KL_DIV(8, 4)
+    DSA_KL_DIV(16, 1) DSA_KL_DIV(16, 2) DSA_KL_DIV(16, 4)
+    DSA_KL_DIV(32, 1) DSA_KL_DIV(32, 2) DSA_KL_DIV(32, 4)
+    DSA_KL_DIV(64, 1) DSA_KL_DIV(64, 2) DSA_KL_DIV(64, 4)
+#undef DSA_KL_DIV
+    return DSA_ERR_UNSUPPORTED;
+}
+
 dsa_status run_attn(const AttnParams& P, cudaStream_t s) {
     const int G = P.Hq / P.Hkv;
     if (G <= 8) return launch_attn_t<1>(P, s);
@@ -551,13 +637,13 @@ dsa_status dsa_sparse_attn_dedup(const void* q, const void* k, const void* v, co
 }
 
 size_t dsa_workspace_size(int op, int64_t L, int B, int Hq, int HI, int topk) {
-    if (op == DSA_OP_INDEXER_KL) {  // score rows only (topk unused)
-        if (L <= 0 || HI <= 0) return 0;
+    if (op == DSA_OP_INDEXER_KL) {  // score rows and per-head log-sum-exps of a chunk (topk unused)
+        if (L <= 0 || HI <= 0 || Hq <= 0) return 0;
         const int64_t ld = prefill_ld(L);
         int64_t rows = (int64_t(4) << 30) / (ld * 4);
         rows = std::max<int64_t>(256, rows / 256 * 256);
         rows = std::min<int64_t>(rows, L);
-        return align_up((size_t)rows * ld * 4, 256);
+        return align_up(chunk_bytes(rows, ld, Hq), 256);
     }
     if (L <= 0 || topk <= 0 || HI <= 0) return 0;
     switch (op) {
@@ -588,36 +674,26 @@ dsa_status dsa_indexer_kl(const void* q, const void* k, const void* qI, const vo
     if (L <= 0 || HI <= 0 || dI <= 0 || !(scale == scale)) return DSA_ERR_INVALID_ARG;
     dsa_status st = check_attn_shape(Hq, Hkv, D);
     if (st != DSA_OK) return st;
-    if (Hq / Hkv > 8 || dI != kIdxBK || !hi_supported_prefill(HI) || L * HI > (int64_t)INT32_MAX)
+    if (!kl_shape_supported(Hq, Hkv) || dI != kIdxBK || !hi_supported_prefill(HI) || L * HI > (int64_t)INT32_MAX)
         return DSA_ERR_UNSUPPORTED;
     if (!ws || !aligned16(ws)) return DSA_ERR_WORKSPACE;
     const int64_t ld = prefill_ld(L);
-    const int TB = indexer_tb(HI, false);
-    const int64_t C = chunk_rows(ws_bytes, ld, 0, L, TB);
+    // chunks of whole blocks of every kernel (indexer 256/HI, pass 1 128/G, pass 2 256/Hq rows), so
+    // that a row's arithmetic does not depend on the chunk size
+    const int TB = std::max(indexer_tb(HI, false), 128);
+    const int64_t C = chunk_rows(ws_bytes, ld, Hq, L, TB);
     if (C < std::min<int64_t>(L, TB)) return DSA_ERR_WORKSPACE;
     float* scores = static_cast<float*>(ws);
+    float* lse2 = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + align_up((size_t)C * ld * 4, 256));
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    static DeviceFlags attr_set;
-    if (!set_smem_limit(indexer_kl_kernel, kl_smem_bytes(4), attr_set)) return DSA_ERR_CUDA;
     for (int64_t t0 = 0; t0 < L; t0 += C) {
         const int n = (int)std::min<int64_t>(C, L - t0);
         st = run_indexer(static_cast<const __nv_bfloat16*>(qI) + t0 * HI * dI, kI,
                          static_cast<const __nv_bfloat16*>(w) + t0 * HI, 1, n, t0, nullptr, t0 + n, HI, scores, ld, s);
         if (st != DSA_OK) return st;
-        KlParams P{};
-        P.q = static_cast<const __nv_bfloat16*>(q) + t0 * Hq * D;
-        P.k = static_cast<const __nv_bfloat16*>(k);
-        P.scores = scores;
-        P.ld = ld;
-        P.T = n;
-        P.q_pos0 = t0;
-        P.Hq = Hq;
-        P.Hkv = Hkv;
-        P.scale_log2 = scale * 1.4426950408889634f;
-        P.kl = kl + t0;
-        LaunchScope ls(K_KL, s);
-        indexer_kl_kernel<<<(n + kKlTokens - 1) / kKlTokens, kKlTokens * 32, kl_smem_bytes(Hkv), s>>>(P);
-        if ((st = launch_status()) != DSA_OK) return st;
+        st = run_kl(static_cast<const __nv_bfloat16*>(q) + t0 * Hq * D, k, scores, ld, n, t0, Hq, Hkv, scale, lse2,
+                    kl + t0, s);
+        if (st != DSA_OK) return st;
     }
     return DSA_OK;
 }

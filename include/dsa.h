@@ -168,11 +168,13 @@ dsa_status dsa_prefill_rows(const void *q, const void *k, const void *v, const v
  *   kl[t]  = sum_s P_t(s) * (log P_t(s) - log Q_t(s))                      (natural log)
  *   q bf16 [L, Hq, D]; k bf16 [L, Hkv, D]; qI bf16 [L, HI, dI]; kI bf16 [L, dI]; w bf16 [L, HI]
  *   kl      float [L] (device, 4-byte aligned), written
- *   ws      score rows for a chunk of queries: at least
+ *   ws      a chunk of queries' score rows and per-head log-sum-exps (Hq floats a row): at least
  *           dsa_workspace_size(DSA_OP_INDEXER_KL, L, 1, Hq, HI, 1) bytes recommended; any size
- *           holding min(L, 256/HI) rows works (smaller sizes mean more, shorter chunks).
- * Supported: D = 128, dI = 64, Hkv in {1, 2, 4}, Hq/Hkv <= 8, HI a power of two <= 64.  Dense
- * cost: 4 x Hq x D flop per causal (t, s) pair plus the indexer.  Status codes as dsa_prefill.
+ *           holding min(L, max(128, 256/HI)) rows works (smaller sizes mean more, shorter chunks;
+ *           the results do not depend on the chunk size).
+ * Supported: D = 128, dI = 64, Hq in {8, 16, 32, 64}, Hkv in {1, 2, 4} with Hq/Hkv >= 2, HI a
+ * power of two <= 64.  Dense cost: 4 x Hq x D flop per causal (t, s) pair plus the indexer.
+ * Status codes as dsa_prefill.
  */
 dsa_status dsa_indexer_kl(const void *q, const void *k, const void *qI, const void *kI, const void *w, int64_t L,
                           int Hq, int Hkv, int D, int HI, int dI, float scale, float *kl, void *ws, size_t ws_bytes,

@@ -32,7 +32,8 @@ def test_workspace_sizes():
     assert dsa.workspace_size(dsa.DSA_OP_DECODE, 131328, 16, 32, 32, 2048) >= 16 * 131328 * 4
     assert dsa.workspace_size(dsa.DSA_OP_INDEX, 100) == 0
     # indexer KL at 32K: all 32768 score rows fit in 4 GiB
-    assert dsa.workspace_size(dsa.DSA_OP_INDEXER_KL, 32768, 1, 32, 32, 1) == 32768 * 32768 * 4
+    # (plus each row's 32 per-head log-sum-exps)
+    assert dsa.workspace_size(dsa.DSA_OP_INDEXER_KL, 32768, 1, 32, 32, 1) == 32768 * 32768 * 4 + 32768 * 32 * 4
     assert dsa.workspace_size(dsa.DSA_OP_PREFILL, 0) == 0
     assert dsa.workspace_size(99, 100) == 0
 
@@ -98,7 +99,10 @@ def test_host_validation_without_gpu():
     assert lib.dsa_indexer_kl(None, *[A] * 4, 1024, 32, 4, 128, 32, 64, f, A, A, 1 << 30, None) == \
         dsa.DSA_ERR_INVALID_ARG
     assert lib.dsa_indexer_kl(*kargs, 32, 4, 64, 32, 64, f, A, A, 1 << 30, None) == dsa.DSA_ERR_UNSUPPORTED
-    assert lib.dsa_indexer_kl(*kargs, 64, 4, 128, 32, 64, f, A, A, 1 << 30, None) == dsa.DSA_ERR_UNSUPPORTED
+    # KL: Hq must be 8/16/32/64 with at least two query heads per KV group
+    assert lib.dsa_indexer_kl(*kargs, 4, 4, 128, 32, 64, f, A, A, 1 << 30, None) == dsa.DSA_ERR_UNSUPPORTED
+    assert lib.dsa_indexer_kl(*kargs, 24, 4, 128, 32, 64, f, A, A, 1 << 30, None) == dsa.DSA_ERR_UNSUPPORTED
+    assert lib.dsa_indexer_kl(*kargs, 8, 8, 128, 32, 64, f, A, A, 1 << 30, None) == dsa.DSA_ERR_UNSUPPORTED
     assert lib.dsa_indexer_kl(*kargs, 32, 4, 128, 32, 64, f, A, None, 0, None) == dsa.DSA_ERR_WORKSPACE
     assert lib.dsa_indexer_kl(*kargs, 32, 4, 128, 32, 64, f, A, A, 64, None) == dsa.DSA_ERR_WORKSPACE
     # self test bounds

@@ -213,6 +213,8 @@ def main():
                     help="query rows of the 32K workload for the KL measurement (default: all 32768)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-dedup", action="store_true", help="skip the adjacent-query dedup attention measurement")
+    ap.add_argument("--dedup-only", action="store_true", help="only the dedup attention measurement (rank 0)")
+    ap.add_argument("--dedup-rows", type=int, default=8192, help="query rows of the dedup measurement")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
     ap.add_argument("--ref-seconds", type=float, default=0.0,
@@ -266,6 +268,10 @@ def main():
             print(json.dumps({"decode": decode}), flush=True)
         return 0
     cfg = synth.CONFIGS[args.workload]
+    if args.dedup_only:
+        if rank == 0:
+            print(json.dumps({"attn_dedup": run_dedup(torch, dsa, cfg, rows=args.dedup_rows)}), flush=True)
+        return 0
     if args.profile_rows:
         return run_profile_case(torch, dsa, cfg, args.profile_rows)
     rows_mode = args.split == "rows"
@@ -414,7 +420,7 @@ def main():
     # ---- adjacent-query dedup attention against the per-token kernel (last 8192 rows)
     dedup = None
     if not args.no_dedup and rank == 0 and world == 1:
-        dedup = run_dedup(torch, dsa, cfg)
+        dedup = run_dedup(torch, dsa, cfg, rows=args.dedup_rows)
 
     cpu = None
     if rank == 0 and not args.no_cpu and world == 1:
@@ -511,6 +517,15 @@ def traffic_units(cfg, work: dict) -> dict:
             "sparse_attn": work["attn_gather_bytes"]}
 
 
+# The gather ceiling of the attention kernel's copy structure when the rows are L2-resident: the same
+# ring of bulk copies (3 producer warps, 2 CTAs per SM) with consumers that only release the slots,
+# measured on one B200 at 1965 MHz (about 17 TB/s of 1 KiB rows; plain 16-byte loads of L2-resident
+# rows reach about 21 TB/s).  Most of the attention's gathered rows hit L2, so this, not the HBM
+# copy rate, is the ceiling its logical gather rate is compared with.
+L2_GATHER_GBS = 17000.0
+L2_GATHER_SOURCE = "bulk-copy ring with trivial consumers, L2-resident 1 KiB rows, one B200 (probe)"
+
+
 def kernel_rooflines(prof: dict, work: dict, steps: int, peaks: dict, workload: str, cfg) -> dict:
     """Per prefill kernel: mean CUDA-event launch time inside the timed region, achieved rate of
     its algorithmic work, and the fraction of the measured peak for its bound.  The indexer is
@@ -543,7 +558,9 @@ def kernel_rooflines(prof: dict, work: dict, steps: int, peaks: dict, workload: 
     logical = (work["attn_gather_bytes"] + work["attn_io_bytes"]) / n_a / (ms_a / 1e3) / 1e9
     kern["sparse_attn"] = {"bound": "hbm", "achieved": logical, "peak": hbm, "unit": "GB/s", "frac": logical / hbm,
                            "achieved_logical": logical, "logical_frac": logical / hbm, "ms_per_launch": ms_a,
-                           "launches_per_step": n_a, "peak_source": "measured HBM copy"}
+                           "launches_per_step": n_a, "peak_source": "measured HBM copy",
+                           "l2_gather_ceiling": {"value": L2_GATHER_GBS, "unit": "GB/s", "frac": logical / L2_GATHER_GBS,
+                                                 "source": L2_GATHER_SOURCE}}
     # DRAM bytes per launch: ncu counters of a small case of the same kernel, scaled by the
     # launch's algorithmic units, used only while the kernel sources are unchanged
     tr = {}

@@ -266,15 +266,24 @@ __device__ __forceinline__ uint32_t stream_collect(TopkSmem& S, const Grp& G, co
     // so that warp w takes exactly the pieces p with p % 4 == w (keys below g_lo are masked)
     g_lo &= ~31;
     constexpr int kStep = kTkUnroll * 128;  // float4 per iteration
+    // software pipelined: the next batch's loads are in flight while this batch is filtered
+    float4 vn[kTkUnroll];
+    auto load_batch = [&](int gb) {
+        const bool in = gb >= g_in_lo && gb + kStep <= g_in_hi;
+#pragma unroll
+        for (int u = 0; u < kTkUnroll; ++u) {
+            const int g = gb + u * 128 + lane_off;
+            vn[u] = (in || g < g_hi) ? __ldcs(row4 + g) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+    };
+    if (g_lo < g_hi) load_batch(g_lo);
     for (int g0 = g_lo; g0 < g_hi; g0 += kStep) {
         // warp-uniform: every float4 of this iteration is in range, so only the score is tested
         const bool interior = g0 >= g_in_lo && g0 + kStep <= g_in_hi;
         float4 v[kTkUnroll];
 #pragma unroll
-        for (int u = 0; u < kTkUnroll; ++u) {
-            const int g = g0 + u * 128 + lane_off;
-            v[u] = (interior || g < g_hi) ? __ldcs(row4 + g) : make_float4(0.f, 0.f, 0.f, 0.f);
-        }
+        for (int u = 0; u < kTkUnroll; ++u) v[u] = vn[u];
+        if (g0 + kStep < g_hi) load_batch(g0 + kStep);
         uint32_t m[kTkUnroll];
         uint32_t c_lo = 0, c_hi = 0;  // candidate counts of float4 u in byte u (u < 4) or byte u-4
 #pragma unroll
@@ -608,7 +617,7 @@ __device__ __forceinline__ uint32_t retarget(uint32_t rs, uint32_t c, long long 
     return (uint32_t)max(1LL, min(m - 1, r2));
 }
 
-__global__ void __launch_bounds__(kTkThreads, 6) topk_kernel(const TopkParams P) {
+__global__ void __launch_bounds__(kTkThreads, 5) topk_kernel(const TopkParams P) {
     extern __shared__ __align__(1024) uint8_t topk_smem[];
     TopkSmem& S = *reinterpret_cast<TopkSmem*>(topk_smem);
     const int r = blockIdx.x, tid = threadIdx.x, warp = tid >> 5;

@@ -24,7 +24,9 @@
 //   - S^T[keys x heads] = K . Q^T and O^T += V^T . P^T on warp-level bf16 MMAs
 //     (m16n8k16, keys or head-dimension rows as M, 8 heads as N), so no MMA lane is wasted on
 //     the small head count; P^T goes from the accumulator layout to the operand layout with
-//     movmatrix; online softmax in fp32 (exp2 domain);
+//     movmatrix; online softmax in fp32 (exp2 domain) against a reference maximum that moves only
+//     when a logit exceeds it by more than 2^8 (one warp vote per tile instead of a shuffle
+//     reduction; the probabilities stay below 2^8 and m + log2(l) is the same log-sum-exp);
 //   - slots past the row's count and entries naming no key (index -1 or >= n_keys) copy a
 //     zero row and get logit -inf.
 // With nsplit > 1 every CTA writes unnormalised partial results (O, running max, running sum)
@@ -250,25 +252,27 @@ __global__ void __launch_bounds__(kAttnThreads, NT == 1 ? 2 : 1) sparse_attn_ker
                 z[2] = v1 ? sacc[nt][2] * P.scale_log2 : -INFINITY;
                 z[3] = v1 ? sacc[nt][3] * P.scale_log2 : -INFINITY;
                 float mx[2] = {fmaxf(z[0], z[2]), fmaxf(z[1], z[3])};
+                float alpha[2] = {1.f, 1.f};
+                // the reference maximum moves only when a logit exceeds it by more than 2^8
+                if (__any_sync(0xffffffffu, mx[0] > m_run[nt][0] + 8.f || mx[1] > m_run[nt][1] + 8.f)) {
 #pragma unroll
-                for (int j = 0; j < 2; ++j) {
-                    mx[j] = fmaxf(mx[j], __shfl_xor_sync(0xffffffffu, mx[j], 4));
-                    mx[j] = fmaxf(mx[j], __shfl_xor_sync(0xffffffffu, mx[j], 8));
-                    mx[j] = fmaxf(mx[j], __shfl_xor_sync(0xffffffffu, mx[j], 16));
+                    for (int j = 0; j < 2; ++j) {
+                        mx[j] = fmaxf(mx[j], __shfl_xor_sync(0xffffffffu, mx[j], 4));
+                        mx[j] = fmaxf(mx[j], __shfl_xor_sync(0xffffffffu, mx[j], 8));
+                        mx[j] = fmaxf(mx[j], __shfl_xor_sync(0xffffffffu, mx[j], 16));
+                        if (mx[j] > m_run[nt][j] + 8.f) {
+                            alpha[j] = m_run[nt][j] == -INFINITY ? 0.f : ex2_approx(m_run[nt][j] - mx[j]);
+                            m_run[nt][j] = mx[j];
+                        }
+                    }
                 }
-                float alpha[2], base[2];
-#pragma unroll
-                for (int j = 0; j < 2; ++j) {
-                    const float m_new = fmaxf(m_run[nt][j], mx[j]);
-                    base[j] = m_new == -INFINITY ? 0.f : m_new;
-                    alpha[j] = exp2f(m_run[nt][j] - base[j]);
-                    m_run[nt][j] = m_new;
-                }
-                const float p0 = exp2f(z[0] - base[0]), p1 = exp2f(z[1] - base[1]);
-                const float p2 = exp2f(z[2] - base[0]), p3 = exp2f(z[3] - base[1]);
+                const float base[2] = {m_run[nt][0] == -INFINITY ? 0.f : m_run[nt][0],
+                                       m_run[nt][1] == -INFINITY ? 0.f : m_run[nt][1]};
+                const float p0 = ex2_approx(z[0] - base[0]), p1 = ex2_approx(z[1] - base[1]);
+                const float p2 = ex2_approx(z[2] - base[0]), p3 = ex2_approx(z[3] - base[1]);
                 l_run[nt][0] = l_run[nt][0] * alpha[0] + p0 + p2;
                 l_run[nt][1] = l_run[nt][1] * alpha[1] + p1 + p3;
-                // rescale only when some running max moved (alpha == 1 leaves O unchanged)
+                // rescale only when some reference maximum moved (alpha == 1 leaves O unchanged)
                 if (__any_sync(0xffffffffu, alpha[0] != 1.f || alpha[1] != 1.f)) {
 #pragma unroll
                     for (int dt = 0; dt < 8; ++dt) {

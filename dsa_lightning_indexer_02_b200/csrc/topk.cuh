@@ -249,7 +249,7 @@ __device__ __forceinline__ uint32_t sample_threshold(TopkSmem& S, const Grp& G, 
 // inclusive scan (5 shuffle steps), which gives every lane the position of each of its
 // candidates -- independent work for the whole batch instead of a ballot chain per load.
 // With chist, every candidate also adds one to bin min((key - hT0) >> hsh, kTkBins - 1) of the
-// 1024-bin histogram chist (which may live in another CTA's shared memory).
+// 1024-bin histogram chist (this CTA's shared memory).
 // Returns how many scores of this warp qualified (may exceed the region; the excess is dropped).
 __device__ __forceinline__ uint32_t stream_collect(TopkSmem& S, const Grp& G, const float4* row4, int g_lo, int g_hi,
                                                    int e_lo, int n, float F0, int region_base,
@@ -677,7 +677,8 @@ __global__ void __launch_bounds__(kTkThreads, 5) topk_kernel(const TopkParams P)
 // 1/kTkCluster of the row.  CTA 0 turns the samples (sent to it through distributed shared
 // memory) into the threshold T0, aimed at rank 2k so that a miss is rare, and into the scale of a
 // histogram of the candidates' key offsets from T0.  Every CTA streams its segment into its own
-// warp regions and adds each candidate to CTA 0's histogram (distributed shared-memory atomics).
+// warp regions and a local histogram of its candidates, which it then adds to CTA 0's
+// (distributed shared-memory atomics, one per non-empty bin).
 // The refinement is then spread over the cluster: CTA 0 finds the bin that holds the k-th key
 // (narrowing it with further distributed histogram rounds while it holds more than kTkBndMax
 // keys), the CTAs send that bin's members to CTA 0, which ranks them and broadcasts the exact
@@ -699,6 +700,7 @@ struct TopkClusterShared {
     int fixed;                        // needed from it, its size, low offset bits not yet fixed
     uint32_t cut_key;                 // last kept key of the boundary bin (broadcast)
     int cut_idx;
+    uint32_t lhist[kTkBins];          // this CTA's candidate histogram, added to CTA 0's after the stream
 };
 
 __device__ __forceinline__ uint32_t rank_target_2k(long long m, long long n, int k) {
@@ -732,7 +734,9 @@ __device__ __forceinline__ void cluster_select(TopkSmem& S, TopkClusterShared& C
     TopkSmem* S0 = cluster.map_shared_rank(&S, 0);
     TopkClusterShared* C0 = cluster.map_shared_rank(&C, 0);
 
-    const int s4 = sample_count4(n4 - gw, kTkCluster);  // per CTA
+    // half the one-CTA kernel's samples: aimed at rank 2k with room for twice that, the estimate
+    // needs less precision, and CTA 0 turns every sample into the threshold alone
+    const int s4 = sample_count4(n4 - gw, 2 * kTkCluster);  // per CTA
     const long long m = 4LL * s4 * kTkCluster;
     uint32_t rs = rank_target_2k(m, ne, k);
     bool done = false;
@@ -757,10 +761,19 @@ __device__ __forceinline__ void cluster_select(TopkSmem& S, TopkClusterShared& C
         cluster.sync();  // T0 everywhere, CTA 0's histogram cleared
         const uint32_t T0 = C.T0, sh = C.sh;
 
-        // ---- stream this CTA's segment into its warp regions and CTA 0's candidate histogram
+        // ---- stream this CTA's segment into its warp regions and a local candidate histogram (a
+        // remote atomic per candidate inside the compaction loop made the stream 4x slower), then
+        // add the histogram to CTA 0's once
+        for (int i = tid; i < kTkBins; i += kTkThreads) C.lhist[i] = 0u;
+        __syncthreads();
         const uint32_t c = stream_collect(S, G, row4, g_lo, g_hi, lo, n, key_floor_float(T0), warp * kTkRegion,
-                                          S0->hist, T0, (int)sh);
+                                          C.lhist, T0, (int)sh);
         if (lane == 0) S.reg_gt[warp] = (int)c;
+        __syncthreads();
+        for (int i = tid; i < kTkBins; i += kTkThreads) {
+            const uint32_t h = C.lhist[i];
+            if (h) atomicAdd(&S0->hist[i], h);
+        }
         cluster.sync();
         if (tid < kTkMaxRegions) src_cnt[tid] = cluster.map_shared_rank(&S, tid / kTkWarps)->reg_gt[tid % kTkWarps];
         __syncthreads();

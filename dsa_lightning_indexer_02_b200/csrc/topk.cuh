@@ -513,13 +513,18 @@ __device__ __forceinline__ bool refine_and_emit(TopkSmem& S, const Grp& G, uint3
     return true;
 }
 
-// Exact radix select over the row (the fallback; row(e) gives the score of key e): histogram passes of
-// 10 + 10 + 10 + 2 bits fix tau and the number of ties to keep, a scan finds the last kept tie,
-// then the kept keys are written in the same order as the fast path (region by region).
-template <class RowAt>
-__device__ __noinline__ void topk_global(TopkSmem& S, const Grp& G, RowAt row, int lo, int n, int k, int* out) {
-    const int tid = G.tid;
-    uint32_t pval = 0, need = (uint32_t)k;
+// Exact radix select over the row (the fallback): histogram passes of 10 + 10 + 10 + 2 bits over
+// the row's keys fix tau and the number of ties to keep; when that is every key equal to tau (the
+// usual case: one boundary key) no tie scan is needed, else a scan finds the last kept tie; then
+// warp w writes region w's kept keys ((index / 32) mod 4 == w) in ascending order after the
+// counts of the regions before it -- the fast path's order.  Every pass keeps eight 16-byte loads
+// per thread (radix) or eight loads per lane (emission) in flight: a row that misses twice costs a
+// few passes over it, not a latency-bound crawl.  `row` is 16-byte aligned.
+__device__ __noinline__ void topk_global(TopkSmem& S, const Grp& G, const float* row, int lo, int n, int k, int* out) {
+    const int tid = G.tid, lane = G.lane(), warp = G.warp();
+    const float4* row4 = reinterpret_cast<const float4*>(row);
+    const int g_lo = lo >> 2, g_hi = (n + 3) >> 2;
+    uint32_t pval = 0, need = (uint32_t)k, eq_cnt = 0;
     int fixed = 32;
     while (fixed > 0) {
         const int width = fixed >= 10 ? 10 : fixed;
@@ -528,50 +533,92 @@ __device__ __noinline__ void topk_global(TopkSmem& S, const Grp& G, RowAt row, i
         G.sync();
         clear_hist(S, G, nbins);
         G.sync();
-        for (int e = lo + tid; e < n; e += kTkThreads) {
-            const uint32_t key = score_key(row(e));
-            if (fixed >= 32 || (key >> fixed) == (pval >> fixed)) atomicAdd(&S.hist[(key >> sh) & (nbins - 1)], 1u);
+        for (int g0 = g_lo + tid; g0 < g_hi; g0 += 8 * kTkThreads) {
+            float4 v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int g = g0 + u * kTkThreads;
+                v[u] = g < g_hi ? __ldcs(row4 + g) : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int g = g0 + u * kTkThreads;
+                const float f[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int e = 4 * g + j;
+                    if (g >= g_hi || e < lo || e >= n) continue;
+                    const uint32_t key = score_key(f[j]);
+                    if (fixed >= 32 || (key >> fixed) == (pval >> fixed))
+                        atomicAdd(&S.hist[(key >> sh) & (nbins - 1)], 1u);
+                }
+            }
         }
         G.sync();
         find_threshold_bin(S, G, nbins, need);
         need -= S.sel_gt;
         pval |= S.sel_bin << sh;
+        if (sh == 0) eq_cnt = S.hist[S.sel_bin];  // every bit fixed: the keys equal to tau
         fixed = sh;
     }
     const uint32_t tau = pval, ties = need;
-    // the kept ties are the `ties` lowest-index keys equal to tau: count ties per 32-key piece in
-    // index order to find the last kept tie's index
-    uint32_t eq_seen = 0;
     int tie_end = n;  // keys == tau with index < tie_end are kept
-    for (int e0 = lo; e0 < n; e0 += kTkThreads) {
-        const int e = e0 + tid;
-        const uint32_t eq = (e < n && score_key(row(e)) == tau) ? 1u : 0u;
-        uint32_t total;
-        const uint32_t ex = block_excl_scan(S, G, eq, total);
-        if (eq && eq_seen + ex == ties - 1) S.sel_gt = (uint32_t)e + 1;  // the last kept tie
-        G.sync();
-        eq_seen += total;
-        if (eq_seen >= ties) {
-            tie_end = (int)S.sel_gt;
-            break;
-        }
-    }
-    // emit region by region (region = (e >> 5) & 3), ascending within a region
-    uint32_t written = 0;
-    for (int region = 0; region < 4; ++region) {
-        for (int p0 = (lo >> 5); p0 * 32 < n; p0 += kTkThreads / 32) {
-            // warp w handles piece p = p0 + w if it belongs to this region
-            const int p = p0 + (tid >> 5);
-            const int e = p * 32 + (tid & 31);
-            const bool mine = (p & 3) == region;
-            const uint32_t key = (mine && e >= lo && e < n) ? score_key(row(e)) : 0u;
-            const bool keep = mine && e >= lo && e < n && (key > tau || (key == tau && e < tie_end));
+    if (ties < eq_cnt) {
+        // keep only the `ties` lowest-index keys equal to tau: count them per 128 keys in order
+        uint32_t eq_seen = 0;
+        for (int e0 = lo; e0 < n; e0 += kTkThreads) {
+            const int e = e0 + tid;
+            const uint32_t eq = (e < n && score_key(row[e]) == tau) ? 1u : 0u;
             uint32_t total;
-            const uint32_t ex = block_excl_scan(S, G, keep ? 1u : 0u, total);
-            if (keep) out[written + ex] = e;
-            written += total;
+            const uint32_t ex = block_excl_scan(S, G, eq, total);
+            if (eq && eq_seen + ex == ties - 1) S.sel_gt = (uint32_t)e + 1;  // the last kept tie
+            G.sync();
+            eq_seen += total;
+            if (eq_seen >= ties) {
+                tie_end = (int)S.sel_gt;
+                break;
+            }
         }
     }
+    // emission: warp w owns region w, pieces p = 4 i + w (keys 32p .. 32p+31), lane = key
+    const int p_first = ((lo >> 5) & ~3) + warp, p_end = (n + 31) >> 5;
+    auto kept = [&](int e, float f) {
+        if (e < lo || e >= n) return false;
+        const uint32_t key = score_key(f);
+        return key > tau || (key == tau && e < tie_end);
+    };
+    uint32_t cnt = 0;
+    for (int p0 = p_first; p0 < p_end; p0 += 4 * 8) {
+        float f[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int e = (p0 + 4 * u) * 32 + lane;
+            f[u] = (p0 + 4 * u < p_end && e < n) ? __ldcs(row + e) : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) cnt += __popc(__ballot_sync(0xffffffffu, kept((p0 + 4 * u) * 32 + lane, f[u])));
+    }
+    if (lane == 0) S.red[warp] = cnt;
+    G.sync();
+    uint32_t base = 0;
+    for (int w = 0; w < warp; ++w) base += S.red[w];
+    for (int p0 = p_first; p0 < p_end; p0 += 4 * 8) {
+        float f[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int e = (p0 + 4 * u) * 32 + lane;
+            f[u] = (p0 + 4 * u < p_end && e < n) ? __ldcs(row + e) : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int e = (p0 + 4 * u) * 32 + lane;
+            const bool keep = kept(e, f[u]);
+            const uint32_t bal = __ballot_sync(0xffffffffu, keep);
+            if (keep) out[base + __popc(bal & ((1u << lane) - 1u))] = e;
+            base += __popc(bal);
+        }
+    }
+    G.sync();  // S.red is reused by the caller's next phase
 }
 
 __device__ __forceinline__ uint32_t rank_target(long long m, long long n, int k) {
@@ -670,7 +717,7 @@ __global__ void __launch_bounds__(kTkThreads, 5) topk_kernel(const TopkParams P)
             if (!done) atomicAdd(&g_counters[1 + 3 * attempt], 1ull);  // [1] first miss, [4] second miss
         }
     }
-    if (!done) topk_global(S, G, [row](int e) { return row[e]; }, lo, n, k, out);
+    if (!done) topk_global(S, G, row, lo, n, k, out);
 }
 
 // Few long rows (decode): a cluster of kTkCluster CTAs per row, each sampling and streaming
@@ -720,12 +767,11 @@ __device__ __forceinline__ int cluster_segment(int lo, int n, int crank, int& g_
 }
 
 // One row's selection by the cluster (every thread of every CTA calls it): ne = n - lo > k.
-// row4[g] is the row's float4 group g (this CTA reads its segment [g_lo, g_hi)); row_at(e) gives
-// any key's score to CTA 0's exact fallback.
-template <class RowAt>
+// row4[g] is the row's float4 group g (this CTA reads its segment [g_lo, g_hi)); CTA 0's exact
+// fallback reads the whole row.
 __device__ __forceinline__ void cluster_select(TopkSmem& S, TopkClusterShared& C, int* src_cnt,
                                                cg::cluster_group& cluster, const float4* row4, int g_lo, int g_hi,
-                                               int lo, int n, int k, int* out, RowAt row_at) {
+                                               int lo, int n, int k, int* out, const float* row) {
     const int crank = (int)cluster.block_rank();
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const Grp G{tid};
@@ -912,7 +958,7 @@ __device__ __forceinline__ void cluster_select(TopkSmem& S, TopkClusterShared& C
     }
     if (!done && crank == 0) {
         if (tid == 0) atomicAdd(&g_counters[5], 1ull);  // exact fallback
-        topk_global(S, G, row_at, lo, n, k, out);
+        topk_global(S, G, row, lo, n, k, out);
     }
     cluster.sync();  // peers keep their shared memory alive until every remote access is done
 }
@@ -938,7 +984,7 @@ __global__ void __launch_bounds__(kTkThreads, 1) topk_cluster_kernel(const TopkP
     int g_lo, g_hi;
     cluster_segment(lo, n, crank, g_lo, g_hi);
     cluster_select(S, C, src_cnt, cluster, reinterpret_cast<const float4*>(row), g_lo, g_hi, lo, n, k, out,
-                   [row](int e) { return row[e]; });
+                   row);
 }
 
 

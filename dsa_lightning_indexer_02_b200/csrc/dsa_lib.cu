@@ -256,6 +256,25 @@ dsa_status run_indexer(const void* qI, const void* kI, const __nv_bfloat16* w, i
 }
 
 // ------------------------------------------------------------------ top-k launch
+// Clusters of the top-k cluster kernel that fit on the device at once with `smem` bytes of
+// dynamic shared memory per CTA (cached per device and size; 0 if the query fails).
+int cluster_residency(int smem, cudaLaunchConfig_t cfg) {
+    static std::mutex mu;
+    static std::vector<std::pair<std::pair<int, int>, int>> cache;
+    const int dev = current_device();
+    std::lock_guard<std::mutex> lock(mu);
+    for (const auto& e : cache)
+        if (e.first.first == dev && e.first.second == smem) return e.second;
+    cfg.dynamicSmemBytes = smem;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, topk_cluster_kernel, &cfg) != cudaSuccess) {
+        (void)cudaGetLastError();
+        n = 0;
+    }
+    cache.push_back({{dev, smem}, n});
+    return n;
+}
+
 dsa_status run_topk(const float* scores, int64_t ld, int rows, int64_t q_pos0, const int* ctx_len, int64_t n_max,
                     int k, int* idx, cudaStream_t s, int64_t window = 0) {
     TopkParams P{scores, ld, rows, q_pos0, ctx_len, n_max, k, idx, window};
@@ -263,13 +282,12 @@ dsa_status run_topk(const float* scores, int64_t ld, int rows, int64_t q_pos0, c
     const int smem = (int)sizeof(TopkSmem);
     // Few long rows: a cluster of CTAs per row; otherwise one CTA per row.
     if ((long long)rows * kTkCluster <= 2LL * sms && n_max > 4LL * kTkCap) {
-        const int csmem = smem;
         static DeviceFlags cattr;
-        if (!set_smem_limit(topk_cluster_kernel, csmem, cattr)) return DSA_ERR_CUDA;
+        if (!set_smem_limit(topk_cluster_kernel, kTkStageOffset + kTkStageMaxF4 * 16, cattr)) return DSA_ERR_CUDA;
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(rows * kTkCluster);
         cfg.blockDim = dim3(kTkThreads);
-        cfg.dynamicSmemBytes = csmem;
+        cfg.dynamicSmemBytes = smem;
         cfg.stream = s;
         cudaLaunchAttribute attr[1];
         attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -278,6 +296,17 @@ dsa_status run_topk(const float* scores, int64_t ld, int rows, int64_t q_pos0, c
         attr[0].val.clusterDim.z = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
+        // Stage every CTA's segment in shared memory when the largest one fits and every cluster
+        // of the launch is still co-resident with the larger footprint (one wave).
+        const int64_t n4 = (n_max + 3) / 4;
+        const int seg_f4 = (int)(((n4 + kTkCluster - 1) / kTkCluster + 31) & ~31LL);
+        if (seg_f4 <= kTkStageMaxF4) {
+            const int ssmem = kTkStageOffset + seg_f4 * 16;
+            if (cluster_residency(ssmem, cfg) >= rows) {
+                P.stage_f4 = seg_f4;
+                cfg.dynamicSmemBytes = ssmem;
+            }
+        }
         LaunchScope ls(K_TOPK, s);
         if (cudaLaunchKernelEx(&cfg, topk_cluster_kernel, P) != cudaSuccess) return DSA_ERR_CUDA;
         return launch_status();

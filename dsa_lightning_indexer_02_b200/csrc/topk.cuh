@@ -66,6 +66,8 @@ struct TopkParams {
     int k;
     int* idx;             // [rows, k]
     long long window;     // > 0: only the last `window` keys of a row (s > t - window) compete
+    int stage_f4;         // cluster kernel: > 0 copies each CTA's segment (up to this many float4)
+                          // into shared memory first; 0 reads it from global memory
 };
 
 struct TopkSmem {
@@ -244,17 +246,22 @@ __device__ __forceinline__ uint32_t sample_threshold(TopkSmem& S, const Grp& G, 
 // Stream float4 groups [g_lo, g_hi) of a row whose keys e_lo <= e < n compete and compact the
 // scores >= F0 into this warp's region, in index order.  Warp w takes the 128-byte pieces p
 // (keys 32p .. 32p+31 of the row) with p % 4 == w: region w.
-// Each batch of kTkUnroll float4 loads per lane is filtered as a whole: the per-float4 candidate
-// counts of a lane (0..4 each) ride in the bytes of two registers through one warp-wide
-// inclusive scan (5 shuffle steps), which gives every lane the position of each of its
-// candidates -- independent work for the whole batch instead of a ballot chain per load.
-// With chist, every candidate also adds one to bin min((key - hT0) >> hsh, kTkBins - 1) of the
-// 1024-bin histogram chist (this CTA's shared memory).
+// Each batch of UN float4 loads per lane is filtered as a whole: the per-float4 candidate counts
+// of a lane (0..4 each) ride in the bytes of UN/4 registers through one warp-wide inclusive scan
+// (5 shuffle steps), which gives every lane the position of each of its candidates --
+// independent work for the whole batch instead of a ballot chain per load.  A float4 that holds
+// no candidate in any lane of the warp is skipped (a warp-uniform test); otherwise each of its
+// four scores is stored under a predicate, without divergent branches.
+// kPipe: the next batch's loads are issued before the current batch is filtered (software
+// pipelining, for a row read from global memory).
+// kStaged: group g is read from a shared-memory copy of the segment, src4[g - g_base]; otherwise
+// from the row in global memory (streaming loads), src4[g].
 // Returns how many scores of this warp qualified (may exceed the region; the excess is dropped).
-__device__ __forceinline__ uint32_t stream_collect(TopkSmem& S, const Grp& G, const float4* row4, int g_lo, int g_hi,
-                                                   int e_lo, int n, float F0, int region_base,
-                                                   uint32_t* chist = nullptr, uint32_t hT0 = 0, int hsh = 0) {
-    static_assert(kTkUnroll == 8, "the packed scan holds 8 counts");
+template <bool kStaged, int UN, bool kPipe>
+__device__ __forceinline__ uint32_t stream_collect(TopkSmem& S, const Grp& G, const float4* src4, int g_lo, int g_hi,
+                                                   int e_lo, int n, float F0, int region_base, int g_base = 0) {
+    static_assert(UN % 8 == 0, "counts ride four per word, masks eight per word");
+    constexpr int kW = UN / 4;  // words of packed per-float4 candidate counts
     const int g_first = g_lo;
     const int lane = G.lane(), warp = G.warp();
     // float4 offset inside a 128-float4 round: piece (lane/8)*4 + warp, float4 lane%8 of it
@@ -265,29 +272,33 @@ __device__ __forceinline__ uint32_t stream_collect(TopkSmem& S, const Grp& G, co
     // pieces are numbered from the start of the row: start at a multiple of 4 pieces (32 float4)
     // so that warp w takes exactly the pieces p with p % 4 == w (keys below g_lo are masked)
     g_lo &= ~31;
-    constexpr int kStep = kTkUnroll * 128;  // float4 per iteration
-    // software pipelined: the next batch's loads are in flight while this batch is filtered
-    float4 vn[kTkUnroll];
+    constexpr int kStep = UN * 128;  // float4 per iteration
+    float4 vn[UN];
     auto load_batch = [&](int gb) {
         const bool in = gb >= g_in_lo && gb + kStep <= g_in_hi;
 #pragma unroll
-        for (int u = 0; u < kTkUnroll; ++u) {
+        for (int u = 0; u < UN; ++u) {
             const int g = gb + u * 128 + lane_off;
-            vn[u] = (in || g < g_hi) ? __ldcs(row4 + g) : make_float4(0.f, 0.f, 0.f, 0.f);
+            vn[u] = (in || g < g_hi) ? (kStaged ? src4[g - g_base] : __ldcs(src4 + g)) : make_float4(0.f, 0.f, 0.f, 0.f);
         }
     };
-    if (g_lo < g_hi) load_batch(g_lo);
+    if (kPipe && g_lo < g_hi) load_batch(g_lo);
     for (int g0 = g_lo; g0 < g_hi; g0 += kStep) {
         // warp-uniform: every float4 of this iteration is in range, so only the score is tested
         const bool interior = g0 >= g_in_lo && g0 + kStep <= g_in_hi;
-        float4 v[kTkUnroll];
+        float4 v[UN];
+        if (!kPipe) load_batch(g0);
 #pragma unroll
-        for (int u = 0; u < kTkUnroll; ++u) v[u] = vn[u];
-        if (g0 + kStep < g_hi) load_batch(g0 + kStep);
-        uint32_t m[kTkUnroll];
-        uint32_t c_lo = 0, c_hi = 0;  // candidate counts of float4 u in byte u (u < 4) or byte u-4
+        for (int u = 0; u < UN; ++u) v[u] = vn[u];
+        if (kPipe && g0 + kStep < g_hi) load_batch(g0 + kStep);
+        uint32_t m[UN / 8];  // 4-bit candidate mask of float4 u in nibble u % 8 of word u / 8
+        uint32_t c[kW];      // candidate count (0..4) of float4 u in byte u % 4 of word u / 4
 #pragma unroll
-        for (int u = 0; u < kTkUnroll; ++u) {
+        for (int w = 0; w < kW; ++w) c[w] = 0;
+#pragma unroll
+        for (int w = 0; w < UN / 8; ++w) m[w] = 0;
+#pragma unroll
+        for (int u = 0; u < UN; ++u) {
             const int g = g0 + u * 128 + lane_off;
             const float f[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
             uint32_t mask = 0;
@@ -299,44 +310,52 @@ __device__ __forceinline__ uint32_t stream_collect(TopkSmem& S, const Grp& G, co
                 for (int j = 0; j < 4; ++j)
                     if (f[j] >= F0 && g * 4 + j < n && g * 4 + j >= e_lo && g >= g_first) mask |= 1u << j;
             }
-            m[u] = mask;
-            if (u < 4) c_lo |= (uint32_t)__popc(mask) << (8 * u);
-            else c_hi |= (uint32_t)__popc(mask) << (8 * (u - 4));
+            m[u >> 3] |= mask << (4 * (u & 7));
+            c[u >> 2] |= (uint32_t)__popc(mask) << (8 * (u & 3));
         }
-        if (__ballot_sync(0xffffffffu, (c_lo | c_hi) != 0) == 0) continue;
+        uint32_t any = 0;
+#pragma unroll
+        for (int w = 0; w < kW; ++w) any |= c[w];
+        if (__ballot_sync(0xffffffffu, any != 0) == 0) continue;
         // inclusive scan over lanes of the packed counts (each prefix <= 128 fits its byte)
-        uint32_t s_lo = c_lo, s_hi = c_hi;
+        uint32_t sc[kW];
+#pragma unroll
+        for (int w = 0; w < kW; ++w) sc[w] = c[w];
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
-            const uint32_t y_lo = __shfl_up_sync(0xffffffffu, s_lo, o), y_hi = __shfl_up_sync(0xffffffffu, s_hi, o);
+            uint32_t y[kW];
+#pragma unroll
+            for (int w = 0; w < kW; ++w) y[w] = __shfl_up_sync(0xffffffffu, sc[w], o);
             if (lane >= o) {
-                s_lo += y_lo;
-                s_hi += y_hi;
+#pragma unroll
+                for (int w = 0; w < kW; ++w) sc[w] += y[w];
             }
         }
-        const uint32_t t_lo = __shfl_sync(0xffffffffu, s_lo, 31), t_hi = __shfl_sync(0xffffffffu, s_hi, 31);
-        const uint32_t e_lo8 = s_lo - c_lo, e_hi8 = s_hi - c_hi;  // exclusive prefixes, bytewise
+        uint32_t t[kW];
+#pragma unroll
+        for (int w = 0; w < kW; ++w) {
+            t[w] = __shfl_sync(0xffffffffu, sc[w], 31);
+            sc[w] -= c[w];  // exclusive prefixes, bytewise
+        }
         // candidates of float4 u follow those of every lane's float4s before u (index order)
         uint32_t base = cnt;
 #pragma unroll
-        for (int u = 0; u < kTkUnroll; ++u) {
-            const uint32_t excl = ((u < 4 ? e_lo8 : e_hi8) >> (8 * (u & 3))) & 0xFFu;
-            const uint32_t tot = ((u < 4 ? t_lo : t_hi) >> (8 * (u & 3))) & 0xFFu;
-            if (m[u]) {
+        for (int u = 0; u < UN; ++u) {
+            const uint32_t tot = (t[u >> 2] >> (8 * (u & 3))) & 0xFFu;
+            if (tot) {  // warp-uniform: some lane has a candidate in float4 u
+                const uint32_t mu = (m[u >> 3] >> (4 * (u & 7))) & 0xFu;
                 const int g = g0 + u * 128 + lane_off;
                 const float f[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-                uint32_t pos = base + excl;
+                uint32_t pos = base + ((sc[u >> 2] >> (8 * (u & 3))) & 0xFFu);
 #pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    if (m[u] & (1u << j)) {
-                        const uint32_t key = score_key(f[j]);
-                        if (pos < (uint32_t)kTkRegion) {
-                            S.cand_key[region_base + pos] = key;
-                            S.cand_idx[region_base + pos] = g * 4 + j;
-                        }
-                        if (chist) atomicAdd(chist + min((key - hT0) >> hsh, (uint32_t)kTkBins - 1u), 1u);
-                        ++pos;
+                for (int j = 0; j < 4; ++j) {
+                    const bool cj = (mu >> j) & 1u;
+                    if (cj && pos < (uint32_t)kTkRegion) {
+                        S.cand_key[region_base + pos] = score_key(f[j]);
+                        S.cand_idx[region_base + pos] = g * 4 + j;
                     }
+                    pos += cj;
+                }
             }
             base += tot;
         }
@@ -627,9 +646,10 @@ __device__ __forceinline__ uint32_t rank_target(long long m, long long n, int k)
 }
 
 // Sample s4 evenly spaced float4 of float4 range [g_lo, g_hi) into keys[base .. base + 4*s4); all
-// of a thread's loads are issued before any is used.
-__device__ __forceinline__ void take_samples(const Grp& G, uint32_t* keys, int base, const float4* row4, int g_lo,
-                                             int g_hi, int e_lo, int n, int s4) {
+// of a thread's loads are issued before any is used.  Float4 group g is read at src4[g - g_base]
+// (the row itself with g_base = 0, or a shared-memory copy of a segment starting at g_base).
+__device__ __forceinline__ void take_samples(const Grp& G, uint32_t* keys, int base, const float4* src4, int g_base,
+                                             int g_lo, int g_hi, int e_lo, int n, int s4) {
     constexpr int kPer = kTkMaxSample4 / kTkThreads;
     float4 v[kPer];
     int gg[kPer];
@@ -639,7 +659,7 @@ __device__ __forceinline__ void take_samples(const Grp& G, uint32_t* keys, int b
     for (int u = 0; u < kPer; ++u) {
         const int i = G.tid + u * kTkThreads;
         gg[u] = g_lo + (int)(((unsigned long long)i * step) >> 32);
-        v[u] = (i < s4 && gg[u] < g_hi) ? row4[gg[u]] : make_float4(0.f, 0.f, 0.f, 0.f);
+        v[u] = (i < s4 && gg[u] < g_hi) ? src4[gg[u] - g_base] : make_float4(0.f, 0.f, 0.f, 0.f);
     }
 #pragma unroll
     for (int u = 0; u < kPer; ++u) {
@@ -689,11 +709,12 @@ __global__ void __launch_bounds__(kTkThreads, 5) topk_kernel(const TopkParams P)
         uint32_t T0 = 0;
         if (ne > kTkCap) {
             if (attempt > 0) __syncthreads();
-            take_samples(G, S.cand_key, 0, row4, g0, n4, lo, n, s4);
+            take_samples(G, S.cand_key, 0, row4, 0, g0, n4, lo, n, s4);
             T0 = sample_threshold(S, G, (int)m, rs);
         }
         // ---- one streaming pass: scores >= T0 into the 4 warp regions
-        const uint32_t c = stream_collect(S, G, row4, g0, n4, lo, n, key_floor_float(T0), warp * kTkRegion);
+        const uint32_t c = stream_collect<false, kTkUnroll, true>(S, G, row4, g0, n4, lo, n, key_floor_float(T0),
+                                                                  warp * kTkRegion);
         if ((tid & 31) == 0) {
             S.reg_kp[warp] = S.cand_key + warp * kTkRegion;
             S.reg_ip[warp] = S.cand_idx + warp * kTkRegion;
@@ -736,6 +757,11 @@ __global__ void __launch_bounds__(kTkThreads, 5) topk_kernel(const TopkParams P)
 // final bin of more than kTkBndMax equal keys, or a second miss, takes the exact radix select
 // on CTA 0.  Dynamic shared memory: sizeof(TopkSmem).
 constexpr int kTkBndMax = 256;
+// Staged segments: after TopkSmem in the cluster kernel's dynamic shared memory, moved by bulk
+// copies of at most kTkStageCopy bytes each; at most kTkStageMaxF4 float4 groups per CTA.
+constexpr int kTkStageOffset = (int)((sizeof(TopkSmem) + 127) / 128 * 128);
+constexpr uint32_t kTkStageCopy = 32768;
+constexpr int kTkStageMaxF4 = 10240;  // 160 KiB
 
 struct TopkClusterShared {
     int kept[kTkCluster][kTkWarps];  // kept keys per (CTA, region); every CTA writes its row into all
@@ -767,11 +793,13 @@ __device__ __forceinline__ int cluster_segment(int lo, int n, int crank, int& g_
 }
 
 // One row's selection by the cluster (every thread of every CTA calls it): ne = n - lo > k.
-// row4[g] is the row's float4 group g (this CTA reads its segment [g_lo, g_hi)); CTA 0's exact
-// fallback reads the whole row.
+// This CTA reads its segment [g_lo, g_hi) of float4 groups at src4[g - g_base]: the row itself
+// (staged false, g_base 0) or its shared-memory copy (staged true).  CTA 0's exact fallback reads
+// the whole row.
 __device__ __forceinline__ void cluster_select(TopkSmem& S, TopkClusterShared& C, int* src_cnt,
-                                               cg::cluster_group& cluster, const float4* row4, int g_lo, int g_hi,
-                                               int lo, int n, int k, int* out, const float* row) {
+                                               cg::cluster_group& cluster, const float4* src4, int g_base,
+                                               bool staged, int g_lo, int g_hi, int lo, int n, int k, int* out,
+                                               const float* row) {
     const int crank = (int)cluster.block_rank();
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const Grp G{tid};
@@ -788,7 +816,7 @@ __device__ __forceinline__ void cluster_select(TopkSmem& S, TopkClusterShared& C
     bool done = false;
     for (int attempt = 0; attempt < 2 && !done; ++attempt) {
         // ---- samples of every segment into CTA 0, which sets T0 and the histogram scale
-        take_samples(G, S0->cand_key, 4 * crank * s4, row4, g_lo, g_hi, lo, n, s4);
+        take_samples(G, S0->cand_key, 4 * crank * s4, src4, g_base, g_lo, g_hi, lo, n, s4);
         cluster.sync();
         if (crank == 0) {
             uint32_t kmax = 0;
@@ -807,14 +835,25 @@ __device__ __forceinline__ void cluster_select(TopkSmem& S, TopkClusterShared& C
         cluster.sync();  // T0 everywhere, CTA 0's histogram cleared
         const uint32_t T0 = C.T0, sh = C.sh;
 
-        // ---- stream this CTA's segment into its warp regions and a local candidate histogram (a
-        // remote atomic per candidate inside the compaction loop made the stream 4x slower), then
-        // add the histogram to CTA 0's once
+        // ---- stream this CTA's segment into its warp regions (a staged segment in batches of
+        // 16 float4 per lane: half the scan chains of the 8-wide form, which at one warp per
+        // scheduler are latency-bound), then count the stored candidates into a local histogram
+        // (a pass over shared memory whose atomics overlap, instead of one inside the compaction
+        // loop) and add it to CTA 0's once (a remote atomic per candidate made the stream 4x
+        // slower)
         for (int i = tid; i < kTkBins; i += kTkThreads) C.lhist[i] = 0u;
-        __syncthreads();
-        const uint32_t c = stream_collect(S, G, row4, g_lo, g_hi, lo, n, key_floor_float(T0), warp * kTkRegion,
-                                          C.lhist, T0, (int)sh);
+        const uint32_t c = staged ? stream_collect<true, 2 * kTkUnroll, false>(S, G, src4, g_lo, g_hi, lo, n,
+                                                                            key_floor_float(T0), warp * kTkRegion,
+                                                                            g_base)
+                                  : stream_collect<false, kTkUnroll, true>(S, G, src4, g_lo, g_hi, lo, n,
+                                                                           key_floor_float(T0), warp * kTkRegion);
         if (lane == 0) S.reg_gt[warp] = (int)c;
+        __syncthreads();
+        for (int w = 0; w < kTkWarps; ++w) {
+            const int cw = min(S.reg_gt[w], kTkRegion);
+            for (int e = tid; e < cw; e += kTkThreads)
+                atomicAdd(&C.lhist[min((S.cand_key[w * kTkRegion + e] - T0) >> sh, (uint32_t)kTkBins - 1u)], 1u);
+        }
         __syncthreads();
         for (int i = tid; i < kTkBins; i += kTkThreads) {
             const uint32_t h = C.lhist[i];
@@ -967,6 +1006,7 @@ __global__ void __launch_bounds__(kTkThreads, 1) topk_cluster_kernel(const TopkP
     extern __shared__ __align__(1024) uint8_t topk_smem[];
     __shared__ TopkClusterShared C;
     __shared__ int src_cnt[kTkMaxRegions];
+    __shared__ uint64_t stage_bar;
     TopkSmem& S = *reinterpret_cast<TopkSmem*>(topk_smem);
     cg::cluster_group cluster = cg::this_cluster();
     const int crank = (int)cluster.block_rank();
@@ -983,8 +1023,35 @@ __global__ void __launch_bounds__(kTkThreads, 1) topk_cluster_kernel(const TopkP
     const float* row = P.scores + (long long)r * P.ld;
     int g_lo, g_hi;
     cluster_segment(lo, n, crank, g_lo, g_hi);
-    cluster_select(S, C, src_cnt, cluster, reinterpret_cast<const float4*>(row), g_lo, g_hi, lo, n, k, out,
-                   row);
+    // Staging: one bulk copy brings this CTA's segment (from its 32-group boundary, where the
+    // stream starts) into shared memory while nothing else is waiting on it, so the samples and
+    // the stream read shared memory instead of paying a DRAM round trip per batch.
+    const int gs = g_lo & ~31;
+    const bool stage = P.stage_f4 > 0 && g_hi > gs && g_hi - gs <= P.stage_f4;  // uniform in the CTA
+    bool staged = false;
+    const float4* src4 = reinterpret_cast<const float4*>(row);
+    int g_base = 0;
+    if (stage) {
+        uint8_t* buf = topk_smem + kTkStageOffset;
+        if (tid == 0) {
+            mbar_init(&stage_bar, 1);
+            fence_mbar_init();
+            const uint32_t bytes = (uint32_t)(g_hi - gs) * 16u;
+            const uint8_t* src = reinterpret_cast<const uint8_t*>(row) + (size_t)gs * 16;
+            mbar_arrive_expect_tx(&stage_bar, bytes);
+            for (uint32_t off = 0; off < bytes; off += kTkStageCopy)
+                bulk_load(buf + off, src + off, min(kTkStageCopy, bytes - off), &stage_bar);
+        }
+        __syncthreads();
+        staged = wait_parity(&stage_bar, 0, 0xA01u);
+        if (staged) {
+            src4 = reinterpret_cast<const float4*>(buf);
+            g_base = gs;
+        }
+    }
+    cluster_select(S, C, src_cnt, cluster, src4, g_base, staged, g_lo, g_hi, lo, n, k, out, row);
+    // a copy that outlived a timed-out wait must land before this CTA's shared memory is released
+    if (stage && !staged) wait_parity(&stage_bar, 0, 0xA02u);
 }
 
 

@@ -700,3 +700,32 @@ def test_topk_cluster_and_one_cta_kernels_agree(cuda_ok):
     cnt = dsa.read_counters(reset=True)
     assert cnt["topk_rows"] == rows and cnt["topk_cluster_rows"] == rows, cnt
     assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("n,kind", [(300_000, "gauss"), (300_000, "ties"), (400_000, "gauss")])
+def test_topk_cluster_staged_and_unstaged_segments(cuda_ok, n, kind):
+    """The cluster kernel copies each CTA's eighth of a row into shared memory when it fits the
+    stage (300K keys: 147 KB per CTA) and streams it from global memory when it does not (400K
+    keys).  Both forms, and the exact fallback over the whole row (integer ties), give the
+    oracle's set in the documented order, entry by entry."""
+    rng = np.random.default_rng(31 + n)
+    rows, k = 3, 2048
+    q_pos0 = n - rows
+    ld = (n + 3) // 4 * 4
+    if kind == "ties":
+        s = rng.integers(-2, 3, size=(rows, ld)).astype(np.float32)
+    else:
+        s = (rng.standard_normal((rows, ld)) * 7).astype(np.float32)
+    idx = torch.full((rows, k), -5, dtype=torch.int32, device="cuda")
+    dsa.read_counters(reset=True)
+    dsa.dsa_topk(torch.from_numpy(s).cuda(), q_pos0, k, idx)
+    assert dsa.sync_status() == dsa.DSA_OK
+    cnt = dsa.read_counters(reset=True)
+    assert cnt["topk_cluster_rows"] == rows and cnt["topk_rows"] == 0, cnt
+    n_r = q_pos0 + np.arange(rows) + 1
+    want, _ = oracle.topk_rows(s.astype(np.float64), n_r, k)
+    got = idx.cpu().numpy()
+    for r in range(rows):
+        assert got[r].tolist() == canonical_order(want[r], int(n_r[r]), 0, k), (n, kind, r)
+    if kind == "ties":
+        assert cnt["topk_cluster_global"] > 0

@@ -704,7 +704,7 @@ def run_decode(torch, dsa, cfg, steps, rank, world, barrier, max_over_ranks, pea
         dsa.dsa_decode(new["q"][j], new["qI"][j], new["w"][j], new["k"][j], new["v"][j], new["kI"][j], kc, vc,
                        kIc, ctx, cfg.k, cfg.scale, out, ws=ws, update_ctx=True)
 
-    for j in range(8):
+    for j in range(min(8, steps)):
         one(j)
     torch.cuda.synchronize()
     ctx.fill_(ctx0)

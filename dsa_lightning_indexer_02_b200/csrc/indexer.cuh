@@ -187,7 +187,10 @@ struct IndexerCfg {
     // TMEM loads of 16 columns, one at a time (the other warps of the SM hide their latency): the
     // warpgroup's COLS_WG weights live in registers for a whole work unit, so the loads stay small.
     // Measured 3 % faster than double-buffered 8-column loads (half the load and wait instructions).
-    static constexpr int CHUNK = 16;
+    // A single epilogue warpgroup (decode: one token per tile) has no other epilogue warps to hide
+    // the load latency behind, so it reads 32 columns per load: one load-and-wait round trip per
+    // tile for 32 heads, and the accumulator goes back to the MMA one round trip earlier.
+    static constexpr int CHUNK = (NWG == 1 && COLS_WG % 32 == 0) ? 32 : 16;
     static constexpr int NCHUNK = COLS_WG / CHUNK;
     // warpgroup 0 holds the roles (warp 0 TMA, warp 1 MMA, warps 2-3 idle); warpgroups 1..NWG the
     // epilogue.  With four epilogue warpgroups the roles hand registers to the epilogue

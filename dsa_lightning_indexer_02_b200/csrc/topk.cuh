@@ -773,6 +773,10 @@ struct TopkClusterShared {
     int fixed;                        // needed from it, its size, low offset bits not yet fixed
     uint32_t cut_key;                 // last kept key of the boundary bin (broadcast)
     int cut_idx;
+    int above[kTkCluster][kTkWarps];  // keys above the boundary bin per (CTA, region) (CTA 0)
+    int bkept[kTkCluster * kTkWarps]; // kept boundary-bin members per (CTA, region) (CTA 0)
+    uint8_t borg[kTkBndMax];          // (CTA, region) of each boundary-bin member (CTA 0)
+    int lab[kTkWarps];                // this CTA's above-bin counts per region
     uint32_t lhist[kTkBins];          // this CTA's candidate histogram, added to CTA 0's after the stream
 };
 
@@ -880,7 +884,11 @@ __device__ __forceinline__ void cluster_select(TopkSmem& S, TopkClusterShared& C
         }
 
         // ---- distributed refinement: the bin holding the k-th key, narrowed while it is large
+        if (tid < kTkWarps) C.lab[tid] = 0;
         if (crank == 0) {
+            // the member list and its per-region tallies start empty (filled after this barrier)
+            if (tid == 0) C.bn = 0;
+            if (tid < kTkCluster * kTkWarps) C.bkept[tid] = 0;
             find_threshold_bin(S, G, kTkBins, (uint32_t)k);
             if (tid < kTkCluster) {
                 TopkClusterShared* D = cluster.map_shared_rank(&C, tid);
@@ -924,21 +932,37 @@ __device__ __forceinline__ void cluster_select(TopkSmem& S, TopkClusterShared& C
         const uint32_t pv = C.pv;
         auto in_bin = [&](uint32_t d) { return fixed >= 32 || (d >> fixed) == (pv >> fixed); };
         auto above = [&](uint32_t d) { return fixed < 32 && (d >> fixed) > (pv >> fixed); };
-        // ---- the boundary bin's members to CTA 0, which ranks them and broadcasts the cutoff
-        if (crank == 0 && tid == 0) C.bn = 0;
-        cluster.sync();
-        for (int w = 0; w < kTkWarps; ++w) {
-            const int cw = min(S.reg_gt[w], kTkRegion);
-            for (int e = tid; e < cw; e += kTkThreads) {
-                const uint32_t key = S.cand_key[w * kTkRegion + e];
-                if (in_bin(key - T0)) {
-                    const int p = atomicAdd(&C0->bn, 1);
-                    if (p < kTkBndMax) {
-                        C0->bkey[p] = key;
-                        C0->bidx[p] = S.cand_idx[w * kTkRegion + e];
+        // ---- the boundary bin's members (with their (CTA, region)) and every region's count of
+        // keys above the bin go to CTA 0, which ranks the members, and broadcasts the cutoff and
+        // each (CTA, region)'s kept count: the row offsets need no further exchange
+        {
+            uint32_t abv[kTkWarps];
+#pragma unroll
+            for (int w = 0; w < kTkWarps; ++w) {
+                abv[w] = 0;
+                const int cw = min(S.reg_gt[w], kTkRegion);
+                for (int e = tid; e < cw; e += kTkThreads) {
+                    const uint32_t key = S.cand_key[w * kTkRegion + e];
+                    abv[w] += above(key - T0) ? 1u : 0u;
+                    if (in_bin(key - T0)) {
+                        const int p = atomicAdd(&C0->bn, 1);
+                        if (p < kTkBndMax) {
+                            C0->bkey[p] = key;
+                            C0->bidx[p] = S.cand_idx[w * kTkRegion + e];
+                            C0->borg[p] = (uint8_t)(crank * kTkWarps + w);
+                        }
                     }
                 }
             }
+#pragma unroll
+            for (int w = 0; w < kTkWarps; ++w) {
+                uint32_t v = abv[w];
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+                if (lane == 0 && v) atomicAdd(&C.lab[w], (int)v);
+            }
+            __syncthreads();
+            if (tid < kTkWarps) C0->above[crank][tid] = C.lab[tid];
         }
         cluster.sync();
         if (crank == 0) {
@@ -952,12 +976,19 @@ __device__ __forceinline__ void cluster_select(TopkSmem& S, TopkClusterShared& C
                     const uint32_t kb = C.bkey[b];
                     rank += (kb > ka) || (kb == ka && C.bidx[b] < ia);
                 }
+                if (rank < need) atomicAdd(&C.bkept[C.borg[a]], 1);
                 if (rank == need - 1u)  // exactly one member: the last kept one
                     for (int q = 0; q < kTkCluster; ++q) {
                         TopkClusterShared* D = cluster.map_shared_rank(&C, q);
                         D->cut_key = ka;
                         D->cut_idx = ia;
                     }
+            }
+            __syncthreads();  // CTA 0 only (uniform branch): every member tallied
+            if (tid < kTkCluster * kTkWarps) {
+                const int q = tid / kTkWarps, w = tid % kTkWarps;
+                const int kq = C.above[q][w] + C.bkept[tid];
+                for (int r2 = 0; r2 < kTkCluster; ++r2) cluster.map_shared_rank(&C, r2)->kept[q][w] = kq;
             }
         }
         cluster.sync();
@@ -967,17 +998,7 @@ __device__ __forceinline__ void cluster_select(TopkSmem& S, TopkClusterShared& C
             const uint32_t d = key - T0;
             return above(d) || (in_bin(d) && (key > cut_key || (key == cut_key && ix <= cut_idx)));
         };
-        // ---- kept keys per region, exchanged; each CTA writes its own at the row's offsets
-        {
-            const int cw = min(S.reg_gt[warp], kTkRegion);
-            uint32_t cntk = 0;
-            for (int e = lane; e < cw; e += 32)
-                cntk += kept(S.cand_key[warp * kTkRegion + e], S.cand_idx[warp * kTkRegion + e]);
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) cntk += __shfl_xor_sync(0xffffffffu, cntk, o);
-            if (lane < kTkCluster) cluster.map_shared_rank(&C, lane)->kept[crank][warp] = (int)cntk;
-        }
-        cluster.sync();
+        // ---- each CTA writes its own kept keys at the row's offsets
         {
             uint32_t base = 0;
             for (int w = 0; w < warp; ++w)

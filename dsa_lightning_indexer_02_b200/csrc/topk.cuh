@@ -364,6 +364,103 @@ __device__ __forceinline__ uint32_t stream_collect(TopkSmem& S, const Grp& G, co
     return cnt;
 }
 
+// stream_collect for a segment staged in shared memory (src4[g - g_base]), 16 float4 per lane
+// per batch.  Candidates are sparse (a few per lane per batch), so instead of a predicated store
+// slot for every score, each lane walks the set bits of its 64-bit candidate mask and re-reads the
+// score from shared memory: the warp runs as many steps as its busiest lane has candidates.
+// Positions are the same as stream_collect's (float4 u first, then lane, then component), so the
+// regions hold the same candidates in the same order.
+__device__ __forceinline__ uint32_t stream_collect_staged(TopkSmem& S, const Grp& G, const float4* src4, int g_lo,
+                                                          int g_hi, int e_lo, int n, float F0, int region_base,
+                                                          int g_base) {
+    constexpr int UN = 16, kW = UN / 4;
+    const int g_first = g_lo;
+    const int lane = G.lane(), warp = G.warp();
+    const int lane_off = (lane >> 3) * 32 + warp * 8 + (lane & 7);
+    const int g_in_lo = max(g_first, (e_lo + 3) >> 2), g_in_hi = min(g_hi, n >> 2);
+    const float* src = reinterpret_cast<const float*>(src4);
+    uint32_t cnt = 0;
+    g_lo &= ~31;
+    constexpr int kStep = UN * 128;
+    for (int g0 = g_lo; g0 < g_hi; g0 += kStep) {
+        const bool interior = g0 >= g_in_lo && g0 + kStep <= g_in_hi;
+        unsigned long long mk = 0;  // 4-bit candidate mask of float4 u at bits 4u .. 4u+3
+        uint32_t c[kW];             // candidate count (0..4) of float4 u in byte u % 4 of word u / 4
+#pragma unroll
+        for (int w = 0; w < kW; ++w) c[w] = 0;
+#pragma unroll
+        for (int u = 0; u < UN; ++u) {
+            const int g = g0 + u * 128 + lane_off;
+            uint32_t mask = 0;
+            if (interior || g < g_hi) {
+                const float4 v = src4[g - g_base];
+                const float f[4] = {v.x, v.y, v.z, v.w};
+                if (interior) {
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) mask |= (f[j] >= F0 ? 1u : 0u) << j;
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        if (f[j] >= F0 && g * 4 + j < n && g * 4 + j >= e_lo && g >= g_first) mask |= 1u << j;
+                }
+            }
+            mk |= (unsigned long long)mask << (4 * u);
+            c[u >> 2] |= (uint32_t)__popc(mask) << (8 * (u & 3));
+        }
+        if (__ballot_sync(0xffffffffu, mk != 0ull) == 0) continue;
+        // exclusive scan over lanes of the packed counts, and the per-float4 totals
+        uint32_t sc[kW], t[kW];
+#pragma unroll
+        for (int w = 0; w < kW; ++w) sc[w] = c[w];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            uint32_t y[kW];
+#pragma unroll
+            for (int w = 0; w < kW; ++w) y[w] = __shfl_up_sync(0xffffffffu, sc[w], o);
+            if (lane >= o) {
+#pragma unroll
+                for (int w = 0; w < kW; ++w) sc[w] += y[w];
+            }
+        }
+#pragma unroll
+        for (int w = 0; w < kW; ++w) {
+            t[w] = __shfl_sync(0xffffffffu, sc[w], 31);
+            sc[w] -= c[w];
+        }
+        // lane u < UN: the candidates of float4s before u, over the whole warp (exclusive prefix)
+        const int lw = (lane >> 2) & (kW - 1);
+        const uint32_t tw = lw == 0 ? t[0] : lw == 1 ? t[1] : lw == 2 ? t[2] : t[3];
+        const uint32_t tot_l = lane < UN ? (tw >> (8 * (lane & 3))) & 0xFFu : 0u;
+        uint32_t incl = tot_l;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        const uint32_t pre_l = incl - tot_l;
+        const uint32_t batch_total = __shfl_sync(0xffffffffu, incl, UN - 1);
+        unsigned long long bits = mk;
+        const int trips = (int)__reduce_max_sync(0xffffffffu, (unsigned)__popcll(mk));
+        for (int it = 0; it < trips; ++it) {
+            const bool has = bits != 0ull;
+            const int b = has ? __ffsll((long long)bits) - 1 : 0;
+            bits &= bits - 1ull;
+            const int u = b >> 2, j = b & 3;
+            const uint32_t pre = __shfl_sync(0xffffffffu, pre_l, u);
+            const uint32_t sw = u < 8 ? (u < 4 ? sc[0] : sc[1]) : (u < 12 ? sc[2] : sc[3]);
+            const uint32_t mu = (uint32_t)(mk >> (4 * u)) & 0xFu;
+            const uint32_t pos = cnt + pre + ((sw >> (8 * (u & 3))) & 0xFFu) + __popc(mu & ((1u << j) - 1u));
+            if (has && pos < (uint32_t)kTkRegion) {
+                const int g = g0 + u * 128 + lane_off;
+                S.cand_key[region_base + pos] = score_key(src[(g - g_base) * 4 + j]);
+                S.cand_idx[region_base + pos] = g * 4 + j;
+            }
+        }
+        cnt += batch_total;
+    }
+    return cnt;
+}
+
 // Exact top-k among the candidates in S's regions (every candidate key >= lo; their total is
 // >= k and includes every key of the row >= lo).  Radix rounds over the key offsets narrow down
 // the bin holding the k-th key until it holds at most kTkSmallBin candidates (or one key value);
@@ -840,15 +937,13 @@ __device__ __forceinline__ void cluster_select(TopkSmem& S, TopkClusterShared& C
         const uint32_t T0 = C.T0, sh = C.sh;
 
         // ---- stream this CTA's segment into its warp regions (a staged segment in batches of
-        // 16 float4 per lane: half the scan chains of the 8-wide form, which at one warp per
-        // scheduler are latency-bound), then count the stored candidates into a local histogram
-        // (a pass over shared memory whose atomics overlap, instead of one inside the compaction
-        // loop) and add it to CTA 0's once (a remote atomic per candidate made the stream 4x
-        // slower)
+        // 16 float4 per lane, each lane walking only its own candidates), then count the stored
+        // candidates into a local histogram (a pass over shared memory whose atomics overlap,
+        // instead of one inside the compaction loop) and add it to CTA 0's once (a remote atomic
+        // per candidate made the stream 4x slower)
         for (int i = tid; i < kTkBins; i += kTkThreads) C.lhist[i] = 0u;
-        const uint32_t c = staged ? stream_collect<true, 2 * kTkUnroll, false>(S, G, src4, g_lo, g_hi, lo, n,
-                                                                            key_floor_float(T0), warp * kTkRegion,
-                                                                            g_base)
+        const uint32_t c = staged ? stream_collect_staged(S, G, src4, g_lo, g_hi, lo, n, key_floor_float(T0),
+                                                          warp * kTkRegion, g_base)
                                   : stream_collect<false, kTkUnroll, true>(S, G, src4, g_lo, g_hi, lo, n,
                                                                            key_floor_float(T0), warp * kTkRegion);
         if (lane == 0) S.reg_gt[warp] = (int)c;

@@ -765,8 +765,11 @@ __device__ __forceinline__ void take_samples(const Grp& G, uint32_t* keys, int b
     }
 }
 
+// Sampled float4 groups per part for n4 groups of competing keys: about n/32 scores (at least 1024,
+// at most 4096) in all.  (An earlier n4/8 rule sampled n/8 to n/16 of the shorter rows: 6 % slower
+// over a 128K sequence's chunks, no fewer misses.)
 __device__ __forceinline__ int sample_count4(int n4, int parts) {
-    return min(kTkMaxSample4, max(256, n4 / 8)) / parts;  // ~n/32 scores in all
+    return min(kTkMaxSample4, max(256, n4 / 32)) / parts;
 }
 
 // Second aim after a miss: the observed count c at rank rs scales about linearly with the rank.

@@ -99,6 +99,18 @@ __device__ __forceinline__ int indexer_unit_of(int round, int cta, int grid) {
     return round * grid + ((round & 1) ? (grid - 1 - cta) : cta);
 }
 
+// Decode (one query token per unit): a CTA's few work units, each with its sequence's context
+// length and the token's head weights (up to 64 bf16), read into shared memory once -- one
+// parallel round of global loads at the start instead of a dependent load (ctx_len, then the
+// weights) in every role at every unit boundary.
+constexpr int kIdxUnitTab = 8;  // rounds per CTA the table holds; more fall back to direct loads
+struct IndexerUnitEntry {
+    IndexerUnit U;
+    long long pos;  // ctx_len[U.p] as given (the append's row; checked before use)
+    int valid, pad;
+    uint4 w[8];     // the unit's token weights, raw bf16
+};
+
 template <int CHUNK>
 __device__ __forceinline__ void tmem_ld_chunk(uint32_t taddr, float (&v)[CHUNK]) {
     if constexpr (CHUNK == 32) tmem_ld_32x32b_x32(taddr, v);
@@ -209,7 +221,9 @@ struct IndexerCfg {
     static constexpr int OFF_BAR = OFF_B + 2 * B_BYTES;
     static constexpr int NBAR = 2 * STAGES + 8;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-    static constexpr int SMEM = OFF_MISC + 16 + 1024;  // + alignment slack
+    static constexpr bool UNIT_TAB = TB == 1;  // decode: the unit table in shared memory
+    static constexpr int OFF_UT = (OFF_MISC + 16 + 15) / 16 * 16;
+    static constexpr int SMEM = OFF_UT + (UNIT_TAB ? kIdxUnitTab * (int)sizeof(IndexerUnitEntry) : 0) + 1024;  // + alignment slack
     static_assert(BN % HI == 0 && BN >= 16 && BN <= 256 && BN % 16 == 0, "bad BN");
     static_assert(HI <= COLS_WG, "a token's heads must stay inside one warpgroup");
     static_assert(HI <= CHUNK || HI % CHUNK == 0, "bad HI");
@@ -235,6 +249,26 @@ __global__ void __launch_bounds__(IndexerCfg<HI, BN, STAGES>::THREADS, 1) indexe
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    IndexerUnitEntry* utab = reinterpret_cast<IndexerUnitEntry*>(smem + C::OFF_UT);
+    // uniform: the decode table covers every round of this CTA
+    const bool use_tab = C::UNIT_TAB && P.ctx_len && (P.num_units + (int)gridDim.x - 1) / (int)gridDim.x <= kIdxUnitTab;
+    if (use_tab) {
+        if (threadIdx.x < kIdxUnitTab) {
+            const int rd = threadIdx.x;
+            const int u = indexer_unit_of(rd, blockIdx.x, gridDim.x);
+            IndexerUnitEntry& E = utab[rd];
+            E.valid = u < P.num_units;
+            if (E.valid) {
+                E.U = indexer_unit<C::TB>(P, u);
+                E.pos = P.ctx_len[E.U.p];
+                const uint4* wsrc = reinterpret_cast<const uint4*>(P.w + (long long)E.U.p * P.Lq * HI);
+#pragma unroll
+                for (int i = 0; i < HI / 8; ++i) E.w[i] = __ldg(wsrc + i);
+            }
+        }
+        __syncthreads();
+    }
+    auto unit_at = [&](int rd, int u) { return use_tab ? utab[rd].U : indexer_unit<C::TB>(P, u); };
 
     if (P.new_kI) {
         // append each sequence's new token in the CTA that owns the key tile holding it, ahead of
@@ -242,8 +276,8 @@ __global__ void __launch_bounds__(IndexerCfg<HI, BN, STAGES>::THREADS, 1) indexe
         for (int rd = 0;; ++rd) {
             const int u = indexer_unit_of(rd, blockIdx.x, gridDim.x);
             if (u >= P.num_units) break;
-            const IndexerUnit U = indexer_unit<C::TB>(P, u);
-            const long long pos = P.ctx_len[U.p];
+            const IndexerUnit U = unit_at(rd, u);
+            const long long pos = use_tab ? utab[rd].pos : P.ctx_len[U.p];
             if (pos < 0 || pos >= P.Lk) {  // reported once per sequence; the sequence is not appended
                 if (U.kt0 == 0 && threadIdx.x == 0) record_error(DSA_DEV_ERR_BOUNDS, 0x501);
                 continue;
@@ -298,7 +332,7 @@ __global__ void __launch_bounds__(IndexerCfg<HI, BN, STAGES>::THREADS, 1) indexe
             for (int rd = 0; ok; ++rd) {
                 const int u = indexer_unit_of(rd, cta, grid);
                 if (u >= P.num_units) break;
-                const IndexerUnit U = indexer_unit<C::TB>(P, u);
+                const IndexerUnit U = unit_at(rd, u);
                 if (U.kt0 >= U.kt1) continue;
                 ok = wait_parity(&q_empty[qbuf], q_ph ^ 1, 0x101, abort_flag);
                 if (!ok) break;
@@ -331,7 +365,7 @@ __global__ void __launch_bounds__(IndexerCfg<HI, BN, STAGES>::THREADS, 1) indexe
             for (int rd = 0; ok; ++rd) {
                 const int u = indexer_unit_of(rd, cta, grid);
                 if (u >= P.num_units) break;
-                const IndexerUnit U = indexer_unit<C::TB>(P, u);
+                const IndexerUnit U = unit_at(rd, u);
                 if (U.kt0 >= U.kt1) continue;
                 ok = wait_parity(&q_full[qbuf], q_ph, 0x201, abort_flag);
                 if (!ok) break;
@@ -369,7 +403,7 @@ __global__ void __launch_bounds__(IndexerCfg<HI, BN, STAGES>::THREADS, 1) indexe
         for (int rd = 0;; ++rd) {
             const int u = indexer_unit_of(rd, cta, grid);
             if (u >= P.num_units) break;
-            const IndexerUnit U = indexer_unit<C::TB>(P, u);
+            const IndexerUnit U = unit_at(rd, u);
             if (U.kt0 >= U.kt1) continue;
             // This unit's weights for this warpgroup's columns (column c = token*HI + head), held in
             // registers for all of the unit's key tiles: columns [c, c+8) are 8 consecutive bf16 of
@@ -382,7 +416,7 @@ __global__ void __launch_bounds__(IndexerCfg<HI, BN, STAGES>::THREADS, 1) indexe
                 for (int cc = 0; cc < C::COLS_WG; cc += 8) {
                     const int c = wg * C::COLS_WG + cc;
                     if ((c + 7) / HI < U.rows) {
-                        const uint4 raw = __ldg(reinterpret_cast<const uint4*>(wu + c));
+                        const uint4 raw = use_tab ? utab[rd].w[c / 8] : __ldg(reinterpret_cast<const uint4*>(wu + c));
                         const uint32_t wv[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
                         for (int e = 0; e < 8; ++e) {

@@ -136,7 +136,17 @@ __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
 // bit for every finite x.  One pipe alone would issue one ReLU per MMA output element and cap
 // the epilogue at the tensor-core rate.
 __device__ __forceinline__ float2 relu_pair_alu(float a, float b) { return make_float2(fmaxf(a, 0.f), fmaxf(b, 0.f)); }
-__device__ __forceinline__ float2 relu2_pair_fma(float a, float b) { return make_float2(a + fabsf(a), b + fabsf(b)); }
+// x + |x| for a pair as one packed add (the absolute value rides on the operand; the same
+// per-element rounding as two scalar adds, half the instructions).
+__device__ __forceinline__ float2 relu2_pair_fma(float a, float b) {
+    uint64_t px, pa, pd;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(px) : "f"(a), "f"(b));
+    asm("mov.b64 %0, {%1, %2};" : "=l"(pa) : "f"(fabsf(a)), "f"(fabsf(b)));
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(pd) : "l"(px), "l"(pa));
+    float2 d;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(d.x), "=f"(d.y) : "l"(pd));
+    return d;
+}
 // Scale that the stored weight of head h carries (see above); heads come in groups of four only
 // when the head count is a multiple of four.
 template <int HI>

@@ -289,7 +289,7 @@ __device__ __forceinline__ uint32_t stream_collect(TopkSmem& S, const Grp& G, co
         for (int u = 0; u < UN; ++u) v[u] = vn[u];
         if (g0 + kStep < g_hi) load_batch(g0 + kStep);
         uint32_t mk = 0;              // 4-bit candidate mask of float4 u at bits 4u .. 4u+3
-        uint32_t c[2] = {0u, 0u};     // candidate count (0..4) of float4 u in byte u % 4 of word u / 4
+        uint32_t c[2];                // candidate count (0..4) of float4 u in byte u % 4 of word u / 4
 #pragma unroll
         for (int u = 0; u < UN; ++u) {
             const int g = g0 + u * 128 + lane_off;
@@ -304,9 +304,20 @@ __device__ __forceinline__ uint32_t stream_collect(TopkSmem& S, const Grp& G, co
                     if (f[j] >= F0 && g * 4 + j < n && g * 4 + j >= e_lo && g >= g_first) mask |= 1u << j;
             }
             mk |= mask << (4 * u);
-            c[u >> 2] |= (uint32_t)__popc(mask) << (8 * (u & 3));
         }
         if (__ballot_sync(0xffffffffu, mk != 0u) == 0) continue;
+        {
+            // the counts from the packed mask: nibble popcounts (0..4 each), then nibbles 0..3 and
+            // 4..7 spread into the bytes of c[0] and c[1] (fewer instructions than a popcount and
+            // a shift-or per float4)
+            uint32_t x = mk - ((mk >> 1) & 0x55555555u);
+            x = (x & 0x33333333u) + ((x >> 2) & 0x33333333u);
+            uint32_t y0 = x & 0xFFFFu, y1 = x >> 16;
+            y0 = (y0 | (y0 << 8)) & 0x00FF00FFu;
+            y1 = (y1 | (y1 << 8)) & 0x00FF00FFu;
+            c[0] = (y0 | (y0 << 4)) & 0x0F0F0F0Fu;
+            c[1] = (y1 | (y1 << 4)) & 0x0F0F0F0Fu;
+        }
         // inclusive scan over lanes of the packed counts (each prefix <= 128 fits its byte)
         uint32_t sc[2] = {c[0], c[1]};
 #pragma unroll

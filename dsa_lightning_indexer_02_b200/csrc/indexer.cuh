@@ -9,8 +9,8 @@
 // Tiling.  One MMA tile is D[128 keys, BN columns] = kI_tile[128 x 64] . Qtile[BN x 64]^T where
 // the BN columns are (token, head) pairs of TB = BN/HI consecutive query tokens.  The key tile
 // is the M operand, so every TMEM lane holds one key and the head sum for a token is a plain
-// in-thread reduction over that token's HI columns; the weights are a broadcast from shared
-// memory and consecutive lanes write consecutive keys (coalesced 128-byte score stores).
+// in-thread reduction over that token's HI columns; the token weights stay in registers for the
+// whole work unit and consecutive lanes write consecutive keys (coalesced 128-byte score stores).
 //
 // Roles (one CTA per SM, persistent):
 //   warp 0        TMA producer: the unit's Q tile (once per unit) and a ring of kI tiles

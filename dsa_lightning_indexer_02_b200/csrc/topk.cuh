@@ -11,9 +11,12 @@
 //   sample   ~n/32 scores at evenly spaced float4s give T0, an estimate of the key at rank
 //            1.5k (two histogram rounds over the sample keys, bins spanning the samples'
 //            own key range);
-//   stream   the row is read once; each warp takes every 4th 128-byte piece (so frames of
-//            correlated scores spread evenly over the warps) and compacts the scores >= T0 into
-//            its own shared-memory region, positions from warp ballots -- no block barrier per load;
+//   stream   the row is read once, 8 float4 per lane per batch with the next batch's loads in
+//            flight while the current one is filtered; each warp takes every 4th 128-byte piece
+//            (so frames of correlated scores spread evenly over the warps) and compacts the
+//            scores >= T0 into its own shared-memory region: one warp-wide scan of the lanes'
+//            packed per-float4 counts places every candidate, then each lane walks only its own
+//            candidate bits -- no block barrier per load;
 //   refine   if every region fits and the total is >= k, the candidates contain the exact
 //            top-k: radix rounds over the key offsets from T0 (first round scaled to the
 //            candidates' key range) narrow the bin that holds the k-th key until it is small, and
@@ -21,8 +24,9 @@
 //   emit     the kept keys are written region by region, each region in ascending key order.
 // If the candidates miss the window [k, capacity], the estimate is redone once, aimed using the
 // observed count, and the row streamed again.  Rows that still miss (or where more than 512
-// keys tie in the boundary bin) take an exact radix select over the row itself (10-bit rounds,
-// then one ordered pass): slower, and rare.
+// keys tie in the boundary bin) take an exact radix select over the row itself (10-bit rounds
+// with eight 16-byte loads in flight per thread, then one ordered pass per warp region): slower,
+// and rare.
 // Output order, the same on every path: when every competing key is kept, ascending; otherwise
 // grouped by region ((index / 32) mod 4, the pieces of one warp) and ascending within a region.
 // Sliding window (SW-DSA, page "DSA注意力机制：多模态学习中的强化推理新范式", showapi.com,

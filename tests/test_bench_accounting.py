@@ -58,3 +58,25 @@ def test_decode_step_bytes_at_16x128k():
     per_seq = ctx * 128 + 8 * ctx + 2048 * 2048 + 8 * 2048
     assert bench.decode_step_bytes(c, ctx) == pytest.approx(16 * per_seq)
     assert bench.decode_step_bytes(c, ctx) == pytest.approx(3.53e8, rel=5e-3)
+
+
+def test_source_hash_ignores_comments_only():
+    """profiles/traffic.json's counters are keyed by bench.lib_hash(): comment and blank-line edits
+    keep the key, any code edit changes it."""
+    code = "__global__ void k(int* p) {\n    p[0] = 1;  // store\n}\n"
+    commented = "// a kernel\n\n/* block\n   comment */\n__global__ void k(int* p) {\n    p[0] = 1;\n}\n"
+    changed = "__global__ void k(int* p) {\n    p[0] = 2;  // store\n}\n"
+    assert bench.source_code_only(code) == bench.source_code_only(commented)
+    assert bench.source_code_only(code) != bench.source_code_only(changed)
+
+
+def test_committed_traffic_matches_the_sources():
+    """The committed DRAM counters were taken on the kernel code now in csrc/ (else the bench would
+    report traffic null)."""
+    import json
+    import os
+    with open(os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "profiles",
+                           "traffic.json")) as f:
+        t = json.load(f)
+    for name in ("indexer", "topk", "sparse_attn"):
+        assert t[name]["lib_sha"] == bench.lib_hash(), name

@@ -562,7 +562,7 @@ def kernel_rooflines(prof: dict, work: dict, steps: int, peaks: dict, workload: 
                            "l2_gather_ceiling": {"value": L2_GATHER_GBS, "unit": "GB/s", "frac": logical / L2_GATHER_GBS,
                                                  "source": L2_GATHER_SOURCE}}
     # DRAM bytes per launch: ncu counters of a small case of the same kernel, scaled by the
-    # launch's algorithmic units, used only while the kernel sources are unchanged
+    # launch's algorithmic units, used only while the kernel code (comments aside) is unchanged
     tr = {}
     tpath = os.path.join(ROOT, "profiles", "traffic.json")
     if os.path.exists(tpath):

@@ -680,8 +680,11 @@ size_t dsa_workspace_size(int op, int64_t L, int B, int Hq, int HI, int topk) {
     case DSA_OP_TOPK:
     case DSA_OP_SPARSE_ATTN: return 0;
     case DSA_OP_PREFILL: {
+        // score rows of up to 16 GiB per chunk: fewer, longer chunks shorten every kernel's
+        // per-launch tail (128K: 1.32 M tokens/s at 8192-row chunks, 1.38 M at 16384 or 32768;
+        // 256K: 0.82 M at 4096, 0.86 M at 8192, 0.87 M at 16384)
         const int64_t ld = prefill_ld(L);
-        int64_t rows = (int64_t(4) << 30) / (ld * 4);
+        int64_t rows = (int64_t(16) << 30) / (ld * 4);
         rows = std::max<int64_t>(256, rows / 256 * 256);
         rows = std::min<int64_t>(rows, L);
         return align_up(chunk_bytes(rows, ld, topk), 256);

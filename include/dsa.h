@@ -241,9 +241,10 @@ size_t dsa_decode_noalloc_scratch_bytes(void);
 /*
  * Bytes of workspace an entry point needs.  op: DSA_OP_*.  L: sequence length (prefill) or cache
  * capacity Lmax (decode); B: sequences (decode); Hq: query heads; HI: indexer heads; topk.
- * DSA_OP_PREFILL returns the recommended size (score rows of up to 4 GiB per chunk plus index
- * rows); DSA_OP_INDEXER_KL the score rows alone (topk ignored); DSA_OP_INDEX/TOPK/SPARSE_ATTN
- * return 0.  Returns 0 for invalid arguments.
+ * DSA_OP_PREFILL returns the recommended size (score rows of up to 16 GiB per chunk plus index
+ * rows; a smaller workspace works too, in more and shorter chunks, somewhat slower);
+ * DSA_OP_INDEXER_KL the score rows alone, up to 4 GiB per chunk (topk ignored);
+ * DSA_OP_INDEX/TOPK/SPARSE_ATTN return 0.  Returns 0 for invalid arguments.
  */
 size_t dsa_workspace_size(int op, int64_t L, int B, int Hq, int HI, int topk);
 

@@ -25,8 +25,10 @@ def test_status_strings_and_version():
 
 
 def test_workspace_sizes():
-    # prefill at 128K: 8192 score rows of 131072 fp32 (4 GiB) + 8192 index rows of 2048 int32
-    assert dsa.workspace_size(dsa.DSA_OP_PREFILL, 131072, 1, 32, 32, 2048) == 8192 * 131072 * 4 + 8192 * 2048 * 4
+    # prefill at 128K: 32768 score rows of 131072 fp32 (16 GiB) + 32768 index rows of 2048 int32
+    assert dsa.workspace_size(dsa.DSA_OP_PREFILL, 131072, 1, 32, 32, 2048) == 32768 * 131072 * 4 + 32768 * 2048 * 4
+    # at 256K: 16384 score rows of 262144
+    assert dsa.workspace_size(dsa.DSA_OP_PREFILL, 262144, 1, 32, 32, 2048) == 16384 * 262144 * 4 + 16384 * 2048 * 4
     # small problems: one chunk covering the whole sequence
     assert dsa.workspace_size(dsa.DSA_OP_PREFILL, 1000, 1, 8, 4, 256) == 1000 * 1000 * 4 + 1024000
     assert dsa.workspace_size(dsa.DSA_OP_DECODE, 131328, 16, 32, 32, 2048) >= 16 * 131328 * 4

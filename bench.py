@@ -212,6 +212,9 @@ def main():
     ap.add_argument("--kl-rows", type=int, default=0,
                     help="query rows of the 32K workload for the KL measurement (default: all 32768)")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-blocks", default="8192",
+                    help="end-to-end leg's row blocks: a size, or 'size x count' items for the first rows "
+                         "then the last size repeated (e.g. 8192x8,16384)")
     ap.add_argument("--no-dedup", action="store_true", help="skip the adjacent-query dedup attention measurement")
     ap.add_argument("--dedup-only", action="store_true", help="only the dedup attention measurement (rank 0)")
     ap.add_argument("--dedup-rows", type=int, default=8192, help="query rows of the dedup measurement")
@@ -349,8 +352,8 @@ def main():
     if not args.no_e2e:
         hout = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
         hidx = torch.empty(idx.shape, dtype=idx.dtype, pin_memory=True)
-        R = 8192
-        blocks = [(r, min(hi, r + R)) for r in range(lo, hi, R)]
+        blocks = e2e_blocks(args.e2e_blocks, lo, hi)
+        R = max(r1 - r0 for r0, r1 in blocks)
         row_bytes = {n: host[n][0].numel() * host[n].element_size() for n in names}
         # this rank's query rows of q/qI/w, and K/V/kI of every position up to its last row
         h2d = sum(row_bytes[n] * (hi - lo) for n in ("q", "qI", "w")) + \
@@ -398,7 +401,8 @@ def main():
         ms_e2e = max_over_ranks(ev0.elapsed_time(ev1) / args.steps)
         e2e = {"value": (cfg.L if rows_mode else weak_scaling_value(cfg.L, world, 1.0)) / (ms_e2e / 1e3),
                "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e,
-               "how": f"dsa_prefill_rows over {len(blocks)} blocks of up to {R} rows; H2D, compute and D2H on "
+               "how": f"dsa_prefill_rows over {len(blocks)} blocks of up to {R} rows ({args.e2e_blocks}); H2D, "
+                      "compute and D2H on "
                       "three streams, pinned host buffers" +
                       ("; each rank copies in its own query rows and the key prefix they need, and copies "
                        "out its own output rows" if rows_mode else "")}
@@ -614,6 +618,26 @@ def run_profile_case(torch, dsa, cfg, spec: str) -> int:
     print(json.dumps({"profile_rows": [r0, n], "workload": cfg.name, "lib_sha": lib_hash(),
                       "units_per_launch": traffic_units(cfg, work), "unit_names": TRAFFIC_UNITS}), flush=True)
     return 0
+
+
+def e2e_blocks(spec: str, lo: int, hi: int) -> list:
+    """Row blocks [r0, r1) covering [lo, hi) for the end-to-end leg.  spec: comma-separated items
+    'size' or 'size x count'; the items are used in order and the last size repeats."""
+    items = []
+    for it in spec.split(","):
+        size, _, count = it.strip().partition("x")
+        items.append((int(size), int(count) if count else None))
+    blocks, r, i = [], lo, 0
+    while r < hi:
+        size, count = items[min(i, len(items) - 1)]
+        n = count if (count and i < len(items)) else 1
+        for _ in range(n):
+            if r >= hi:
+                break
+            blocks.append((r, min(hi, r + size)))
+            r = blocks[-1][1]
+        i += 1
+    return blocks
 
 
 def source_code_only(text: str) -> str:

@@ -80,3 +80,14 @@ def test_committed_traffic_matches_the_sources():
         t = json.load(f)
     for name in ("indexer", "topk", "sparse_attn"):
         assert t[name]["lib_sha"] == bench.lib_hash(), name
+
+
+@pytest.mark.parametrize("spec", ["ramp", "8192", "8192x8,16384", "4096x4,8192x4,16384x4,8192"])
+@pytest.mark.parametrize("lo,hi", [(0, 131072), (0, 262144), (0, 32768), (0, 1000), (65536, 131072), (5, 50000)])
+def test_e2e_blocks_partition_the_rows(spec, lo, hi):
+    """The end-to-end leg's blocks cover [lo, hi) exactly, in order, without gaps or overlap, so its
+    copies and timing count every row once."""
+    b = bench.e2e_blocks(spec, lo, hi)
+    assert b[0][0] == lo and b[-1][1] == hi
+    assert all(b[i][1] == b[i + 1][0] for i in range(len(b) - 1))
+    assert all(r1 > r0 for r0, r1 in b)
